@@ -1,0 +1,358 @@
+"""Benchmark of the svdq_w4a4 linear layer on B200.
+
+One step = one pass of the whole layer hot path (activation quantizer, then the
+W4A4 GEMM with its low-rank/bias epilogue) over the FLUX 1024x1024 MLP pair at
+4608 tokens: up-projection 3072 -> 12288 and down-projection 12288 -> 3072,
+NVFP4, rank 32, through the C ABI.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU runs are independent replicas (the layer has no exchange step), one
+process per GPU, timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "svdq_w4a4 linear TOPS (2*M*N*K per layer) at FLUX shapes"
+UNIT = "TOPS"
+WORKLOAD = "c4_mlp_4608x3072x12288_r32"
+LAYERS = [l for l in wl.WORKLOADS[WORKLOAD] if l.fmt == wl.NVFP4]
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _traffic():
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        return json.load(open(p))
+    return {}
+
+
+def _layer_flops(l):
+    return 2.0 * l.M * l.N * l.K
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample(prepared, xs, rows: int):
+    """Time the oracle (as it stands) on `rows` token rows of each layer."""
+    import oracle
+
+    t0 = time.perf_counter()
+    flops = 0.0
+    for l, prep, X in zip(LAYERS, prepared, xs):
+        act = oracle.quantize_act(X[:rows], prep)
+        oracle.forward_from_act(act, prep)
+        flops += 2.0 * rows * l.N * l.K
+    return flops, time.perf_counter() - t0
+
+
+def _oracle_prep(canon):
+    return dict(N=canon["N"], K=canon["K"], rank=canon["rank"], fmt=canon["fmt"], inv_lambda=canon["inv_lambda"],
+                L1=canon["L1"], L2=canon["L2"], wcodes=canon["wcodes"], wscales=canon["wscales"],
+                bias=canon["bias"], g_x=canon["g_x"], g_w=canon["g_w"])
+
+
+def cpu_baseline(canons, xs, target_s=15.0):
+    import oracle
+
+    preps = [_oracle_prep(c) for c in canons]
+    rows = 2
+    flops, dt = oracle_sample(preps, xs, rows)
+    rows = int(max(2, min(512, rows * target_s / max(dt, 1e-3))))
+    flops, dt = oracle_sample(preps, xs, rows)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{rows} token rows of each MLP layer (up {LAYERS[0].K}->{LAYERS[0].N}, "
+                      f"down {LAYERS[1].K}->{LAYERS[1].N}), NVFP4 r32, quantize + W4A4 product + output, "
+                      f"{dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- setup
+def _prepare_layers(seed=0):
+    """Product-side preparation (C ABI svdq_prepare on the host) of both layers."""
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    canons, xs = [], []
+    for l in LAYERS:
+        X, W, b = wl.make_layer_inputs(l, seed)
+        amax = np.abs(wl.bf16_bits_to_f32(X)).max(axis=0).astype(np.float32)
+        canons.append(svdq.svdq_prepare(W, b, amax, 0.5, l.rank, l.fmt))
+        xs.append(X)
+    return canons, xs
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    canons, xs = _prepare_layers()
+    import oracle
+
+    preps = [_oracle_prep(c) for c in canons]
+    rows = 4
+    for _ in range(args.warmup):
+        oracle_sample(preps, xs, rows)
+    tot_f, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, t = oracle_sample(preps, xs, rows)
+        tot_f += f
+        tot_t += t
+    val = tot_f / tot_t / 1e12
+    sample = f"{rows} token rows of each MLP layer per step (full layer is {LAYERS[0].M} rows)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD + "_nvfp4", "sample": sample},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    st = svdq.svdq_device_check(local)
+    if st != svdq.SVDQ_OK:
+        raise SystemExit(svdq.svdq_status_string(st))
+    canons, xs = _prepare_layers()
+    lins = [svdq.SvdqLinear(c, device=dev) for c in canons]
+    xd = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in xs]
+    ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in LAYERS]
+    wss = [lin.workspace(l.M) for lin, l in zip(lins, LAYERS)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    def step(ev=None):
+        for i, (lin, l) in enumerate(zip(lins, LAYERS)):
+            if ev is not None:
+                ev[2 * i].record(stream)
+            svdq.svdq_quantize_act(lin.handle, xd[i], l.M, wss[i], sp)
+            if ev is not None:
+                ev[2 * i + 1].record(stream)
+            svdq.svdq_gemm(lin.handle, l.M, ys[i], wss[i], sp)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    for lin, l in zip(lins, LAYERS):
+        assert lin.status(l.M) == 0, "kernel reported an error during warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.zero_()  # L2 flush between timed steps (outside the events)
+            step(evs[k])
+        torch.cuda.synchronize()
+    _barrier(world)
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    q_ms = [e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in evs]
+    g_ms = [e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) for e in evs]
+    g_up = [e[1].elapsed_time(e[2]) for e in evs]
+    g_dn = [e[3].elapsed_time(e[4]) for e in evs]
+    total_ms = _max_over_ranks(sum(step_ms), world)
+    for lin, l in zip(lins, LAYERS):
+        assert lin.status(l.M) == 0, "kernel reported an error during timing"
+
+    flops_step = sum(_layer_flops(l) for l in LAYERS)
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (the NVFP4 GEMM), tensor-bound
+    hbm, bf16, bf16_sus, src = _peaks()
+    fp4_peak = bf16 * 4.0  # measured bf16 dense x nominal fp4:bf16 ratio (9 / 2.25)
+    g_avg_ms = statistics.mean(g_ms) / 2
+    achieved = flops_step / 2 / (g_avg_ms * 1e-3) / 1e12
+    traffic = _traffic().get("gemm_nvfp4")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak, "traffic": traffic,
+                "peak_source": f"{src} bf16 {bf16} TFLOP/s (burst) x 4 (nominal fp4/bf16)",
+                "kernel": "k_gemm_nvfp4", "flops_per_launch": flops_step / 2}
+    # the activation quantizer is HBM-bound: algorithmic bytes per launch
+    qbytes = 0.0
+    for l in LAYERS:
+        qbytes += 2 * l.M * l.K + l.M * l.K / 2 + l.M * l.K / 16 + 2 * l.M * l.rank + 2 * l.K * l.rank + 4 * l.K
+    q_avg_ms = statistics.mean(q_ms)
+    quant = {"bound": "hbm", "achieved": qbytes / (q_avg_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+             "frac": qbytes / (q_avg_ms * 1e-3) / 1e9 / hbm, "bytes_per_step": qbytes, "kernel": "k_quantize"}
+
+    # end to end through the C ABI with host buffers: H2D of X, forward, D2H of Y
+    xh = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs]
+    yh = [torch.empty(l.M, l.N, dtype=torch.bfloat16).pin_memory() for l in LAYERS]
+    e2e_steps = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        for i, (lin, l) in enumerate(zip(lins, LAYERS)):
+            xd[i].copy_(xh[i], non_blocking=True)
+            svdq.svdq_forward(lin.handle, xd[i], l.M, ys[i], wss[i], sp)
+            yh[i].copy_(ys[i], non_blocking=True)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for i, (lin, l) in enumerate(zip(lins, LAYERS)):
+            xd[i].copy_(xh[i], non_blocking=True)
+            svdq.svdq_forward(lin.handle, xd[i], l.M, ys[i], wss[i], sp)
+            yh[i].copy_(ys[i], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = sum(2 * l.M * l.K for l in LAYERS)
+    d2h = sum(2 * l.M * l.N for l in LAYERS)
+    e2e = {"value": world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales) + bf16 low-rank, f32 accumulate", "data": "synthetic",
+        "config": {"workload": WORKLOAD + "_nvfp4", "layers": [f"{l.M}x{l.K}->{l.N}" for l in LAYERS],
+                   "rank": LAYERS[0].rank, "l2": "flushed between steps (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roofline, "quantize_roofline": quant,
+        "per_layer_us": {"gemm_up": statistics.median(g_up) * 1e3, "gemm_down": statistics.median(g_dn) * 1e3,
+                         "quantize_both": statistics.median(q_ms) * 1e3,
+                         "step_p10_p50_p90": [float(np.percentile(step_ms, p)) * 1e3 for p in (10, 50, 90)]},
+        "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(canons, xs)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    del lins
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = _dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,319 @@
+// K2: NVFP4 W4A4 GEMM of the svdq_w4a4 layer on 5th-generation tensor cores,
+// with the low-rank up-projection and the output epilogue fused in.
+//
+//   Y = g_x g_w * [ sum_blocks (s_x s_w) (qx . qw)  +  t . (L2 / (g_x g_w)) ] + b
+//
+// "Суть метода" ("Hugging Face встроила Nunchaku в Diffusers ..."): the 4-bit
+// product of quantized activations and quantized residual weights, plus the
+// 16-bit low-rank branch, plus the bias.  Because both per-tensor scales are
+// powers of two, L2 / (g_x g_w) is exact in bf16 and the low-rank product can
+// accumulate into the same fp32 tensor-memory accumulator as the block-scaled
+// 4-bit product; the epilogue then only applies the exact power-of-two scale,
+// adds the bias and rounds to bf16.
+//
+// Persistent, warp-specialized CTA (one per SM), tile 128 x 192:
+//   warp 0      TMA producer: per stage a 128x256 activation-code tile and a
+//               192x256 weight-code tile (128-byte swizzle), plus the matching
+//               E4M3 scale-factor atoms with bulk copies; the t / L2^T chunks of
+//               the low-rank branch ride the same ring first.
+//   warp 1      owns tensor memory (512 columns: two 192-column fp32
+//               accumulators for ping-pong with the epilogue, scale factors);
+//               one lane copies the scale factors into tensor memory
+//               (tcgen05.cp) and issues tcgen05.mma kind::f16 (low rank, K=16)
+//               and kind::mxf4nvf4 block16 (K=64) into the accumulator.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, scale, bias,
+//               bf16 round-to-nearest-even, 16-byte stores.
+// Every wait is bounded (see sm100.cuh); no load uses cluster multicast.
+#include <cuda_bf16.h>
+
+#include <cstring>
+
+#include "sm100.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+namespace {
+
+constexpr int BM = kGemmBM;   // 128
+constexpr int BN = kNvfp4BN;  // 192
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * 128;  // 256 fp4 per row
+constexpr int B_BYTES = BN * 128;
+constexpr int SFA_BYTES = 4 * kSfAtomBytes;      // 4 k-atoms x 128 rows
+constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;  // 4 k-atoms x 256 rows (192 used)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SFA_COL = 2 * BN;       // 384
+constexpr uint32_t SFB_COL = 2 * BN + 16;  // 400
+constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(BM, BN);
+constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(SFB_COL + 32 <= TMEM_COLS, "tensor memory budget");
+
+struct GemmMaps {
+  CUtensorMap a, b, t[3], l2[3];
+};
+
+struct GParams {
+  int M, N, K, m_tiles, n_tiles, num_tiles, k_stages, katoms;
+  int n_lr;
+  int lr_off[4], lr_w[4];
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* bias;
+  uint16_t* Y;
+  float out_scale;
+  int* status;
+  unsigned long long limit;
+};
+
+__device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
+
+__global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant__ GemmMaps maps, const GParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* mma_done = acc_empty + 2;   // [1]
+  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  WaitCtl wc{abort_flag, p.status, p.limit};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int units = p.n_lr + p.k_stages;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&maps.a);
+      prefetch_tmap(&maps.b);
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        for (int u = 0; u < units; ++u, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * STAGE_BYTES;
+          if (u < p.n_lr) {
+            const int w = p.lr_w[u], mi = lr_map_index(w);
+            mbar_arrive_expect_tx(&full[s], (uint32_t)(BM + BN) * 2 * w);
+            tma_load_2d(&maps.t[mi], &full[s], st, p.lr_off[u], mt * BM);
+            tma_load_2d(&maps.l2[mi], &full[s], st + A_BYTES, p.lr_off[u], nt * BN);
+          } else {
+            const int ks = u - p.n_lr;
+            mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+            tma_load_2d(&maps.a, &full[s], st, ks * 128, mt * BM);
+            tma_load_2d(&maps.b, &full[s], st + A_BYTES, ks * 128, nt * BN);
+            bulk_load(st + A_BYTES + B_BYTES, p.sfa + ((size_t)mt * p.katoms + 4 * ks) * kSfAtomBytes, SFA_BYTES,
+                      &full[s]);
+            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES,
+                      p.sfb + ((size_t)nt * p.katoms + 4 * ks) * 2 * kSfAtomBytes, SFB_BYTES, &full[s]);
+          }
+        }
+      }
+      if (!ok) {  // drain the copies still in flight
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, p.limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++local) {
+        const int b = local & 1;
+        if (!mbar_wait(&acc_empty[b], ((local >> 1) & 1) ^ 1, wc)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * BN);
+        uint32_t accum = 0;
+        for (int u = 0; u < units; ++u, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
+          if (u < p.n_lr) {
+            const int w = p.lr_w[u];
+            const uint32_t layout = w == 64 ? LAYOUT_SW128 : (w == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
+            const uint32_t sbo = 8u * 2u * (uint32_t)w;  // 8 rows of w bf16
+            for (int kk = 0; kk < w / 16; ++kk) {
+              mma_bf16(d, make_sdesc(a_addr + 32 * kk, 16, sbo, layout), make_sdesc(b_addr + 32 * kk, 16, sbo, layout),
+                       IDESC_BF16, accum);
+              accum = 1;
+            }
+          } else {
+            const uint32_t sfa_s = b_addr + B_BYTES;
+            const uint32_t sfb_s = sfa_s + SFA_BYTES;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tmem_cp_32x128b_x4(tmem + SFA_COL + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * j, make_sdesc(sfb_s + j * 2 * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * j + 4,
+                                 make_sdesc(sfb_s + j * 2 * kSfAtomBytes + kSfAtomBytes, 0, 128, LAYOUT_NONE));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              mma_nvf4(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
+                       make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), IDESC_NVF4, tmem + SFA_COL + 4 * j,
+                       tmem + SFB_COL + 8 * j, accum);
+              accum = 1;
+            }
+          }
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&acc_full[b]);
+      }
+      umma_commit(mma_done);  // every MMA issued above has completed when this fires
+      mbar_wait_drain(mma_done, 0, p.limit);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+    const int row = 32 * q + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+      const int b = local & 1;
+      if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) break;
+      tc_fence_after();
+      const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+      const int m = mt * BM + row;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tbase + 32 * c, r);
+        tmem_ld_wait();
+        if (c == BN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[b]);
+        }
+        const int n0 = nt * BN + 32 * c;
+        if (m < p.M) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int n = n0 + 8 * j;
+            if (n < p.N) {
+              const float4 b0 = __ldg((const float4*)(p.bias + n));
+              const float4 b1 = __ldg((const float4*)(p.bias + n + 4));
+              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              uint32_t o[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float y0 = fmaf(__uint_as_float(r[8 * j + 2 * e]), p.out_scale, bb[2 * e]);
+                const float y1 = fmaf(__uint_as_float(r[8 * j + 2 * e + 1]), p.out_scale, bb[2 * e + 1]);
+                __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+                o[e] = *(uint32_t*)&h;
+              }
+              *(uint4*)(p.Y + (size_t)m * p.N + n) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+int sm_count(int dev) {
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace
+
+int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w, cudaStream_t stream) {
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int K = (int)L->K, N = (int)L->N, r = L->rank;
+  int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
+                          (uint64_t)K / 2, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SVDQ_OK) return st;
+  maps.b = L->map_w;
+  GParams p{};
+  const LowRankChunks ch = lowrank_chunks(r);
+  p.n_lr = ch.n;
+  for (int i = 0; i < ch.n; ++i) {
+    p.lr_off[i] = ch.off[i];
+    p.lr_w[i] = ch.width[i];
+  }
+  if (r > 0) {
+    const int widths[3] = {64, 32, 16};
+    const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_64B,
+                                       CU_TENSOR_MAP_SWIZZLE_32B};
+    for (int i = 0; i < 3; ++i) {
+      if (widths[i] > r) continue;
+      st = encode_tmap_2d(&maps.t[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.t, (uint64_t)r, (uint64_t)M,
+                          (uint64_t)r * 2, widths[i], BM, swz[i]);
+      if (st != SVDQ_OK) return st;
+      maps.l2[i] = L->map_l2[i];
+    }
+  }
+  p.M = (int)M;
+  p.N = N;
+  p.K = K;
+  p.m_tiles = (int)((M + BM - 1) / BM);
+  p.n_tiles = (N + BN - 1) / BN;
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.k_stages = K / kKStage;
+  p.katoms = K / 64;
+  p.sfa = ws + w.scales;
+  p.sfb = L->wscales;
+  p.bias = L->bias;
+  p.Y = (uint16_t*)Y;
+  p.out_scale = L->g_x * L->g_w;
+  p.status = (int*)(ws + w.status);
+  p.limit = wait_limit_cycles();
+  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+  if (cudaFuncSetAttribute(k_gemm_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  const int grid = p.num_tiles < sm_count(L->device) ? p.num_tiles : sm_count(L->device);
+  k_gemm_nvfp4<<<grid, THREADS, smem, stream>>>(maps, p);
+  return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+}  // namespace svdq

@@ -1,0 +1,103 @@
+// Internal declarations shared by the host half and the kernels of libsvdq.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/svdq.h"
+
+namespace svdq {
+
+// Tile geometry of the kernels (compile-time contract between pack, the
+// activation quantizer and the GEMMs).
+constexpr int kKStage = 256;       // K elements per pipeline stage / per quantizer chunk
+constexpr int kGemmBM = 128;       // GEMM tile rows (tokens), = tcgen05 M
+constexpr int kNvfp4BN = 192;      // NVFP4 GEMM tile columns (output features)
+constexpr int kInt4BN = 128;       // INT4 GEMM tile columns
+constexpr int kSfAtomRows = 128;   // rows per tensor-core scale-factor atom
+constexpr int kSfAtomBytes = 512;  // 128 rows x 4 blocks of 16
+constexpr int kMaxRank = 128;
+constexpr size_t kAlign = 1024;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Byte offset of the E4M3 scale of (row, block) in a scale-factor atom tiling
+// whose row tiles are `tile_rows` rows (128 for activations, 192 for weights)
+// and each tile is padded to a multiple of 128 rows:
+//   tile t = row / tile_rows, atom a = (row % tile_rows) / 128 inside the tile,
+//   k-atom = block / 4, within the atom: (row%32)*16 + ((row/32)%4)*4 + block%4.
+inline __host__ __device__ size_t sf_offset(int64_t row, int64_t block, int64_t katoms, int tile_rows) {
+  const int64_t tile = row / tile_rows;
+  const int64_t rin = row % tile_rows;
+  const int atoms_per_tile = (tile_rows + kSfAtomRows - 1) / kSfAtomRows;
+  const int64_t a = rin / kSfAtomRows;
+  const int64_t ra = rin % kSfAtomRows;
+  return (size_t)(((tile * katoms + block / 4) * atoms_per_tile + a) * kSfAtomBytes + (ra % 32) * 16 +
+                  ((ra / 32) % 4) * 4 + (block % 4));
+}
+
+struct Blob {  // offsets (bytes) of the packed-weight regions
+  size_t inv_lambda, L1t, L2t, bias, wcodes, wscales, total;
+};
+Blob blob_layout(int64_t N, int64_t K, int rank, int fmt);
+
+struct Workspace {
+  size_t codes, scales, t, status, total;
+  size_t codes_bytes, scales_bytes, t_bytes;
+};
+Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M);
+
+struct LowRankChunks {
+  int n;
+  int off[4];
+  int width[4];  // 64, 32 or 16 bf16 columns
+};
+LowRankChunks lowrank_chunks(int rank);
+
+}  // namespace svdq
+
+// The opaque layer handle.
+struct svdq_layer {
+  int64_t N, K;
+  int rank, fmt;
+  float g_x, g_w;
+  int device;
+  const uint8_t* blob;
+  svdq::Blob off;
+  const float* inv_lambda;
+  const uint16_t* L1t;  // [rank, K]
+  const uint16_t* L2t;  // [N, rank]
+  const float* bias;    // [N]
+  const uint8_t* wcodes;
+  const uint8_t* wscales;
+  CUtensorMap map_w;         // weight codes
+  CUtensorMap map_l1;        // L1^T, box {64, rank}, 128B swizzle (quantizer)
+  CUtensorMap map_l2[3];     // L2^T chunks of width 64/32/16
+};
+
+namespace svdq {
+
+namespace host {
+int prepare(const uint16_t* W, const uint16_t* bias, const float* act_absmax, float alpha, svdq_canonical* c);
+uint16_t f32_to_bf16(float f);
+float bf16_to_f32(uint16_t h);
+}  // namespace host
+
+// Tensor-map encoding through the driver entry point (no link-time libcuda).
+int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+unsigned long long wait_limit_cycles();
+
+// Kernel launchers (return svdq_status).
+int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
+                    cudaStream_t stream);
+int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w,
+                      cudaStream_t stream);
+int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w, int32_t* acc_dbg,
+                     cudaStream_t stream);
+
+}  // namespace svdq

