@@ -272,9 +272,12 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   L->wcodes = L->blob + b.wcodes;
   L->wscales = L->blob + b.wscales;
   int e = SVDQ_OK;
-  if (fmt == SVDQ_NVFP4_G16)
+  if (fmt == SVDQ_NVFP4_G16)  // 256 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
                        (uint64_t)K / 2, 128, kNvfp4BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  else  // 128 packed codes (64 B) per row per stage, widened to int8 in shared memory
+    e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
+                       (uint64_t)K / 2, 64, kInt4BN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (e == SVDQ_OK && rank > 0) {
     e = encode_tmap_2d(&L->map_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L1t, (uint64_t)K, (uint64_t)rank,
                        (uint64_t)K * 2, 64, (uint32_t)rank, CU_TENSOR_MAP_SWIZZLE_128B);

@@ -12,10 +12,17 @@ import numpy as np
 import oracle
 import workloads as wl
 
-# Output tolerance on bf16 Y: the stated rel-L2 <= 1e-3 and max-abs 2e-2,
-# widened elementwise by one bf16 ulp of the oracle value, because two
-# correct fp32 accumulations in different orders round to neighbouring bf16
-# values once |y| >= 2 (ulp >= 2^-6 > ... and 2^-3 at |y| ~ 16).
+# Tolerances.
+# t: the oracle sums bf16(x^) L1 exactly (binary64) and rounds once to bf16; the
+#    GPU sums in fp32 in tensor-core order.  Any fp32 summation order of K terms
+#    is within gamma_K * sum|terms| of the exact sum (gamma_K ~ K u, u = 2^-24;
+#    taken as K 2^-23 to cover truncating accumulators), plus one bf16 ulp of
+#    the final rounding.
+# Y: the stated gates rel-L2 <= 1e-3 and max-abs 2e-2.  Elementwise, 2e-2 is
+#    widened by one bf16 ulp of the oracle value (two correct accumulation
+#    orders round to neighbouring bf16 values once |y| >= 4) and by the forward
+#    error of the fp32 arithmetic: the t bound carried through L2, and the fp32
+#    accumulation bound of the main product.
 REL_L2 = 1e-3
 MAX_ABS = 2e-2
 
@@ -30,28 +37,59 @@ def bf16_ulp(x):
     return np.ldexp(1.0, (e - 7).astype(np.int64))
 
 
-def y_stats(y_gpu_bits, y_orc_bits):
+def t_sum_bound(act: dict, prep: dict):
+    """fp32 summation bound of t = bf16(x^) L1, per element [M, r]."""
+    K = prep["K"]
+    if not prep["rank"]:
+        return np.zeros((act["xhat"].shape[0], 0))
+    S = np.abs(bf(oracle.f32_to_bf16(act["xhat"]))) @ np.abs(bf(prep["L1"]))
+    return K * 2.0**-23 * S
+
+
+def y_error_bound(act: dict, prep: dict):
+    """Forward-error allowance of y (beyond the final bf16 rounding) for the rows of `act`."""
+    K = prep["K"]
+    fmt = prep["fmt"]
+    gx = prep["g_x"] if fmt == oracle.NVFP4 else 1.0
+    gw = prep["g_w"] if fmt == oracle.NVFP4 else 1.0
+    dqx = np.abs(oracle.dequant(act["codes"], act["scales"], fmt, gx))
+    dqw = np.abs(oracle.dequant(prep["wcodes"], prep["wscales"], fmt, gw))
+    bound = (K + prep["rank"]) * 2.0**-23 * (dqx @ dqw.T)
+    if prep["rank"]:
+        t = bf(act["t"])
+        dt = bf16_ulp(t) + t_sum_bound(act, prep)
+        L2 = np.abs(bf(prep["L2"]))
+        bound += dt @ L2 + (K + prep["rank"]) * 2.0**-23 * (np.abs(t) @ L2)
+    return bound
+
+
+def y_stats(y_gpu_bits, y_orc_bits, extra=None):
     g, o = bf(y_gpu_bits), bf(y_orc_bits)
     d = np.abs(g - o)
+    lim = MAX_ABS + bf16_ulp(o) + (0.0 if extra is None else extra)
     return dict(rel_l2=float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30)), max_abs=float(d.max()),
-                n_over_abs=int(np.sum(d > MAX_ABS)), n_flip=int(np.sum(g != o)),
-                worst_excess=float(np.max(d - (MAX_ABS + bf16_ulp(o)))), nonfinite=int(np.sum(~np.isfinite(g))))
+                n_over_abs=int(np.sum(d > MAX_ABS)), n_over_abs_ulp=int(np.sum(d > MAX_ABS + bf16_ulp(o))),
+                n_flip=int(np.sum(g != o)), worst_excess=float(np.max(d - lim)),
+                nonfinite=int(np.sum(~np.isfinite(g))))
 
 
-def assert_y_close(y_gpu_bits, y_orc_bits):
-    s = y_stats(y_gpu_bits, y_orc_bits)
+def assert_y_close(y_gpu_bits, y_orc_bits, act=None, prep=None):
+    extra = y_error_bound(act, prep) if act is not None else None
+    s = y_stats(y_gpu_bits, y_orc_bits, extra)
     assert s["nonfinite"] == 0, s
     assert s["rel_l2"] <= REL_L2, s
     assert s["worst_excess"] <= 0.0, s
     return s
 
 
-def assert_t_close(t_gpu, t_orc):
+def assert_t_close(t_gpu, t_orc, act=None, prep=None):
     g, o = bf(t_gpu), bf(t_orc)
     lim = bf16_ulp(np.maximum(np.abs(g), np.abs(o)))
+    if act is not None:
+        lim = lim + t_sum_bound(act, prep)
     bad = np.abs(g - o) > lim
     assert not bad.any(), (int(bad.sum()), float(np.abs(g - o).max()))
-    return float(np.mean(g != o))
+    return dict(t_flip_frac=float(np.mean(g != o)), t_max_abs=float(np.abs(g - o).max()) if g.size else 0.0)
 
 
 @functools.lru_cache(maxsize=16)

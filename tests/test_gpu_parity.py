@@ -33,7 +33,7 @@ def _check_act(gl, X, prep):
     np.testing.assert_array_equal(got["codes"], ref["codes"])
     np.testing.assert_array_equal(got["scales"], ref["scales"])
     if prep["rank"]:
-        assert_t_close(got["t"], ref["t"])
+        assert_t_close(got["t"], ref["t"], ref, prep)
     return ref
 
 
@@ -55,8 +55,8 @@ def test_forward_nvfp4(M, K, N, rank):
     gl = GpuLayer(prep)
     y = gl.forward(X)
     assert gl.status(M) == 0
-    ref = oracle.forward(X, prep)
-    assert_y_close(y, ref)
+    act = oracle.quantize_act(X, prep)
+    assert_y_close(y, oracle.forward_from_act(act, prep), act, prep)
 
 
 def test_forward_empty_and_reuse():
@@ -87,13 +87,13 @@ def test_flux_workloads_nvfp4(name):
     ref = oracle.quantize_act(X, prep)
     np.testing.assert_array_equal(got["codes"], ref["codes"])
     np.testing.assert_array_equal(got["scales"], ref["scales"])
-    assert_t_close(got["t"], ref["t"])
+    st = assert_t_close(got["t"], ref["t"], ref, prep)
     # sampled output rows: first/last tile rows and a seeded spread
     rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], np.random.default_rng(1).choice(M, 40, replace=False)]))
     sub = {k: v[rows] for k, v in ref.items()}
     y_ref = oracle.forward_from_act(sub, prep)
-    s = assert_y_close(y[rows], y_ref)
-    print(name, s)
+    s = assert_y_close(y[rows], y_ref, sub, prep)
+    print(name, s, st)
 
 
 def test_wait_timeout_reports_status():
@@ -117,4 +117,57 @@ def test_wait_timeout_reports_status():
     svdq.svdq_workspace_init(gl.lin.handle, 512, gl.lin.workspace(512))
     y = gl.forward(X)
     assert gl.status(512) == 0
-    assert_y_close(y, oracle.forward(X, prep))
+    act = oracle.quantize_act(X, prep)
+    assert_y_close(y, oracle.forward_from_act(act, prep), act, prep)
+
+
+@pytest.mark.parametrize("M,K,N,rank", [(128, 256, 128, 0), (128, 256, 128, 16), (300, 1024, 576, 32),
+                                        (77, 512, 400, 48), (256, 768, 208, 128), (1, 256, 384, 32)])
+def test_forward_int4(M, K, N, rank):
+    layer = wl.small_layer(M, K, N, rank, "int4", layer_id=11 + M)
+    X, W, b, prep = oracle_layer(layer)
+    gl = GpuLayer(prep)
+    y = gl.forward(X)
+    assert gl.status(M) == 0
+    act = oracle.quantize_act(X, prep)
+    assert_y_close(y, oracle.forward_from_act(act, prep), act, prep)
+
+
+@pytest.mark.parametrize("M,K,N", [(128, 256, 128), (300, 512, 400), (64, 1024, 256)])
+def test_int4_group_accumulators_exact(M, K, N):
+    """The int32 per-group accumulators of the INT4 GEMM equal the integer
+    triple loop bit for bit."""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    layer = wl.small_layer(M, K, N, 16, "int4", layer_id=3 + M)
+    X, W, b, prep = oracle_layer(layer)
+    gl = GpuLayer(prep)
+    act = gl.quantize(X)
+    acc = torch.zeros(K // 64, M, N, dtype=torch.int32, device="cuda:0")
+    svdq.svdq_int4_group_acc(gl.lin.handle, M, gl.lin.workspace(M), acc)
+    torch.cuda.synchronize()
+    assert gl.status(M) == 0
+    ref = oracle.int4_group_acc(act["codes"], prep["wcodes"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("name", ["c1", "c3_int4", "c4up_int4", "c4dn_int4"])
+def test_flux_workloads_int4(name):
+    layers = {l.name: l for ls in wl.WORKLOADS.values() for l in ls}
+    layer = layers[name]
+    X, W, b, prep = oracle_layer(layer)
+    gl = GpuLayer(prep)
+    M = layer.M
+    y = gl.forward(X)
+    assert gl.status(M) == 0
+    got = gl.read_act(M)
+    ref = oracle.quantize_act(X, prep)
+    np.testing.assert_array_equal(got["codes"], ref["codes"])
+    np.testing.assert_array_equal(got["scales"], ref["scales"])
+    st = assert_t_close(got["t"], ref["t"], ref, prep)
+    rows = np.unique(np.concatenate([[0, 1, M // 2, M - 1], np.random.default_rng(2).choice(M, min(M, 40), replace=False)]))
+    sub = {k: v[rows] for k, v in ref.items()}
+    s = assert_y_close(y[rows], oracle.forward_from_act(sub, prep), sub, prep)
+    print(name, s, st)
