@@ -83,6 +83,8 @@ _EXPORTS = {
     "svdq_read_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.POINTER(ctypes.c_int)]),
     "svdq_set_wait_limit": (ctypes.c_int, [ctypes.c_uint64]),
+    "svdq_forward_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                            ctypes.c_void_p]),
 }
 
 
@@ -248,6 +250,11 @@ def svdq_read_status(h, M: int, ws) -> int:
     v = ctypes.c_int()
     _check(lib().svdq_read_status(h, M, _ptr(ws), ws.numel(), ctypes.byref(v)), "svdq_read_status")
     return int(v.value)
+
+
+def svdq_forward_noalloc(h, X, M: int, Y, stream=None) -> None:
+    """Forward without a caller workspace (library-owned 32 MiB scratch per GPU)."""
+    _check(lib().svdq_forward_noalloc(h, _ptr(X), M, _ptr(Y), _stream(stream)), "svdq_forward_noalloc")
 
 
 def svdq_set_wait_limit(cycles: int) -> None:

@@ -7,7 +7,7 @@
 #include <cstddef>
 #include <cstdint>
 
-#include "../../include/svdq.h"
+#include "svdq.h"
 
 namespace svdq {
 

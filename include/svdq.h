@@ -31,7 +31,9 @@
  *     bits 4..7.  INT4 nibbles are two's complement.
  *   - Ownership: every pointer argument is owned by the caller.  Host functions
  *     take host pointers; svdq_forward and friends take device pointers and a
- *     stream and only enqueue work.  The library allocates no device memory.
+ *     stream and only enqueue work.  The library allocates no device memory
+ *     (svdq_forward_noalloc's fixed scratch array, below, is static device data
+ *     of the library module, not a run-time allocation).
  *   - Errors: every call returns an svdq_status; nothing aborts, throws or exits.
  *     Device-side failures (an in-kernel wait that ran past its limit) are
  *     recorded in a status word inside the caller's workspace and read with
@@ -176,6 +178,25 @@ svdq_status svdq_int4_group_acc(const svdq_layer* layer, int64_t M, void* ws, si
  * recorded by a kernel). */
 svdq_status svdq_read_status(const svdq_layer* layer, int64_t M, const void* ws, size_t ws_bytes,
                              int* device_status);
+
+/* svdq_forward for callers that cannot allocate device memory: for example an
+ * extension running inside a host framework that owns every device allocation
+ * and forbids cudaMalloc, or a service that must not allocate after start-up.
+ * (No counterpart in the method's description; it is a deployment variant.)
+ * X, Y are device pointers (16-byte aligned), `stream` a cudaStream_t, and the
+ * current device must be the layer's.  Instead of a caller workspace, the
+ * quantized activations, t and the status word live in one library-owned
+ * device array of 32 MiB, which exists once per GPU that loads the library and
+ * stays allocated until the process exits.  Problems whose workspace
+ * (svdq_workspace_size) exceeds 32 MiB return SVDQ_ERR_INVALID_ARG (e.g. at
+ * K = 12288, rank 32: up to about 4700 tokens).  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress), so make that
+ * first call before any stream capture.  Each call zeroes the status word;
+ * the array keeps the last call's contents otherwise.  All calls share the
+ * array: calls whose GPU work can overlap (other streams, other threads) race
+ * and must be serialized by the caller.  Allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine); asynchronous like svdq_forward. */
+svdq_status svdq_forward_noalloc(const svdq_layer* layer, const void* X, int64_t M, void* Y, void* stream);
 
 /* Upper bound, in SM clock cycles, on every in-kernel wait of later launches
  * (default 2^31, about a second).  A wait that runs past it makes the kernel
