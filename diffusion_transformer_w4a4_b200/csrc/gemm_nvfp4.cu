@@ -17,12 +17,14 @@
 //               E4M3 scale-factor atoms with bulk copies; the t / L2^T chunks of
 //               the low-rank branch ride the same ring first.
 //   warp 1      owns tensor memory (512 columns: two 192-column fp32
-//               accumulators for ping-pong with the epilogue, scale factors);
-//               one lane copies the scale factors into tensor memory
-//               (tcgen05.cp) and issues tcgen05.mma kind::f16 (low rank, K=16)
-//               and kind::mxf4nvf4 block16 (K=64) into the accumulator.
+//               accumulators for ping-pong with the epilogue, and two 48-column
+//               scale-factor buffers so the copies for the next stage overlap
+//               the MMAs of the current one); one lane copies the scale factors
+//               into tensor memory (tcgen05.cp) and issues tcgen05.mma
+//               kind::f16 (low rank, K=16) and kind::mxf4nvf4 block16 (K=64).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, scale, bias,
-//               bf16 round-to-nearest-even, 16-byte stores.
+//               bf16 round-to-nearest-even into a 128B-swizzled shared-memory
+//               staging tile, written to Y by TMA bulk-tensor stores.
 // Every wait is bounded (see sm100.cuh); no load uses cluster multicast.
 #include <cuda_bf16.h>
 
@@ -44,15 +46,17 @@ constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;  // 4 k-atoms x 256 rows (192 us
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SFA_COL = 2 * BN;       // 384
-constexpr uint32_t SFB_COL = 2 * BN + 16;  // 400
+constexpr uint32_t SF_COL = 2 * BN;  // 384: two buffers of [SFA 16 | SFB 32] columns
+constexpr uint32_t SF_BUF_COLS = 48;
+constexpr int EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 rows x 64 bf16, 128B-swizzled
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * 2 * EPI_STAGE_BYTES;
 constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-static_assert(SFB_COL + 32 <= TMEM_COLS, "tensor memory budget");
+static_assert(SF_COL + 2 * SF_BUF_COLS <= TMEM_COLS, "tensor memory budget");
 
 struct GemmMaps {
-  CUtensorMap a, b, t[3], l2[3];
+  CUtensorMap a, b, t[3], l2[3], y;
 };
 
 struct GParams {
@@ -73,7 +77,8 @@ __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 
 __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant__ GemmMaps maps, const GParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint8_t* epi_stage = smem + STAGES * STAGE_BYTES;  // [4 warps][2][EPI_STAGE_BYTES]
+  uint64_t* full = (uint64_t*)(smem + SMEM_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
@@ -148,7 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int it = 0, local = 0;
+      int it = 0, local = 0, kst = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++local) {
         const int b = local & 1;
@@ -177,18 +182,21 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
           } else {
             const uint32_t sfa_s = b_addr + B_BYTES;
             const uint32_t sfb_s = sfa_s + SFA_BYTES;
+            const uint32_t sfa_t = tmem + SF_COL + (uint32_t)(kst & 1) * SF_BUF_COLS;
+            const uint32_t sfb_t = sfa_t + 16;
+            ++kst;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              tmem_cp_32x128b_x4(tmem + SFA_COL + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-              tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * j, make_sdesc(sfb_s + j * 2 * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-              tmem_cp_32x128b_x4(tmem + SFB_COL + 8 * j + 4,
+              tmem_cp_32x128b_x4(sfa_t + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4(sfb_t + 8 * j, make_sdesc(sfb_s + j * 2 * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4(sfb_t + 8 * j + 4,
                                  make_sdesc(sfb_s + j * 2 * kSfAtomBytes + kSfAtomBytes, 0, 128, LAYOUT_NONE));
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               mma_nvf4(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
-                       make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), IDESC_NVF4, tmem + SFA_COL + 4 * j,
-                       tmem + SFB_COL + 8 * j, accum);
+                       make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), IDESC_NVF4, sfa_t + 4 * j, sfb_t + 8 * j,
+                       accum);
               accum = 1;
             }
           }
@@ -202,47 +210,65 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
-    const int row = 32 * q + lane;
-    int local = 0;
+    uint8_t* stg = epi_stage + (warp - 2) * 2 * EPI_STAGE_BYTES;
+    int local = 0, sbuf = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
       const int b = local & 1;
       if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) break;
       tc_fence_after();
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-      const int m = mt * BM + row;
+      const int m0 = mt * BM + 32 * q;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tbase + 32 * c, r);
-        tmem_ld_wait();
-        if (c == BN / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(&acc_empty[b]);
-        }
-        const int n0 = nt * BN + 32 * c;
-        if (m < p.M) {
+      for (int c = 0; c < BN / 64; ++c) {
+        const int n0 = nt * BN + 64 * c;
+        uint8_t* dst = stg + sbuf * EPI_STAGE_BYTES + lane * 128;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int n = n0 + 8 * j;
-            if (n < p.N) {
-              const float4 b0 = __ldg((const float4*)(p.bias + n));
-              const float4 b1 = __ldg((const float4*)(p.bias + n + 4));
-              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-              uint32_t o[4];
+        for (int h = 0; h < 2; ++h) {
+          float bb[32];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float y0 = fmaf(__uint_as_float(r[8 * j + 2 * e]), p.out_scale, bb[2 * e]);
-                const float y1 = fmaf(__uint_as_float(r[8 * j + 2 * e + 1]), p.out_scale, bb[2 * e + 1]);
-                __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-                o[e] = *(uint32_t*)&h;
-              }
-              *(uint4*)(p.Y + (size_t)m * p.N + n) = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int j = 0; j < 8; ++j) {
+            const int n = n0 + 32 * h + 4 * j;
+            const float4 v = (n < p.N) ? __ldg((const float4*)(p.bias + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            bb[4 * j] = v.x;
+            bb[4 * j + 1] = v.y;
+            bb[4 * j + 2] = v.z;
+            bb[4 * j + 3] = v.w;
+          }
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + 64 * c + 32 * h, r);
+          tmem_ld_wait();
+          if (c == BN / 64 - 1 && h == 1) {
+            tc_fence_before();
+            mbar_arrive(&acc_empty[b]);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 16-byte chunk 4h+k of this row, swizzled
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 8 * k + 2 * e;
+              const float y0 = fmaf(__uint_as_float(r[j]), p.out_scale, bb[j]);
+              const float y1 = fmaf(__uint_as_float(r[j + 1]), p.out_scale, bb[j + 1]);
+              __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
+              o[e] = *(uint32_t*)&hv;
             }
+            const int chunk = 4 * h + k;
+            *(uint4*)(dst + ((chunk ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&maps.y, stg + sbuf * EPI_STAGE_BYTES, n0, m0);
+          bulk_commit();
+          bulk_wait_read<1>();  // the other staging buffer is free again
+        }
+        __syncwarp();
+        sbuf ^= 1;
       }
     }
+    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
@@ -308,7 +334,10 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
   p.out_scale = L->g_x * L->g_w;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
-  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+  st = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 32,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SVDQ_OK) return st;
+  const size_t smem = 1024 + (size_t)SMEM_BYTES + 256;
   if (cudaFuncSetAttribute(k_gemm_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   const int grid = p.num_tiles < sm_count(L->device) ? p.num_tiles : sm_count(L->device);

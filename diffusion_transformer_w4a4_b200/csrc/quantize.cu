@@ -7,16 +7,25 @@
 // per-tensor scale g_x), and the 16-bit low-rank down-projection
 // t = bf16( bf16(x^) L1 ) with fp32 accumulation.
 //
-// Layout of the work: a CTA owns 32 token rows and walks K in 256-column
-// chunks.  A producer warp streams X chunks [32 x 256] and the matching L1^T
-// slices [rank x 256] (four 64-column boxes, 128-byte swizzle) into a
-// multi-stage shared-memory ring with TMA.  Eight consumer warps quantize four
-// rows each (a lane holds 8 consecutive elements, so a 16-element NVFP4 block
-// is a lane pair and a 64-element INT4 group is 8 lanes; group maxima use
-// warp shuffles), write codes/scales with coalesced stores, stage bf16(x^) in
-// shared memory, then run the down-projection on tensor cores with
-// mma.sync m16n8k16 (fp32 accumulation) from ldmatrix fragments.  HBM traffic
-// is one read of X plus the 4-bit codes, scales and t.
+// Work split: a CTA owns 128 token rows and one slice of K (the K range is cut
+// into enough slices that about one CTA per SM is in flight).  Per 128-column
+// chunk:
+//   warp 8      TMA: the X tile [128 x 128] into a ring that the quantizing
+//               warps release as soon as they have read it;
+//   warp 10     TMA: the matching L1^T slice [rank x 128] (two 64-column boxes,
+//               128-byte swizzle) into a small ring released by the MMAs;
+//   warps 0-7   quantize 16 rows each (a lane holds 16 consecutive elements:
+//               one NVFP4 block, or a quarter of a 64-element INT4 group whose
+//               maximum takes two warp shuffles; products in packed f32x2),
+//               store codes and scales, and write bf16(x^) into a
+//               128-byte-swizzled K-major tile;
+//   warp 9      issues tcgen05.mma kind::f16 (M = 128 tokens, N = rank, K = 16)
+//               on that tile and the L1^T slice, accumulating the slice's part of
+//               t in tensor memory.
+// At the end the slice's fp32 partial of t leaves tensor memory; the last CTA of
+// a row block to finish (arrival counter) adds the slices in a fixed order and
+// writes bf16 t, so the result does not depend on scheduling.  HBM traffic is
+// one read of X plus the codes, scales and t.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -26,20 +35,27 @@
 namespace svdq {
 namespace {
 
-constexpr int kRows = 32;          // token rows per CTA
-constexpr int kConsumerWarps = 8;  // 4 rows each
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kXTileBytes = kRows * kKStage * 2;  // 16 KiB
-constexpr int kAPitch = kKStage * 2 + 16;         // padded bf16 row pitch (conflict-free ldmatrix)
-constexpr int kATileBytes = kRows * kAPitch;
+constexpr int kRows = kQRows;    // 128
+constexpr int kChunk = kQChunk;  // 128
+constexpr int kConsumerWarps = 8;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kL1Warp = 10;
+constexpr int kThreads = 11 * 32;
+constexpr int kXTileBytes = kRows * kChunk * 2;  // 32 KiB
+constexpr int kAHalfBytes = kRows * 128;         // 64 bf16 columns, 128B-swizzled
+constexpr int kATileBytes = 2 * kAHalfBytes;     // 32 KiB
+constexpr int kSmemBudget = 220 * 1024;
 
 struct QParams {
-  int M, K, rank, stages, nchunks, katoms;
+  int M, K, xstages, lstages, nslices, nch, katoms;
   const float* inv_lambda;
-  float g, den;  // NVFP4 per-tensor scale and 6*g
+  float g, inv_g, den;  // NVFP4 per-tensor scale, its exact inverse, 6*g
   uint8_t* codes;
   uint8_t* scales;
   uint16_t* t;
+  float* tpart;  // [nslices, M, rank] when nslices > 1
+  int* counters;
   int* status;
   unsigned long long limit;
 };
@@ -57,6 +73,18 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
   return out;
 }
 
+// (a0, a1) * (b0, b1) with one packed instruction; each product is an ordinary
+// binary32 round-to-nearest multiply.
+__device__ __forceinline__ void mul2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%0, %1};\n\t"
+      "mov.b64 y, {%2, %3};\n\t"
+      "mul.rn.f32x2 z, x, y;\n\t"
+      "mov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+
 __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
@@ -69,267 +97,349 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {  // c in [0, 0x7E]
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
-}
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
-// Accumulator layout per warp: WN warps split the rank's n8 tiles, WK warps
-// split the 16 k-steps of a chunk; 2 m16 tiles (32 rows) x NT n8 tiles.
-constexpr int gcd_c(int a, int b) { return b == 0 ? a : gcd_c(b, a % b); }
 template <int RANK>
-struct RankCfg {
-  static constexpr int NT8 = RANK / 8;
-  static constexpr int WN = NT8 > 0 ? gcd_c(NT8, kConsumerWarps) : 1;  // divides both
-  static constexpr int WK = kConsumerWarps / WN;
-  static constexpr int NT = NT8 > 0 ? NT8 / WN : 0;
-};
+__host__ __device__ constexpr uint32_t tmem_cols() {
+  return RANK <= 32 ? 32u : (RANK <= 64 ? 64u : 128u);
+}
 
 template <int FMT, int RANK>
 __global__ void __launch_bounds__(kThreads, 1)
     k_quantize(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1, QParams p) {
-  using C = RankCfg<RANK>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int S = p.stages;
-  const int l1_bytes = RANK * kKStage * 2;  // 4 boxes of RANK rows x 128 B
-  const int stage_bytes = kXTileBytes + l1_bytes;
-  uint8_t* atile = smem + S * stage_bytes;                      // 2 x [32][kAPitch]
-  uint64_t* full = (uint64_t*)(atile + 2 * kATileBytes);        // [S]
-  uint64_t* empty = full + S;                                   // [S]
-  volatile int* abort_flag = (volatile int*)(empty + S);
+  const int XS = p.xstages, LS = p.lstages;
+  constexpr int kL1Bytes = RANK * kChunk * 2;  // two boxes of RANK rows x 128 B
+  uint8_t* xring = smem;                          // [XS][kXTileBytes]
+  uint8_t* atile = xring + XS * kXTileBytes;      // [2][kATileBytes] when RANK > 0
+  uint8_t* lring = atile + (RANK > 0 ? 2 * kATileBytes : 0);  // [LS][kL1Bytes]
+  float* rtab = (float*)(lring + LS * kL1Bytes);  // [128] 1/e4m3
+  uint64_t* full_x = (uint64_t*)(rtab + 128);
+  uint64_t* empty_x = full_x + XS;
+  uint64_t* full_l = empty_x + XS;
+  uint64_t* empty_l = full_l + LS;
+  uint64_t* xready = empty_l + LS;  // [2]
+  uint64_t* xfree = xready + 2;     // [2]
+  uint64_t* tdone = xfree + 2;
+  uint32_t* tmem_slot = (uint32_t*)(tdone + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  volatile int* ticket = abort_flag + 1;
+  volatile int* decision = abort_flag + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kRows;
+  const int rowblock = blockIdx.x, slice = blockIdx.y;
+  const int m0 = rowblock * kRows;
+  const int c_begin = (int)((int64_t)slice * p.nch / p.nslices);
+  const int c_end = (int)((int64_t)(slice + 1) * p.nch / p.nslices);
+  const int nchunks = c_end - c_begin;
   WaitCtl wc{abort_flag, p.status, p.limit};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(&full_x[s], 1);
+      mbar_init(&empty_x[s], kConsumerWarps);
     }
+    for (int s = 0; s < LS; ++s) {
+      mbar_init(&full_l[s], 1);
+      mbar_init(&empty_l[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&xready[b], kConsumerWarps);
+      mbar_init(&xfree[b], 1);
+    }
+    mbar_init(tdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (FMT == SVDQ_NVFP4_G16 && threadIdx.x < 128)  // exact reciprocals of the E4M3 values
+    rtab[threadIdx.x] = (threadIdx.x == 0 || threadIdx.x == 0x7F) ? 0.f : __frcp_rn(e4m3_value(threadIdx.x));
+  if constexpr (RANK > 0) {
+    if (warp == kMmaWarp) {
+      tmem_alloc(tmem_slot, tmem_cols<RANK>());
+      tmem_relinquish();
+    }
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
 
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ X producer
     if (lane == 0) {
       prefetch_tmap(&map_x);
-      if constexpr (RANK > 0) prefetch_tmap(&map_l1);
       int issued = 0;
-      for (int c = 0; c < p.nchunks; ++c) {
-        const int s = c % S;
-        if (!mbar_wait(&empty[s], ((c / S) & 1) ^ 1, wc)) break;
-        uint8_t* st = smem + s * stage_bytes;
-        mbar_arrive_expect_tx(&full[s], stage_bytes);
-        tma_load_2d(&map_x, &full[s], st, c * kKStage, m0);
-        if constexpr (RANK > 0) {
-#pragma unroll
-          for (int b = 0; b < 4; ++b) tma_load_2d(&map_l1, &full[s], st + kXTileBytes + b * RANK * 128, c * kKStage + 64 * b, 0);
-        }
-        issued = c + 1;
+      for (int i = 0; i < nchunks; ++i) {
+        const int s = i % XS;
+        if (!mbar_wait(&empty_x[s], ((i / XS) & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&full_x[s], kXTileBytes);
+        tma_load_2d(&map_x, &full_x[s], xring + s * kXTileBytes, (c_begin + i) * kChunk, m0);
+        issued = i + 1;
       }
       if (*abort_flag) {  // drain copies that are still in flight before leaving
-        for (int c = (issued > S ? issued - S : 0); c < issued; ++c)
-          mbar_wait_drain(&full[c % S], (c / S) & 1, p.limit);
+        for (int i = (issued > XS ? issued - XS : 0); i < issued; ++i)
+          mbar_wait_drain(&full_x[i % XS], (i / XS) & 1, p.limit);
+      }
+    }
+  } else if (warp == kL1Warp) {
+    // ------------------------------------------------------------ L1^T producer
+    if constexpr (RANK > 0) {
+      if (lane == 0) {
+        prefetch_tmap(&map_l1);
+        int issued = 0;
+        for (int i = 0; i < nchunks; ++i) {
+          const int s = i % LS;
+          if (!mbar_wait(&empty_l[s], ((i / LS) & 1) ^ 1, wc)) break;
+          const int k0 = (c_begin + i) * kChunk;
+          uint8_t* dst = lring + s * kL1Bytes;
+          mbar_arrive_expect_tx(&full_l[s], kL1Bytes);
+          tma_load_2d(&map_l1, &full_l[s], dst, k0, 0);
+          tma_load_2d(&map_l1, &full_l[s], dst + RANK * 128, k0 + 64, 0);
+          issued = i + 1;
+        }
+        if (*abort_flag) {
+          for (int i = (issued > LS ? issued - LS : 0); i < issued; ++i)
+            mbar_wait_drain(&full_l[i % LS], (i / LS) & 1, p.limit);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if constexpr (RANK > 0) {
+      if (lane == 0) {
+        const uint32_t tmem = *tmem_slot;
+        constexpr uint32_t idesc = idesc_bf16_f32(kRows, RANK);
+        for (int i = 0; i < nchunks; ++i) {
+          const int s = i % LS, buf = i & 1;
+          if (!mbar_wait(&xready[buf], (i >> 1) & 1, wc)) break;
+          if (!mbar_wait(&full_l[s], (i / LS) & 1, wc)) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(atile + buf * kATileBytes);
+          const uint32_t b_addr = smem_u32(lring + s * kL1Bytes);
+#pragma unroll
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
+            const uint32_t h = kk >> 2, koff = (kk & 3) * 32;
+            mma_bf16(tmem, make_sdesc(a_addr + h * kAHalfBytes + koff, 16, 1024, LAYOUT_SW128),
+                     make_sdesc(b_addr + h * RANK * 128 + koff, 16, 1024, LAYOUT_SW128), idesc,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&xfree[buf]);
+          umma_commit(&empty_l[s]);
+        }
+        umma_commit(tdone);  // fires when every MMA above has completed
+        if (*abort_flag) mbar_wait_drain(tdone, 0, p.limit);
       }
     }
   } else {
-    // ------------------------------------------------------------ consumers
-    float acc[2][C::NT > 0 ? C::NT : 1][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int b = 0; b < (C::NT > 0 ? C::NT : 1); ++b)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[a][b][q] = 0.f;
-    const int wn = warp % C::WN, wk = warp / C::WN;
+    // ------------------------------------------------------------ quantizing warps
+    const int rsub = lane >> 3;  // row within the warp's 4-row step
+    const int j = lane & 7;      // 16-column group within the chunk
     const int K2 = p.K / 2;
-
-    for (int c = 0; c < p.nchunks; ++c) {
-      const int s = c % S;
-      const bool ok = mbar_wait(&full[s], (c / S) & 1, wc);
-      uint8_t* st = smem + s * stage_bytes;
-      uint8_t* at = atile + (c & 1) * kATileBytes;
+    for (int i = 0; i < nchunks; ++i) {
+      const int s = i % XS, buf = i & 1;
+      bool ok = mbar_wait(&full_x[s], (i / XS) & 1, wc);
+      if constexpr (RANK > 0) ok = ok && mbar_wait(&xfree[buf], ((i >> 1) & 1) ^ 1, wc);
       if (ok) {
-        const int k0 = c * kKStage + lane * 8;
-        const float4 il0 = __ldg((const float4*)(p.inv_lambda + k0));
-        const float4 il1 = __ldg((const float4*)(p.inv_lambda + k0 + 4));
-        const float il[8] = {il0.x, il0.y, il0.z, il0.w, il1.x, il1.y, il1.z, il1.w};
+        const uint8_t* st = xring + s * kXTileBytes;
+        const int k0 = (c_begin + i) * kChunk;
+        const int kk0 = k0 + 16 * j;
+        float il[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = warp * 4 + i;
+        for (int q = 0; q < 4; ++q) {
+          const float4 t4 = __ldg((const float4*)(p.inv_lambda + kk0 + 4 * q));
+          il[4 * q] = t4.x;
+          il[4 * q + 1] = t4.y;
+          il[4 * q + 2] = t4.z;
+          il[4 * q + 3] = t4.w;
+        }
+        uint8_t* at = atile + buf * kATileBytes + (j >> 2) * kAHalfBytes;
+#pragma unroll 2
+        for (int it = 0; it < 4; ++it) {
+          const int row = warp * 16 + 4 * it + rsub;
           const int m = m0 + row;
-          const uint4 raw = *(const uint4*)(st + row * (kKStage * 2) + lane * 16);
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-          float v[8];
+          const uint4 r0 = *(const uint4*)(st + row * (kChunk * 2) + 32 * j);
+          const uint4 r1 = *(const uint4*)(st + row * (kChunk * 2) + 32 * j + 16);
+          const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+          float v[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[2 * j] = __fmul_rn(__uint_as_float(w[j] << 16), il[2 * j]);
-            v[2 * j + 1] = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), il[2 * j + 1]);
+          for (int e = 0; e < 8; ++e) {
+            v[2 * e] = __uint_as_float(w[e] << 16);
+            v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+            mul2(v[2 * e], v[2 * e + 1], il[2 * e], il[2 * e + 1]);
           }
           float amax = 0.f;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-          uint32_t packed = 0;
+          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
+          uint2 packed = make_uint2(0u, 0u);
           if (FMT == SVDQ_NVFP4_G16) {
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, p.den));
             if (sb != 0) {
-              const float inv = __fdiv_rn(1.0f, __fmul_rn(e4m3_value(sb), p.g));
-              float q[8];
+              // 1 / (e4m3(sb) * g) exactly: g is a power of two
+              const float inv = rtab[sb] * p.inv_g;
+              float q0[8], q1[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) q[j] = __fmul_rn(v[j], inv);
-              packed = cvt_e2m1x8(q);
+              for (int e = 0; e < 4; ++e) {
+                q0[2 * e] = v[2 * e];
+                q0[2 * e + 1] = v[2 * e + 1];
+                q1[2 * e] = v[8 + 2 * e];
+                q1[2 * e + 1] = v[9 + 2 * e];
+                mul2(q0[2 * e], q0[2 * e + 1], inv, inv);
+                mul2(q1[2 * e], q1[2 * e + 1], inv, inv);
+              }
+              packed = make_uint2(cvt_e2m1x8(q0), cvt_e2m1x8(q1));
             }
-            // gather the four block scales of each 64-column atom into one word
-            const int base = lane & ~7;
-            const uint32_t s0 = __shfl_sync(0xffffffffu, sb, base + 0);
-            const uint32_t s1 = __shfl_sync(0xffffffffu, sb, base + 2);
-            const uint32_t s2 = __shfl_sync(0xffffffffu, sb, base + 4);
-            const uint32_t s3 = __shfl_sync(0xffffffffu, sb, base + 6);
-            if ((lane & 7) == 0 && m < p.M) {
-              const int blk = c * (kKStage / 16) + (lane >> 3) * 4;
-              *(uint32_t*)(p.scales + sf_offset(m, blk, p.katoms, kSfAtomRows)) =
-                  s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
-            }
+            const int base = lane & ~3;  // 4 lanes = 64 columns = one scale-factor atom word
+            const uint32_t s1 = __shfl_sync(0xffffffffu, sb, base + 1);
+            const uint32_t s2 = __shfl_sync(0xffffffffu, sb, base + 2);
+            const uint32_t s3 = __shfl_sync(0xffffffffu, sb, base + 3);
+            if ((lane & 3) == 0 && m < p.M)
+              *(uint32_t*)(p.scales + sf_offset(m, kk0 / 16, p.katoms, kSfAtomRows)) =
+                  sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
           } else {
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
             const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
             const float S16 = __half2float(s16);
             if (S16 != 0.f) {
-              const float inv = __fdiv_rn(1.0f, S16);
+              const float inv = __frcp_rn(S16);
+              uint32_t pk[2] = {0u, 0u};
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                int q = __float2int_rn(__fmul_rn(v[j], inv));
-                q = max(-8, min(7, q));
-                packed |= (uint32_t)(q & 0xF) << (4 * j);
+              for (int e = 0; e < 16; e += 2) {
+                float y0 = v[e], y1 = v[e + 1];
+                mul2(y0, y1, inv, inv);
+                // round half to even on the clamped value: the 4 low bits of
+                // (y + 1.5 * 2^23) are the two's-complement code
+                y0 = fminf(fmaxf(y0, -8.0f), 7.0f);
+                y1 = fminf(fmaxf(y1, -8.0f), 7.0f);
+                const uint32_t c0 = __float_as_uint(__fadd_rn(y0, 12582912.0f)) & 0xFu;
+                const uint32_t c1 = __float_as_uint(__fadd_rn(y1, 12582912.0f)) & 0xFu;
+                pk[e >> 3] |= (c0 | (c1 << 4)) << (4 * (e & 7));
               }
+              packed = make_uint2(pk[0], pk[1]);
             }
-            if ((lane & 7) == 0 && m < p.M) {
-              const int grp = c * (kKStage / 64) + (lane >> 3);
-              ((__half*)p.scales)[(size_t)grp * p.M + m] = s16;
-            }
+            if ((lane & 3) == 0 && m < p.M) ((__half*)p.scales)[(size_t)(kk0 / 64) * p.M + m] = s16;
           }
-          if (m < p.M) *(uint32_t*)(p.codes + (size_t)m * K2 + c * (kKStage / 2) + lane * 4) = packed;
+          if (m < p.M) *(uint2*)(p.codes + (size_t)m * K2 + kk0 / 2) = packed;
           if constexpr (RANK > 0) {
-            uint4 xb;
-            __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
-            __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
-            __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
-            xb.x = *(uint32_t*)&h0;
-            xb.y = *(uint32_t*)&h1;
-            xb.z = *(uint32_t*)&h2;
-            xb.w = *(uint32_t*)&h3;
-            *(uint4*)(at + row * kAPitch + lane * 16) = xb;
+            uint32_t b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+              b[e] = *(uint32_t*)&h;
+            }
+            const int c0 = 2 * (j & 3);
+            *(uint4*)(at + row * 128 + ((c0 ^ (row & 7)) << 4)) = make_uint4(b[0], b[1], b[2], b[3]);
+            *(uint4*)(at + row * 128 + (((c0 + 1) ^ (row & 7)) << 4)) = make_uint4(b[4], b[5], b[6], b[7]);
           }
         }
       }
-      if constexpr (RANK > 0) {
-        named_bar_sync(1, kConsumerWarps * 32);  // bf16(x^) tile complete
-        if (ok) {
-          const uint8_t* l1t = st + kXTileBytes;
-          const uint32_t a_base = smem_u32(at);
-          const uint32_t l_base = smem_u32(l1t);
-#pragma unroll 4
-          for (int ks = wk; ks < kKStage / 16; ks += C::WK) {
-            uint32_t af[2][4];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              const int row = mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-              const int col = ks * 16 + 8 * (lane >> 4);
-              ldmatrix_x4(a_base + row * kAPitch + col * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-            }
-#pragma unroll
-            for (int nt = 0; nt < (C::NT > 0 ? C::NT : 1); ++nt) {
-              const int n = 8 * (wn + C::WN * nt) + (lane & 7);
-              const int kl = ks * 16 + 8 * ((lane >> 3) & 1);
-              const int box = kl >> 6, chunk = (kl & 63) >> 3;
-              const uint32_t addr = l_base + box * (RANK * 128) + n * 128 + ((chunk ^ (n & 7)) << 4);
-              uint32_t b0, b1;
-              ldmatrix_x2(addr, b0, b1);
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) mma_16816(acc[mt][nt], af[mt], b0, b1);
-            }
-          }
-        }
-      }
+      if constexpr (RANK > 0) fence_proxy_async_smem();  // x^ tile -> tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) {
+        mbar_arrive(&empty_x[s]);  // the X tile has been read
+        if constexpr (RANK > 0) mbar_arrive(&xready[buf]);
+      }
     }
 
     if constexpr (RANK > 0) {
-      // cross-warp reduction of the k-split partial sums in a fixed order
-      // (k-split 0, then 1, ...), in place in one [32][RANK] fp32 buffer
-      named_bar_sync(1, kConsumerWarps * 32);  // all MMAs done: the A tiles are free
-      float* red = (float*)atile;
-      const int g = lane >> 2, q = lane & 3;
-      for (int k = 0; k < C::WK; ++k) {
-        if (wk == k) {
+      if (warp < 4) {
+        // the slice's partial t leaves tensor memory (warp w owns lanes 32w..32w+31)
+        mbar_wait(tdone, 0, wc);
+        tc_fence_after();
+        const int row = 32 * warp + lane;
+        const int m = m0 + row;
+        const uint32_t tl = *tmem_slot + ((uint32_t)(32 * warp) << 16);
+        float acc[RANK];
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
+        for (int c = 0; c < RANK / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tl + 16 * c, r);
+          tmem_ld_wait();
 #pragma unroll
-            for (int nt = 0; nt < (C::NT > 0 ? C::NT : 1); ++nt) {
-              const int col = 8 * (wn + C::WN * nt) + 2 * q;
-              float* r0 = red + (size_t)(mt * 16 + g) * RANK + col;
-              float* r1 = red + (size_t)(mt * 16 + g + 8) * RANK + col;
-              if (k == 0) {
-                r0[0] = acc[mt][nt][0]; r0[1] = acc[mt][nt][1];
-                r1[0] = acc[mt][nt][2]; r1[1] = acc[mt][nt][3];
-              } else {
-                r0[0] += acc[mt][nt][0]; r0[1] += acc[mt][nt][1];
-                r1[0] += acc[mt][nt][2]; r1[1] += acc[mt][nt][3];
+          for (int j = 0; j < 16; ++j) acc[16 * c + j] = __uint_as_float(r[j]);
+        }
+        // one go/no-go decision for all 128 threads, so every barrier below is uniform
+        named_bar_sync(2, 128);
+        if (threadIdx.x == 0) *decision = *abort_flag ? 0 : 1;
+        named_bar_sync(2, 128);
+        if (*decision) {
+          if (p.nslices == 1) {
+            if (m < p.M) {
+#pragma unroll
+              for (int j = 0; j < RANK; j += 2) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+                *(uint32_t*)(p.t + (size_t)m * RANK + j) = *(uint32_t*)&h;
               }
             }
-        }
-        named_bar_sync(1, kConsumerWarps * 32);
-      }
-      if (!*abort_flag) {
-        for (int idx = threadIdx.x; idx < kRows * RANK / 2; idx += kConsumerWarps * 32) {
-          const int row = idx / (RANK / 2), col = 2 * (idx % (RANK / 2));
-          const float s0 = red[(size_t)row * RANK + col], s1 = red[(size_t)row * RANK + col + 1];
-          const int m = m0 + row;
-          if (m < p.M) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(s0, s1);
-            *(uint32_t*)(p.t + (size_t)m * RANK + col) = *(uint32_t*)&h;
+          } else {
+            if (m < p.M) {
+              float* dst = p.tpart + ((size_t)slice * p.M + m) * RANK;
+#pragma unroll
+              for (int j = 0; j < RANK; j += 4)
+                *(float4*)(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+            }
+            __threadfence();
+            named_bar_sync(2, 128);
+            if (threadIdx.x == 0) *ticket = atomicAdd(p.counters + rowblock, 1);
+            named_bar_sync(2, 128);
+            if (*ticket == p.nslices - 1) {  // last slice of this row block: fixed-order sum
+              __threadfence();
+              if (m < p.M) {
+#pragma unroll
+                for (int j = 0; j < RANK; j += 4) {
+                  float4 sum = __ldcg((const float4*)(p.tpart + (size_t)m * RANK + j));
+                  for (int sl = 1; sl < p.nslices; ++sl) {
+                    const float4 v = __ldcg((const float4*)(p.tpart + ((size_t)sl * p.M + m) * RANK + j));
+                    sum.x += v.x;
+                    sum.y += v.y;
+                    sum.z += v.z;
+                    sum.w += v.w;
+                  }
+                  __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+                  __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                  *(uint2*)(p.t + (size_t)m * RANK + j) = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+                }
+              }
+              if (threadIdx.x == 0) p.counters[rowblock] = 0;  // ready for the next call
+            }
           }
         }
       }
     }
   }
+
+  tc_fence_before();
   __syncthreads();
+  if constexpr (RANK > 0) {
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(*tmem_slot, tmem_cols<RANK>());
+    }
+  }
 }
 
 template <int FMT, int RANK>
 int launch_rank(const CUtensorMap& mx, const CUtensorMap& ml1, const QParams& p, int64_t M, cudaStream_t stream) {
-  const int l1_bytes = RANK * kKStage * 2;
-  const int stage_bytes = kXTileBytes + l1_bytes;
+  constexpr int kL1Bytes = RANK * kChunk * 2;
+  constexpr int kFixed = (RANK > 0 ? 2 * kATileBytes : 0) + 512 + 512;
   QParams q = p;
-  int S = (200 * 1024 - 2 * kATileBytes) / stage_bytes;
-  if (S > 4) S = 4;
-  if (S < 1) S = 1;
-  q.stages = S;
-  const size_t smem = 1024 + (size_t)S * stage_bytes + 2 * kATileBytes + 2 * S * sizeof(uint64_t) + 16;
+  q.lstages = RANK > 0 ? (RANK <= 64 ? 3 : 2) : 0;
+  int XS = (kSmemBudget - kFixed - q.lstages * kL1Bytes) / kXTileBytes;
+  if (XS > 5) XS = 5;
+  if (XS < 2) XS = 2;
+  q.xstages = XS;
+  const size_t smem = 1024 + (size_t)XS * kXTileBytes + (size_t)q.lstages * kL1Bytes + kFixed;
   auto kern = k_quantize<FMT, RANK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;
-  const unsigned grid = (unsigned)((M + kRows - 1) / kRows);
+  const dim3 grid((unsigned)((M + kRows - 1) / kRows), (unsigned)p.nslices);
   kern<<<grid, kThreads, smem, stream>>>(mx, ml1, q);
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
@@ -357,21 +467,24 @@ int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, 
                     cudaStream_t stream) {
   CUtensorMap mx;
   int st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)L->K, (uint64_t)M,
-                          (uint64_t)L->K * 2, kKStage, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+                          (uint64_t)L->K * 2, kChunk, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != SVDQ_OK) return st;
   QParams p{};
   p.M = (int)M;
   p.K = (int)L->K;
-  p.rank = L->rank;
-  p.nchunks = (int)(L->K / kKStage);
+  p.nch = (int)(L->K / kChunk);
+  p.nslices = w.nslices;
   p.katoms = (int)(L->K / 64);
   p.inv_lambda = L->inv_lambda;
   p.g = L->g_x;
+  p.inv_g = 1.0f / L->g_x;  // exact: g_x is a power of two
   p.den = 6.0f * L->g_x;
   p.codes = ws + w.codes;
   p.scales = ws + w.scales;
   p.t = (uint16_t*)(ws + w.t);
+  p.tpart = (float*)(ws + w.tpart);
   p.status = (int*)(ws + w.status);
+  p.counters = (int*)(ws + w.status + 16);
   p.limit = wait_limit_cycles();
   if (L->fmt == SVDQ_NVFP4_G16) return launch_fmt<SVDQ_NVFP4_G16>(mx, L->map_l1, p, M, L->rank, stream);
   return launch_fmt<SVDQ_INT4_G64>(mx, L->map_l1, p, M, L->rank, stream);

@@ -81,8 +81,15 @@ Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M) {
   w.t = o;
   w.t_bytes = (size_t)M * rank * 2;
   o = align_up(o + w.t_bytes, kAlign);
+  // control block: status word, then one arrival counter per 128-row block
   w.status = o;
-  o = align_up(o + 16, kAlign);
+  w.ctrl_bytes = 16 + 4 * (size_t)((M + kQRows - 1) / kQRows);
+  o = align_up(o + w.ctrl_bytes, kAlign);
+  // fp32 partial low-rank sums of the quantizer's K slices
+  w.nslices = quant_slices(M, K);
+  w.tpart = o;
+  w.tpart_bytes = (w.nslices > 1 && rank > 0) ? (size_t)w.nslices * M * rank * 4 : 0;
+  o = align_up(o + w.tpart_bytes, kAlign);
   w.total = o;
   return w;
 }
@@ -332,7 +339,8 @@ svdq_status svdq_workspace_init(const svdq_layer* L, int64_t M, void* ws, size_t
   Workspace w;
   svdq_status st = check_ws(L, M, ws, ws_bytes, &w);
   if (st != SVDQ_OK) return st;
-  if (cudaMemsetAsync((uint8_t*)ws + w.status, 0, 16, (cudaStream_t)stream) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (cudaMemsetAsync((uint8_t*)ws + w.status, 0, w.ctrl_bytes, (cudaStream_t)stream) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
   return SVDQ_OK;
 }
 

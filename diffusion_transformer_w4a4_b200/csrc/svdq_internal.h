@@ -20,6 +20,9 @@ constexpr int kInt4BN = 128;       // INT4 GEMM tile columns
 constexpr int kSfAtomRows = 128;   // rows per tensor-core scale-factor atom
 constexpr int kSfAtomBytes = 512;  // 128 rows x 4 blocks of 16
 constexpr int kMaxRank = 128;
+constexpr int kQRows = 128;   // activation quantizer: token rows per CTA (= tcgen05 M)
+constexpr int kQChunk = 128;  // activation quantizer: K columns per pipeline chunk
+constexpr int kQSmCount = 148;  // SM count the quantizer's K-split is sized for (fixed, so sizes are device-free)
 constexpr size_t kAlign = 1024;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -44,9 +47,22 @@ struct Blob {  // offsets (bytes) of the packed-weight regions
 };
 Blob blob_layout(int64_t N, int64_t K, int rank, int fmt);
 
+// Number of K slices the activation quantizer splits each 128-row block into,
+// so that about one CTA per SM is in flight; partial low-rank sums of the
+// slices are reduced in a fixed order.
+inline int quant_slices(int64_t M, int64_t K) {
+  const int64_t rb = (M + kQRows - 1) / kQRows;
+  const int64_t nch = K / kQChunk;
+  int64_t ns = kQSmCount / (rb > 0 ? rb : 1);
+  if (ns < 1) ns = 1;
+  if (ns > nch) ns = nch;
+  return (int)ns;
+}
+
 struct Workspace {
-  size_t codes, scales, t, status, total;
-  size_t codes_bytes, scales_bytes, t_bytes;
+  size_t codes, scales, t, status, tpart, total;
+  size_t codes_bytes, scales_bytes, t_bytes, ctrl_bytes, tpart_bytes;
+  int nslices;
 };
 Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M);
 

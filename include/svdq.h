@@ -145,13 +145,16 @@ void svdq_layer_destroy(svdq_layer* layer);
 /* Workspace for M tokens: quantized activations, low-rank t and a status word.
  * layout: offsets/sizes[0] act codes u8 [M, K/2]; [1] act scales (NVFP4: E4M3
  * in the tensor-core scale-factor layout of 128-row tiles; INT4: fp16 [K/64, M]);
- * [2] t bf16 [M, rank]; [3] status word int32. */
+ * [2] t bf16 [M, rank]; [3] status word int32 (first word of a small control
+ * block that also holds the quantizer's split-K counters).  The total size also
+ * covers the quantizer's fp32 partial sums of t. */
 svdq_status svdq_workspace_size(const svdq_layer* layer, int64_t M, size_t* bytes);
 svdq_status svdq_workspace_layout(const svdq_layer* layer, int64_t M, size_t offsets[4], size_t sizes[4]);
 
-/* Zero the workspace status word (enqueued on `stream`, a cudaStream_t).
- * Required once before the first svdq_forward on a fresh workspace; the status
- * is sticky until the next init. */
+/* Zero the workspace control block: the status word and the quantizer's split-K
+ * counters (enqueued on `stream`, a cudaStream_t).  Required once before the
+ * first svdq_forward on a fresh workspace; the kernels keep the counters at zero
+ * between calls, and the status is sticky until the next init. */
 svdq_status svdq_workspace_init(const svdq_layer* layer, int64_t M, void* ws, size_t ws_bytes, void* stream);
 
 /* Y[M,N] = layer(X[M,K]).  X, Y, ws are device pointers (16-byte aligned),
@@ -189,9 +192,9 @@ svdq_status svdq_read_status(const svdq_layer* layer, int64_t M, const void* ws,
  * device array of 32 MiB, which exists once per GPU that loads the library and
  * stays allocated until the process exits.  Problems whose workspace
  * (svdq_workspace_size) exceeds 32 MiB return SVDQ_ERR_INVALID_ARG (e.g. at
- * K = 12288, rank 32: up to about 4700 tokens).  The first call on a device
+ * K = 12288, rank 32: up to about 4300 tokens).  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress), so make that
- * first call before any stream capture.  Each call zeroes the status word;
+ * first call before any stream capture.  Each call zeroes the control block;
  * the array keeps the last call's contents otherwise.  All calls share the
  * array: calls whose GPU work can overlap (other streams, other threads) race
  * and must be serialized by the caller.  Allocates nothing (no cudaMalloc,
