@@ -18,10 +18,12 @@
 //               the low-rank branch ride the same ring first.
 //   warp 1      owns tensor memory (512 columns: two 192-column fp32
 //               accumulators for ping-pong with the epilogue, and two 48-column
-//               scale-factor buffers so the copies for the next stage overlap
-//               the MMAs of the current one); one lane copies the scale factors
-//               into tensor memory (tcgen05.cp) and issues tcgen05.mma
-//               kind::f16 (low rank, K=16) and kind::mxf4nvf4 block16 (K=64).
+//               scale-factor buffers); one lane issues tcgen05.mma kind::f16
+//               (low rank, K=16) and kind::mxf4nvf4 block16 (K=64).
+//   warps 6-9   move each stage's E4M3 scale-factor atoms from shared memory
+//               into their tensor-memory lane quarter with tcgen05.st, in the
+//               replicated layout the block-scaled MMA reads, so the transfer
+//               runs beside the tensor pipe instead of inside it.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, scale, bias,
 //               bf16 round-to-nearest-even into a 128B-swizzled shared-memory
 //               staging tile, written to Y by TMA bulk-tensor stores.
@@ -44,7 +46,7 @@ constexpr int B_BYTES = BN * 128;
 constexpr int SFA_BYTES = 4 * kSfAtomBytes;      // 4 k-atoms x 128 rows
 constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;  // 4 k-atoms x 256 rows (192 used)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 2 * BN;  // 384: two buffers of [SFA 16 | SFB 32] columns
 constexpr uint32_t SF_BUF_COLS = 48;
@@ -83,7 +85,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   uint64_t* acc_full = empty + STAGES;  // [2]
   uint64_t* acc_empty = acc_full + 2;   // [2]
   uint64_t* mma_done = acc_empty + 2;   // [1]
-  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  uint64_t* sf_ready = mma_done + 1;    // [2]
+  uint64_t* sf_free = sf_ready + 2;     // [2]
+  uint32_t* tmem_slot = (uint32_t*)(sf_free + 2);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,6 +103,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       mbar_init(&acc_empty[b], 128);
     }
     mbar_init(mma_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sf_ready[b], 4);
+      mbar_init(&sf_free[b], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -180,18 +188,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
               accum = 1;
             }
           } else {
-            const uint32_t sfa_s = b_addr + B_BYTES;
-            const uint32_t sfb_s = sfa_s + SFA_BYTES;
-            const uint32_t sfa_t = tmem + SF_COL + (uint32_t)(kst & 1) * SF_BUF_COLS;
-            const uint32_t sfb_t = sfa_t + 16;
-            ++kst;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              tmem_cp_32x128b_x4(sfa_t + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-              tmem_cp_32x128b_x4(sfb_t + 8 * j, make_sdesc(sfb_s + j * 2 * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-              tmem_cp_32x128b_x4(sfb_t + 8 * j + 4,
-                                 make_sdesc(sfb_s + j * 2 * kSfAtomBytes + kSfAtomBytes, 0, 128, LAYOUT_NONE));
+            const int sb = kst & 1;
+            if (!mbar_wait(&sf_ready[sb], (kst >> 1) & 1, wc)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const uint32_t sfa_t = tmem + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+            const uint32_t sfb_t = sfa_t + 16;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               mma_nvf4(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
@@ -199,6 +203,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
                        accum);
               accum = 1;
             }
+            umma_commit(&sf_free[sb]);
+            ++kst;
           }
           umma_commit(&empty[s]);
         }
@@ -206,6 +212,44 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       }
       umma_commit(mma_done);  // every MMA issued above has completed when this fires
       mbar_wait_drain(mma_done, 0, p.limit);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ scale-factor movers
+    // Warp q owns tensor-memory lanes 32q..32q+31.  Lane l writes, for every
+    // 128-row scale-factor atom of the stage, the atom's 16-byte row l (the
+    // scales of rows l, l+32, l+64, l+96 for 4 consecutive K blocks) into 4
+    // consecutive columns -- the same bytes in every lane quarter.
+    const int q = warp & 3;
+    int it = 0, kst = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int u = 0; u < units; ++u, ++it) {
+        if (u < p.n_lr) continue;
+        const int s = it % STAGES, sb = kst & 1;
+        ok = mbar_wait(&full[s], (it / STAGES) & 1, wc) && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+        if (!ok) break;
+        const uint8_t* sfa_s = smem + s * STAGE_BYTES + A_BYTES + B_BYTES;
+        const uint8_t* sfb_s = sfa_s + SFA_BYTES;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
+          ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + h) * kSfAtomBytes + lane * 16);
+            rb[8 * j + 4 * h] = b4.x; rb[8 * j + 4 * h + 1] = b4.y; rb[8 * j + 4 * h + 2] = b4.z; rb[8 * j + 4 * h + 3] = b4.w;
+          }
+        }
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+        tmem_st_32x32b_x16(tq, ra);
+        tmem_st_32x32b_x32(tq + 16, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready[sb]);
+        ++kst;
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
