@@ -10,18 +10,23 @@
 // tcgen05.mma kind::i8 (int32 accumulation).  Because both scales change every
 // 64 columns of K, each group's int32 accumulator is drained and rescaled by
 // the epilogue warps into an fp32 running sum held in registers, while the
-// tensor core fills the other of two ping-pong accumulators.
+// tensor core fills the next of four accumulators.  Every accumulator starts
+// at the integer 0x4B400000, the bit pattern of 1.5 * 2^23: after adding a
+// group sum (|sum| <= 64 * 8 * 8 = 4096) the int32 result read as binary32 is
+// exactly 1.5 * 2^23 + sum, so one packed subtraction recovers the sum as a
+// float without an integer-to-float conversion.
 //
 // Persistent, warp-specialized CTA (one per SM), tile 128 x 128:
-//   warp 0      TMA producer: packed codes [128 x 64 B] for A and B per
-//               128-column K stage (raw ring), and the bf16 t / L2^T chunks
-//               of the low-rank branch (own buffer).
-//   warp 1      owns tensor memory (2 x 128 columns) and issues the MMAs:
+//   warp 0      TMA producer: packed codes [128 x 128 B] (128-byte swizzle)
+//               for A and B per 256-column K stage (raw ring), and the bf16
+//               t / L2^T chunks of the low-rank branch (own buffer).
+//   warp 1      owns tensor memory (4 x 128 columns) and issues the MMAs:
 //               kind::f16 for t . L2 (its own accumulator unit, which seeds the
-//               running sum), then 2 x kind::i8 (K=32) per 64-group.
-//   warps 2-5   converters: raw int4 -> int8, sign-extended, written in the
+//               running sum), then 2 x kind::i8 (K=32) per 64-group, four
+//               groups per stage.
+//   warps 2-3   converters: raw int4 -> int8, sign-extended, written in the
 //               128-byte-swizzled K-major layout the MMA reads (conv ring).
-//   warps 6-13  epilogue (two per lane quarter, 64 columns each): tcgen05.ld
+//   warps 4-11  epilogue (two per lane quarter, 64 columns each): tcgen05.ld
 //               each unit; y += s_x s_w float(acc);
 //               bias, bf16 round-to-nearest-even, 16-byte stores.  With a
 //               debug output pointer it instead writes the raw int32 group
@@ -40,21 +45,28 @@ namespace {
 
 constexpr int BM = kGemmBM;  // 128
 constexpr int BN = kInt4BN;  // 128
-constexpr int BK = 128;      // K elements per stage (2 groups of 64)
-constexpr int RAW_STAGES = 4;
-constexpr int CONV_STAGES = 3;
-constexpr int RAW_A = BM * BK / 2;  // 8 KiB packed
+constexpr int BK = 256;      // K elements per stage (4 groups of 64)
+constexpr int GPS = BK / 64;  // groups per stage
+constexpr int RAW_STAGES = 2;
+constexpr int CONV_STAGES = 2;
+constexpr int RAW_A = BM * BK / 2;  // 16 KiB packed, one 128-byte swizzled row per token
 constexpr int RAW_B = BN * BK / 2;
 constexpr int RAW_BYTES = RAW_A + RAW_B;
-constexpr int CONV_A = BM * BK;  // 16 KiB int8
-constexpr int CONV_B = BN * BK;
+constexpr int CONV_HALF = BM * 128;  // int8 sub-tile of 128 K columns, 128-byte swizzled
+constexpr int CONV_A = 2 * CONV_HALF;
+constexpr int CONV_B = 2 * CONV_HALF;
 constexpr int CONV_BYTES = CONV_A + CONV_B;
 constexpr int LR_A = BM * 128;  // one low-rank chunk: up to 64 bf16 per row
 constexpr int LR_B = BN * 128;
 constexpr int EPI_WARPS = 8;  // two per tensor-memory lane quarter, 64 columns each
 constexpr int EPI_COLS = BN / 2;
-constexpr int THREADS = (6 + EPI_WARPS) * 32;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int CONV_WARPS = 2;
+constexpr int EPI_WARP0 = 2 + CONV_WARPS;
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;  // 12 warps: 3 per scheduler, up to 168 registers each
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int NACC = 4;  // accumulator buffers
+constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23 as binary32
+constexpr float MAGIC = 12582912.0f;
 constexpr uint32_t IDESC_S8 = idesc_s8_s32(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
 
@@ -67,7 +79,7 @@ struct I4Params {
   int n_lr;
   int lr_off[4], lr_w[4];
   const __half* sx;  // [K/64, M]
-  const __half* sw;  // [K/64, N]
+  const float* sw;   // [K/64, N], fp16 group scales widened to f32
   const float* bias;
   uint16_t* Y;
   int32_t* acc_dbg;  // [K/64, M, N] or null
@@ -76,6 +88,36 @@ struct I4Params {
 };
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
+
+// 32 lanes x 32 columns of tensor memory <- the magic integer
+__device__ __forceinline__ void tmem_fill_magic(uint32_t taddr) {
+  const uint32_t v = MAGIC_BITS;
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ void sub2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "sub.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "mul.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
+}
+// (y0, y1) += (a0, a1) * (b0, b1), one rounding each
+__device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\tmov.b64 z, {%0, %1};\n\t"
+      "fma.rn.f32x2 z, x, y, z;\n\tmov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(y0), "+f"(y1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -102,9 +144,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   uint64_t* conv_empty = conv_full + CONV_STAGES;
   uint64_t* lr_full = conv_empty + CONV_STAGES;
   uint64_t* lr_empty = lr_full + 1;
-  uint64_t* acc_full = lr_empty + 1;  // [2]
-  uint64_t* acc_empty = acc_full + 2;  // [2]
-  uint64_t* mma_done = acc_empty + 2;
+  uint64_t* acc_full = lr_empty + 1;      // [NACC]
+  uint64_t* acc_empty = acc_full + NACC;  // [NACC]
+  uint64_t* mma_done = acc_empty + NACC;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -114,15 +156,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < RAW_STAGES; ++s) {
       mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], 4);
+      mbar_init(&raw_empty[s], CONV_WARPS);
     }
     for (int s = 0; s < CONV_STAGES; ++s) {
-      mbar_init(&conv_full[s], 4);
+      mbar_init(&conv_full[s], CONV_WARPS);
       mbar_init(&conv_empty[s], 1);
     }
     mbar_init(lr_full, 1);
     mbar_init(lr_empty, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], EPI_WARPS * 32);
     }
@@ -138,6 +180,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp >= EPI_WARP0) {  // every accumulator starts at the magic integer
+    const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(((warp - EPI_WARP0) >> 2) * EPI_COLS);
+    for (int b = 0; b < NACC; ++b) {
+      tmem_fill_magic(tq + b * BN);
+      tmem_fill_magic(tq + b * BN + 32);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -183,8 +236,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         if (p.n_lr > 0) {
-          const int b = unit & 1;
-          if (!mbar_wait(&acc_empty[b], ((unit >> 1) & 1) ^ 1, wc)) break;
+          const int b = unit % NACC;
+          if (!mbar_wait(&acc_empty[b], ((unit / NACC) & 1) ^ 1, wc)) break;
           tc_fence_after();
           uint32_t accum = 0;
           for (int u = 0; u < p.n_lr; ++u, ++lit) {
@@ -216,18 +269,18 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(conv + s * CONV_BYTES), b_addr = a_addr + CONV_A;
-          for (int g = 0; g < 2; ++g, ++unit) {
-            const int b = unit & 1;
-            if (!mbar_wait(&acc_empty[b], ((unit >> 1) & 1) ^ 1, wc)) {
+          for (int g = 0; g < GPS; ++g, ++unit) {
+            const int b = unit % NACC;
+            if (!mbar_wait(&acc_empty[b], ((unit / NACC) & 1) ^ 1, wc)) {
               ok = false;
               break;
             }
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
-              const uint32_t off = 64 * g + 32 * kk;
+              const uint32_t off = (g >> 1) * CONV_HALF + 64 * (g & 1) + 32 * kk;
               mma_s8(tmem + b * BN, make_sdesc(a_addr + off, 16, 1024, LAYOUT_SW128),
-                     make_sdesc(b_addr + off, 16, 1024, LAYOUT_SW128), IDESC_S8, kk);
+                     make_sdesc(b_addr + off, 16, 1024, LAYOUT_SW128), IDESC_S8, 1u);
             }
             umma_commit(&acc_full[b]);
           }
@@ -237,9 +290,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
       umma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, p.limit);
     }
-  } else if (warp < 6) {
+  } else if (warp < EPI_WARP0) {
     // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - 64;  // 0..127
+    const int ct = threadIdx.x - 64;  // 0..CONV_WARPS*32-1
     int rit = 0, cit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
@@ -251,16 +304,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
         const uint8_t* src = raw + rs * RAW_BYTES;
         uint8_t* dst = conv + cs * CONV_BYTES;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {  // A then B
-          const uint8_t* sh = src + half * RAW_A;
-          uint8_t* dh = dst + half * CONV_A;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int id = i * 128 + ct;
-            const int row = id >> 3, chunk = id & 7;
-            const uint2 pk = *(const uint2*)(sh + row * (BK / 2) + chunk * 8);
+        for (int op = 0; op < 2; ++op) {  // A then B
+          const uint8_t* sh = src + op * RAW_A;
+          uint8_t* dh = dst + op * CONV_A;
+#pragma unroll 4
+          for (int i = 0; i < (BM * 16) / (CONV_WARPS * 32); ++i) {
+            const int id = i * (CONV_WARPS * 32) + ct;
+            const int row = id >> 4, c8 = id & 15;  // 8 packed bytes = 16 codes
+            const uint2 pk = *(const uint2*)(sh + row * 128 + ((((c8 >> 1) ^ (row & 7)) << 4) | ((c8 & 1) << 3)));
             const uint2 w0 = widen8(pk.x), w1 = widen8(pk.y);
-            *(uint4*)(dh + row * BK + ((chunk ^ (row & 7)) << 4)) = make_uint4(w0.x, w0.y, w1.x, w1.y);
+            *(uint4*)(dh + (c8 >> 3) * CONV_HALF + row * 128 + (((c8 & 7) ^ (row & 7)) << 4)) =
+                make_uint4(w0.x, w0.y, w1.x, w1.y);
           }
         }
         fence_async_smem();
@@ -274,7 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int half = (warp - 6) >> 2;
+    const int half = (warp - EPI_WARP0) >> 2;
     const int row = 32 * q + lane;
     int unit = 0;
     bool ok = true;
@@ -287,8 +341,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
 #pragma unroll
       for (int j = 0; j < EPI_COLS; ++j) y[j] = 0.f;
       if (p.n_lr > 0) {
-        const int b = unit & 1;
-        if (!mbar_wait(&acc_full[b], (unit >> 1) & 1, wc)) break;
+        const int b = unit % NACC;
+        if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) break;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < EPI_COLS / 32; ++c) {
@@ -298,28 +352,27 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
 #pragma unroll
           for (int j = 0; j < 32; ++j) y[32 * c + j] = __uint_as_float(r[j]);
         }
+        tmem_fill_magic(tl + b * BN);  // re-arm for an integer unit
+        tmem_fill_magic(tl + b * BN + 32);
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
         ++unit;
       }
       for (int g = 0; g < p.groups; ++g, ++unit) {
-        const int b = unit & 1;
-        if (!mbar_wait(&acc_full[b], (unit >> 1) & 1, wc)) {
+        const int b = unit % NACC;
+        if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const float sx = (m < p.M) ? __half2float(p.sx[(size_t)g * p.M + m]) : 0.f;
-        const __half* swg = p.sw + (size_t)g * p.N + n0;
+        const float* swg = p.sw + (size_t)g * p.N + n0;
 #pragma unroll
         for (int c = 0; c < EPI_COLS / 32; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tl + b * BN + 32 * c, r);
           tmem_ld_wait();
-          if (c == EPI_COLS / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(&acc_empty[b]);
-          }
           if (DBG) {
             if (m < p.M) {
 #pragma unroll
@@ -327,35 +380,31 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
                 const int n = n0 + 32 * c + j;
                 if (n < p.N)
                   *(uint4*)(p.acc_dbg + ((size_t)g * p.M + m) * p.N + n) =
-                      make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+                      make_uint4(r[j] - MAGIC_BITS, r[j + 1] - MAGIC_BITS, r[j + 2] - MAGIC_BITS, r[j + 3] - MAGIC_BITS);
               }
             }
           } else {
 #pragma unroll
-            for (int j8 = 0; j8 < 4; ++j8) {
-              const int n = n0 + 32 * c + 8 * j8;
-              float s[8];
-              if (n < p.N) {
-                const uint4 hv = __ldg((const uint4*)(swg + 32 * c + 8 * j8));
-                const __half2* h2 = (const __half2*)&hv;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 f = __half22float2(h2[e]);
-                  s[2 * e] = f.x;
-                  s[2 * e + 1] = f.y;
-                }
-              } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) s[e] = 0.f;
-              }
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int j = 32 * c + 8 * j8 + e;
-                y[j] = fmaf(sx * s[e], (float)(int)r[8 * j8 + e], y[j]);
-              }
+            for (int j = 0; j < 32; j += 4) {
+              const int n = n0 + 32 * c + j;
+              const float4 w4 = (n < p.N) ? __ldg((const float4*)(swg + 32 * c + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+              float f0 = __uint_as_float(r[j]), f1 = __uint_as_float(r[j + 1]);
+              float f2 = __uint_as_float(r[j + 2]), f3 = __uint_as_float(r[j + 3]);
+              sub2(f0, f1, MAGIC, MAGIC);  // exact: the group's integer sums
+              sub2(f2, f3, MAGIC, MAGIC);
+              float s0 = w4.x, s1 = w4.y, s2 = w4.z, s3 = w4.w;
+              mul2(s0, s1, sx, sx);
+              mul2(s2, s3, sx, sx);
+              fma2(y[32 * c + j], y[32 * c + j + 1], s0, s1, f0, f1);
+              fma2(y[32 * c + j + 2], y[32 * c + j + 3], s2, s3, f2, f3);
             }
           }
         }
+        tmem_fill_magic(tl + b * BN);  // re-arm this accumulator
+        tmem_fill_magic(tl + b * BN + 32);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&acc_empty[b]);
       }
       if (!ok) break;
       if (!DBG && m < p.M) {
@@ -407,7 +456,7 @@ int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const
   std::memset(&maps, 0, sizeof(maps));
   const int K = (int)L->K, N = (int)L->N, r = L->rank;
   int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
-                          (uint64_t)K / 2, BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+                          (uint64_t)K / 2, BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != SVDQ_OK) return st;
   maps.b = L->map_w;
   I4Params p{};
@@ -438,7 +487,7 @@ int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const
   p.k_stages = K / BK;
   p.groups = K / 64;
   p.sx = (const __half*)(ws + w.scales);
-  p.sw = (const __half*)L->wscales;
+  p.sw = (const float*)L->wscales;
   p.bias = L->bias;
   p.Y = (uint16_t*)Y;
   p.acc_dbg = acc_dbg;

@@ -59,7 +59,7 @@ Blob blob_layout(int64_t N, int64_t K, int rank, int fmt) {
     const size_t tiles = (size_t)((N + kNvfp4BN - 1) / kNvfp4BN);
     o = align_up(o + tiles * (size_t)(K / 64) * 2 * kSfAtomBytes, kAlign);
   } else {
-    o = align_up(o + (size_t)(K / 64) * N * 2, kAlign);
+    o = align_up(o + (size_t)(K / 64) * N * 4, kAlign);
   }
   b.total = o;
   return b;
@@ -220,10 +220,10 @@ svdq_status svdq_pack(const svdq_canonical* c, void* blob_v, size_t blob_bytes) 
       for (int64_t blk = 0; blk < B; ++blk) blob[b.wscales + sf_offset(n, blk, K / 64, kNvfp4BN)] = s[n * B + blk];
   } else {
     const uint16_t* s = (const uint16_t*)c->wscales;
-    uint16_t* d = (uint16_t*)(blob + b.wscales);
+    float* d = (float*)(blob + b.wscales);
     const int64_t G = K / 64;
     for (int64_t n = 0; n < N; ++n)
-      for (int64_t g = 0; g < G; ++g) d[g * N + n] = s[n * G + g];
+      for (int64_t g = 0; g < G; ++g) d[g * N + n] = host::f16_to_f32(s[n * G + g]);  // exact
   }
   return SVDQ_OK;
 }
@@ -282,9 +282,9 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   if (fmt == SVDQ_NVFP4_G16)  // 256 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
                        (uint64_t)K / 2, 128, kNvfp4BN, CU_TENSOR_MAP_SWIZZLE_128B);
-  else  // 128 packed codes (64 B) per row per stage, widened to int8 in shared memory
+  else  // 256 packed codes (128 B) per row per stage, widened to int8 in shared memory
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
-                       (uint64_t)K / 2, 64, kInt4BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+                       (uint64_t)K / 2, 128, kInt4BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e == SVDQ_OK && rank > 0) {
     e = encode_tmap_2d(&L->map_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L1t, (uint64_t)K, (uint64_t)rank,
                        (uint64_t)K * 2, 64, (uint32_t)rank, CU_TENSOR_MAP_SWIZZLE_128B);

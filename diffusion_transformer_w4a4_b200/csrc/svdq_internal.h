@@ -100,6 +100,7 @@ namespace host {
 int prepare(const uint16_t* W, const uint16_t* bias, const float* act_absmax, float alpha, svdq_canonical* c);
 uint16_t f32_to_bf16(float f);
 float bf16_to_f32(uint16_t h);
+float f16_to_f32(uint16_t h);
 }  // namespace host
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda).

@@ -122,7 +122,7 @@ svdq_status svdq_packed_size(int64_t N, int64_t K, int rank, int fmt, size_t* by
  *   inv_lambda f32 [K] | L1^T bf16 [rank, K] | L2^T bf16 [N, rank] (NVFP4: times
  *   1/(g_x g_w), an exact power of two) | bias f32 [N] | wcodes u8 [N, K/2] |
  *   wscales: NVFP4 -> E4M3 in 192-row tiles of the tensor-core scale-factor
- *   layout, INT4 -> fp16 [K/64, N]. */
+ *   layout, INT4 -> the fp16 group scales widened exactly to f32, [K/64, N]. */
 svdq_status svdq_pack(const svdq_canonical* c, void* blob, size_t blob_bytes);
 
 /* ------------------------------------------------------------------------ */

@@ -185,6 +185,7 @@ def test_pack_layout(lib, fmt):
         return start
     o_il, o_l1, o_l2, o_b, o_wc = take(K * 4), take(r * K * 2), take(N * r * 2), take(N * 4), take(N * K // 2)
     o_ws = o
+    assert blob.size == (o + (N * K // 64 * 4 if fmt == "int4" else (N + 191) // 192 * (K // 64) * 1024) + 1023) // 1024 * 1024
     assert np.array_equal(blob[o_il:o_il + 4 * K].view(np.float32), c["inv_lambda"])
     assert np.array_equal(blob[o_l1:o_l1 + 2 * r * K].view(np.uint16).reshape(r, K), c["L1"].T)
     l2t = oracle.bf16_to_f32(blob[o_l2:o_l2 + 2 * N * r].view(np.uint16).reshape(N, r)).astype(np.float64)
@@ -193,8 +194,8 @@ def test_pack_layout(lib, fmt):
     assert np.array_equal(blob[o_b:o_b + 4 * N].view(np.float32), oracle.bf16_to_f32(c["bias"]))
     assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"])
     if fmt == "int4":
-        ws = blob[o_ws:o_ws + N * K // 64 * 2].view(np.uint16).reshape(K // 64, N)
-        assert np.array_equal(ws, c["wscales"].T)
+        ws = blob[o_ws:o_ws + N * K // 64 * 4].view(np.float32).reshape(K // 64, N)
+        assert np.array_equal(ws, c["wscales"].T.view(np.float16).astype(np.float32))
     else:
         rows, blocks = np.meshgrid(np.arange(N), np.arange(K // 16), indexing="ij")
         offs = _sf_offset(rows, blocks, K // 64, 192)
