@@ -1,36 +1,35 @@
 // K3: INT4 W4A4 GEMM of the svdq_w4a4 layer on 5th-generation tensor cores.
 //
 //   Y = t . L2  +  sum_g  s_x[m,g] s_w[n,g] acc_g[m,n]  +  b,
-//   acc_g[m,n] = sum_{k in group g} qx[m,k] qw[n,k]   (exact int32)
+//   acc_g[m,n] = sum_{k in group g} qx[m,k] qw[n,k]   (an exact integer)
 //
 // "Суть метода" ("Hugging Face встроила Nunchaku в Diffusers ...") with the INT4
 // variant of the next paragraph: signed 4-bit codes in groups of 64 along K with
-// fp16 group scales.  Tensor cores have no 4-bit integer kind, so the packed
-// codes are widened to int8 in shared memory and multiplied with
-// tcgen05.mma kind::i8 (int32 accumulation).  Because both scales change every
-// 64 columns of K, each group's int32 accumulator is drained and rescaled by
-// the epilogue warps into an fp32 running sum held in registers, while the
-// tensor core fills the next of four accumulators.  Every accumulator starts
-// at the integer 0x4B400000, the bit pattern of 1.5 * 2^23: after adding a
-// group sum (|sum| <= 64 * 8 * 8 = 4096) the int32 result read as binary32 is
-// exactly 1.5 * 2^23 + sum, so one packed subtraction recovers the sum as a
-// float without an integer-to-float conversion.
+// fp16 group scales.  Tensor cores have no 4-bit integer kind.  Every integer
+// of [-8, 7] is exact in FP8 E4M3, so the activation quantizer and the weight
+// packer store each code as the E4M3 byte of its value and the group products
+// run as tcgen05.mma kind::f8f6f4 with an f32 accumulator: the products are
+// integers of magnitude <= 64 and a group's sum is an integer of magnitude
+// <= 4096, all exact in binary32, so the accumulator holds acc_g exactly.
+// Because both scales change every 64 columns of K, each group's accumulator is
+// drained by the epilogue warps into an fp32 running sum held in registers,
+// y += (s_x s_w) acc_g, while the tensor core fills the next of four
+// accumulators.  The drain is the kernel's bound: two fp32 operations per
+// output and group against one 128 x 128 x 64 MMA.
 //
 // Persistent, warp-specialized CTA (one per SM), tile 128 x 128:
-//   warp 0      TMA producer: packed codes [128 x 128 B] (128-byte swizzle)
-//               for A and B per 256-column K stage (raw ring), and the bf16
-//               t / L2^T chunks of the low-rank branch (own buffer).
+//   warp 0      TMA producer: E4M3 codes [128 x 128 B] (128-byte swizzle) for
+//               A and B per 128-column K stage (two groups); the two groups'
+//               scales (f32 s_w [2 x 128], fp16 s_x [2 x 128]) into a ring of
+//               their own; the bf16 t / L2^T chunks of the low-rank branch.
 //   warp 1      owns tensor memory (4 x 128 columns) and issues the MMAs:
 //               kind::f16 for t . L2 (its own accumulator unit, which seeds the
-//               running sum), then 2 x kind::i8 (K=32) per 64-group, four
-//               groups per stage.
-//   warps 2-3   converters: raw int4 -> int8, sign-extended, written in the
-//               128-byte-swizzled K-major layout the MMA reads (conv ring).
-//   warps 4-11  epilogue (two per lane quarter, 64 columns each): tcgen05.ld
-//               each unit; y += s_x s_w float(acc);
+//               running sum), then 2 x kind::f8f6f4 (K = 32) per group.
+//   warps 2-9   epilogue (two per lane quarter, 64 columns each): tcgen05.ld
+//               each unit; y += (s_x s_w) acc in packed f32x2 arithmetic;
 //               bias, bf16 round-to-nearest-even, 16-byte stores.  With a
-//               debug output pointer it instead writes the raw int32 group
-//               accumulators (integer-path parity).
+//               debug output pointer it instead writes the group accumulators
+//               as int32 (integer-path parity).
 // Every wait is bounded (sm100.cuh); no load uses cluster multicast.
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -45,41 +44,38 @@ namespace {
 
 constexpr int BM = kGemmBM;  // 128
 constexpr int BN = kInt4BN;  // 128
-constexpr int BK = 256;      // K elements per stage (4 groups of 64)
-constexpr int GPS = BK / 64;  // groups per stage
-constexpr int RAW_STAGES = 2;
-constexpr int CONV_STAGES = 2;
-constexpr int RAW_A = BM * BK / 2;  // 16 KiB packed, one 128-byte swizzled row per token
-constexpr int RAW_B = BN * BK / 2;
-constexpr int RAW_BYTES = RAW_A + RAW_B;
-constexpr int CONV_HALF = BM * 128;  // int8 sub-tile of 128 K columns, 128-byte swizzled
-constexpr int CONV_A = 2 * CONV_HALF;
-constexpr int CONV_B = 2 * CONV_HALF;
-constexpr int CONV_BYTES = CONV_A + CONV_B;
+constexpr int BK = 128;      // K codes (bytes) per stage: two groups of 64
+constexpr int GPS = BK / 64;
+constexpr int STAGES = 5;
+constexpr int STAGE_A = BM * BK;  // 16 KiB, one 128-byte swizzled row per token
+constexpr int STAGE_B = BN * BK;
+constexpr int STAGE_BYTES = STAGE_A + STAGE_B;
 constexpr int LR_A = BM * 128;  // one low-rank chunk: up to 64 bf16 per row
 constexpr int LR_B = BN * 128;
+constexpr int SC_SLOTS = 8;                   // scale ring: one slot per K stage
+constexpr int SC_SW = GPS * BN * 4;           // f32 s_w [GPS][BN]
+constexpr int SC_SX = GPS * BM * 2;           // fp16 s_x [GPS][BM]
+constexpr int SC_BYTES = SC_SW + SC_SX;       // 1.5 KiB, a multiple of 128
 constexpr int EPI_WARPS = 8;  // two per tensor-memory lane quarter, 64 columns each
 constexpr int EPI_COLS = BN / 2;
-constexpr int CONV_WARPS = 2;
-constexpr int EPI_WARP0 = 2 + CONV_WARPS;
-constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;  // 12 warps: 3 per scheduler, up to 168 registers each
+constexpr int EPI_WARP0 = 2;
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;  // 10 warps: up to 200 registers each
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NACC = 4;  // accumulator buffers
-constexpr uint32_t MAGIC_BITS = 0x4B400000u;  // 1.5 * 2^23 as binary32
-constexpr float MAGIC = 12582912.0f;
-constexpr uint32_t IDESC_S8 = idesc_s8_s32(BM, BN);
+constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + LR_A + LR_B + (size_t)SC_SLOTS * SC_BYTES + 256;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(SC_SW % 128 == 0 && SC_BYTES % 128 == 0, "TMA destinations stay 128-byte aligned");
 
 struct I4Maps {
-  CUtensorMap a, b, t[3], l2[3];
+  CUtensorMap a, b, sw, sx, t[3], l2[3];
 };
 
 struct I4Params {
-  int M, N, K, m_tiles, n_tiles, num_tiles, k_stages, groups;
+  int M, N, K, m_tiles, n_tiles, num_tiles, k_stages;
   int n_lr;
   int lr_off[4], lr_w[4];
-  const __half* sx;  // [K/64, M]
-  const float* sw;   // [K/64, N], fp16 group scales widened to f32
   const float* bias;
   uint16_t* Y;
   int32_t* acc_dbg;  // [K/64, M, N] or null
@@ -89,22 +85,6 @@ struct I4Params {
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
 
-// 32 lanes x 32 columns of tensor memory <- the magic integer
-__device__ __forceinline__ void tmem_fill_magic(uint32_t taddr) {
-  const uint32_t v = MAGIC_BITS;
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-
-__device__ __forceinline__ void sub2(float& a0, float& a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
-      "sub.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(b0), "f"(b1));
-}
 __device__ __forceinline__ void mul2(float& a0, float& a1, float b0, float b1) {
   asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
       "mul.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
@@ -119,30 +99,31 @@ __device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 8 packed nibbles (two's complement, element 2i in the low nibble of byte i)
-// -> 8 sign-extended int8, in element order, as two words.
-__device__ __forceinline__ uint2 widen8(uint32_t w) {
-  const uint32_t lo = __vsub4((w & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);         // elements 0,2,4,6
-  const uint32_t hi = __vsub4(((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);  // elements 1,3,5,7
-  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+// y[0..31] += (sx * sw[0..31]) * acc[0..31]
+__device__ __forceinline__ void drain32(float* y, const uint32_t (&r)[32], const float* sw, float sx) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 w4 = *(const float4*)(sw + j);  // the same address in every lane: a broadcast
+    float c0 = w4.x, c1 = w4.y, c2 = w4.z, c3 = w4.w;
+    mul2(c0, c1, sx, sx);  // exact: a product of two fp16 values
+    mul2(c2, c3, sx, sx);
+    fma2(y[j], y[j + 1], c0, c1, __uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+    fma2(y[j + 2], y[j + 3], c2, c3, __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+  }
 }
 
 template <bool DBG>
 __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant__ I4Maps maps, const I4Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* conv = smem;                                // [CONV_STAGES][CONV_BYTES]  (1024-aligned)
-  uint8_t* lrbuf = conv + CONV_STAGES * CONV_BYTES;    // [LR_A + LR_B]
-  uint8_t* raw = lrbuf + LR_A + LR_B;                  // [RAW_STAGES][RAW_BYTES]
-  uint64_t* raw_full = (uint64_t*)(raw + RAW_STAGES * RAW_BYTES);
-  uint64_t* raw_empty = raw_full + RAW_STAGES;
-  uint64_t* conv_full = raw_empty + RAW_STAGES;
-  uint64_t* conv_empty = conv_full + CONV_STAGES;
-  uint64_t* lr_full = conv_empty + CONV_STAGES;
+  uint8_t* stages = smem;                             // [STAGES][STAGE_BYTES]  (1024-aligned)
+  uint8_t* lrbuf = stages + STAGES * STAGE_BYTES;     // [LR_A + LR_B]
+  uint8_t* scring = lrbuf + LR_A + LR_B;              // [SC_SLOTS][SC_BYTES]
+  uint64_t* full = (uint64_t*)(scring + SC_SLOTS * SC_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* sc_full = empty + STAGES;
+  uint64_t* sc_empty = sc_full + SC_SLOTS;
+  uint64_t* lr_full = sc_empty + SC_SLOTS;
   uint64_t* lr_empty = lr_full + 1;
   uint64_t* acc_full = lr_empty + 1;      // [NACC]
   uint64_t* acc_empty = acc_full + NACC;  // [NACC]
@@ -154,13 +135,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   WaitCtl wc{abort_flag, p.status, p.limit};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < RAW_STAGES; ++s) {
-      mbar_init(&raw_full[s], 1);
-      mbar_init(&raw_empty[s], CONV_WARPS);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    for (int s = 0; s < CONV_STAGES; ++s) {
-      mbar_init(&conv_full[s], CONV_WARPS);
-      mbar_init(&conv_empty[s], 1);
+    for (int s = 0; s < SC_SLOTS; ++s) {
+      mbar_init(&sc_full[s], 1);
+      mbar_init(&sc_empty[s], EPI_WARPS);
     }
     mbar_init(lr_full, 1);
     mbar_init(lr_empty, 1);
@@ -180,24 +161,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp >= EPI_WARP0) {  // every accumulator starts at the magic integer
-    const uint32_t tq = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(((warp - EPI_WARP0) >> 2) * EPI_COLS);
-    for (int b = 0; b < NACC; ++b) {
-      tmem_fill_magic(tq + b * BN);
-      tmem_fill_magic(tq + b * BN + 32);
-    }
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&maps.a);
       prefetch_tmap(&maps.b);
-      int rit = 0, lit = 0;
+      prefetch_tmap(&maps.sw);
+      prefetch_tmap(&maps.sx);
+      int it = 0, sit = 0, lit = 0;  // operand stages, scale stages, low-rank chunks issued
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
@@ -211,28 +183,40 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
           tma_load_2d(&maps.t[mi], lr_full, lrbuf, p.lr_off[u], mt * BM);
           tma_load_2d(&maps.l2[mi], lr_full, lrbuf + LR_A, p.lr_off[u], nt * BN);
         }
-        for (int ks = 0; ks < p.k_stages && ok; ++ks, ++rit) {
-          const int s = rit % RAW_STAGES;
-          if (!mbar_wait(&raw_empty[s], ((rit / RAW_STAGES) & 1) ^ 1, wc)) {
+        for (int ks = 0; ks < p.k_stages && ok; ++ks) {
+          const int s = it % STAGES, ss = sit % SC_SLOTS;
+          if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
             ok = false;
             break;
           }
-          uint8_t* st = raw + s * RAW_BYTES;
-          mbar_arrive_expect_tx(&raw_full[s], RAW_BYTES);
-          tma_load_2d(&maps.a, &raw_full[s], st, ks * (BK / 2), mt * BM);
-          tma_load_2d(&maps.b, &raw_full[s], st + RAW_A, ks * (BK / 2), nt * BN);
+          uint8_t* st = stages + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(&maps.a, &full[s], st, ks * BK, mt * BM);
+          tma_load_2d(&maps.b, &full[s], st + STAGE_A, ks * BK, nt * BN);
+          ++it;
+          if (!mbar_wait(&sc_empty[ss], ((sit / SC_SLOTS) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sc = scring + ss * SC_BYTES;
+          mbar_arrive_expect_tx(&sc_full[ss], SC_BYTES);
+          tma_load_2d(&maps.sw, &sc_full[ss], sc, nt * BN, ks * GPS);
+          tma_load_2d(&maps.sx, &sc_full[ss], sc + SC_SW, mt * BM, ks * GPS);
+          ++sit;
         }
       }
       if (!ok) {  // drain copies still in flight
-        for (int j = (rit > RAW_STAGES ? rit - RAW_STAGES : 0); j < rit; ++j)
-          mbar_wait_drain(&raw_full[j % RAW_STAGES], (j / RAW_STAGES) & 1, p.limit);
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, p.limit);
+        for (int j = (sit > SC_SLOTS ? sit - SC_SLOTS : 0); j < sit; ++j)
+          mbar_wait_drain(&sc_full[j % SC_SLOTS], (j / SC_SLOTS) & 1, p.limit);
         if (lit > 0) mbar_wait_drain(lr_full, (lit - 1) & 1, p.limit);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int cit = 0, lit = 0, unit = 0;
+      int it = 0, lit = 0, unit = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         if (p.n_lr > 0) {
@@ -261,14 +245,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
           umma_commit(&acc_full[b]);
           ++unit;
         }
-        for (int ks = 0; ks < p.k_stages && ok; ++ks, ++cit) {
-          const int s = cit % CONV_STAGES;
-          if (!mbar_wait(&conv_full[s], (cit / CONV_STAGES) & 1, wc)) {
+        for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, wc)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(conv + s * CONV_BYTES), b_addr = a_addr + CONV_A;
+          const uint32_t a_addr = smem_u32(stages + s * STAGE_BYTES), b_addr = a_addr + STAGE_A;
           for (int g = 0; g < GPS; ++g, ++unit) {
             const int b = unit % NACC;
             if (!mbar_wait(&acc_empty[b], ((unit / NACC) & 1) ^ 1, wc)) {
@@ -277,60 +261,25 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
             }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const uint32_t off = (g >> 1) * CONV_HALF + 64 * (g & 1) + 32 * kk;
-              mma_s8(tmem + b * BN, make_sdesc(a_addr + off, 16, 1024, LAYOUT_SW128),
-                     make_sdesc(b_addr + off, 16, 1024, LAYOUT_SW128), IDESC_S8, 1u);
+            for (int kk = 0; kk < 2; ++kk) {  // K = 32 codes (bytes) per instruction
+              const uint32_t off = 64 * g + 32 * kk;
+              mma_f8f6f4(tmem + b * BN, make_sdesc(a_addr + off, 16, 1024, LAYOUT_SW128),
+                         make_sdesc(b_addr + off, 16, 1024, LAYOUT_SW128), IDESC_E4M3, (uint32_t)kk);
             }
             umma_commit(&acc_full[b]);
           }
-          umma_commit(&conv_empty[s]);
+          umma_commit(&empty[s]);
         }
       }
       umma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, p.limit);
-    }
-  } else if (warp < EPI_WARP0) {
-    // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - 64;  // 0..CONV_WARPS*32-1
-    int rit = 0, cit = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-      for (int ks = 0; ks < p.k_stages; ++ks, ++rit, ++cit) {
-        const int rs = rit % RAW_STAGES, cs = cit % CONV_STAGES;
-        ok = mbar_wait(&raw_full[rs], (rit / RAW_STAGES) & 1, wc) &&
-             mbar_wait(&conv_empty[cs], ((cit / CONV_STAGES) & 1) ^ 1, wc);
-        if (!ok) break;
-        const uint8_t* src = raw + rs * RAW_BYTES;
-        uint8_t* dst = conv + cs * CONV_BYTES;
-#pragma unroll
-        for (int op = 0; op < 2; ++op) {  // A then B
-          const uint8_t* sh = src + op * RAW_A;
-          uint8_t* dh = dst + op * CONV_A;
-#pragma unroll 4
-          for (int i = 0; i < (BM * 16) / (CONV_WARPS * 32); ++i) {
-            const int id = i * (CONV_WARPS * 32) + ct;
-            const int row = id >> 4, c8 = id & 15;  // 8 packed bytes = 16 codes
-            const uint2 pk = *(const uint2*)(sh + row * 128 + ((((c8 >> 1) ^ (row & 7)) << 4) | ((c8 & 1) << 3)));
-            const uint2 w0 = widen8(pk.x), w1 = widen8(pk.y);
-            *(uint4*)(dh + (c8 >> 3) * CONV_HALF + row * 128 + (((c8 & 7) ^ (row & 7)) << 4)) =
-                make_uint4(w0.x, w0.y, w1.x, w1.y);
-          }
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&conv_full[cs]);
-          mbar_arrive(&raw_empty[rs]);
-        }
-      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int half = (warp - EPI_WARP0) >> 2;
     const int row = 32 * q + lane;
-    int unit = 0;
+    int it = 0, unit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
@@ -344,67 +293,61 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
         const int b = unit % NACC;
         if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) break;
         tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(tl + b * BN, r0);
+        tmem_ld_32x32b_x32(tl + b * BN + 32, r1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < EPI_COLS / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tl + b * BN + 32 * c, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[32 * c + j] = __uint_as_float(r[j]);
+        for (int j = 0; j < 32; ++j) {
+          y[j] = __uint_as_float(r0[j]);
+          y[32 + j] = __uint_as_float(r1[j]);
         }
-        tmem_fill_magic(tl + b * BN);  // re-arm for an integer unit
-        tmem_fill_magic(tl + b * BN + 32);
-        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
         ++unit;
       }
-      for (int g = 0; g < p.groups; ++g, ++unit) {
-        const int b = unit % NACC;
-        if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) {
+      for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+        const int ss = it % SC_SLOTS;
+        if (!mbar_wait(&sc_full[ss], (it / SC_SLOTS) & 1, wc)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const float sx = (m < p.M) ? __half2float(p.sx[(size_t)g * p.M + m]) : 0.f;
-        const float* swg = p.sw + (size_t)g * p.N + n0;
-#pragma unroll
-        for (int c = 0; c < EPI_COLS / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(tl + b * BN + 32 * c, r);
+        const uint8_t* sc = scring + ss * SC_BYTES;
+        for (int g = 0; g < GPS; ++g, ++unit) {
+          const int b = unit % NACC;
+          if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tl + b * BN, r0);
+          tmem_ld_32x32b_x32(tl + b * BN + 32, r1);
           tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&acc_empty[b]);  // the accumulator is in registers now
           if (DBG) {
             if (m < p.M) {
+              const int gg = ks * GPS + g;
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const int n = n0 + 32 * c + j;
+              for (int j = 0; j < EPI_COLS; j += 4) {
+                const int n = n0 + j;
+                const uint32_t* rr = j < 32 ? r0 + j : r1 + (j - 32);
                 if (n < p.N)
-                  *(uint4*)(p.acc_dbg + ((size_t)g * p.M + m) * p.N + n) =
-                      make_uint4(r[j] - MAGIC_BITS, r[j + 1] - MAGIC_BITS, r[j + 2] - MAGIC_BITS, r[j + 3] - MAGIC_BITS);
+                  *(int4*)(p.acc_dbg + ((size_t)gg * p.M + m) * p.N + n) =
+                      make_int4(__float2int_rz(__uint_as_float(rr[0])), __float2int_rz(__uint_as_float(rr[1])),
+                                __float2int_rz(__uint_as_float(rr[2])), __float2int_rz(__uint_as_float(rr[3])));
               }
             }
           } else {
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const int n = n0 + 32 * c + j;
-              const float4 w4 = (n < p.N) ? __ldg((const float4*)(swg + 32 * c + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
-              float f0 = __uint_as_float(r[j]), f1 = __uint_as_float(r[j + 1]);
-              float f2 = __uint_as_float(r[j + 2]), f3 = __uint_as_float(r[j + 3]);
-              sub2(f0, f1, MAGIC, MAGIC);  // exact: the group's integer sums
-              sub2(f2, f3, MAGIC, MAGIC);
-              float s0 = w4.x, s1 = w4.y, s2 = w4.z, s3 = w4.w;
-              mul2(s0, s1, sx, sx);
-              mul2(s2, s3, sx, sx);
-              fma2(y[32 * c + j], y[32 * c + j + 1], s0, s1, f0, f1);
-              fma2(y[32 * c + j + 2], y[32 * c + j + 3], s2, s3, f2, f3);
-            }
+            const float sx = __half2float(((const __half*)(sc + SC_SW))[g * BM + row]);
+            const float* sw = (const float*)sc + g * BN + half * EPI_COLS;
+            drain32(y, r0, sw, sx);
+            drain32(y + 32, r1, sw + 32, sx);
           }
         }
-        tmem_fill_magic(tl + b * BN);  // re-arm this accumulator
-        tmem_fill_magic(tl + b * BN + 32);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&acc_empty[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sc_empty[ss]);
       }
       if (!ok) break;
       if (!DBG && m < p.M) {
@@ -455,8 +398,15 @@ int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const
   I4Maps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int K = (int)L->K, N = (int)L->N, r = L->rank;
-  int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
-                          (uint64_t)K / 2, BK / 2, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  const int64_t sld = int4_scale_ld(M);
+  int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K, (uint64_t)M, (uint64_t)K,
+                          BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SVDQ_OK) return st;
+  st = encode_tmap_2d(&maps.sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, L->wscales, (uint64_t)N, (uint64_t)K / 64,
+                      (uint64_t)N * 4, BN, GPS, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != SVDQ_OK) return st;
+  st = encode_tmap_2d(&maps.sx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws + w.scales, (uint64_t)sld, (uint64_t)K / 64,
+                      (uint64_t)sld * 2, BM, GPS, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != SVDQ_OK) return st;
   maps.b = L->map_w;
   I4Params p{};
@@ -485,24 +435,22 @@ int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const
   p.n_tiles = (N + BN - 1) / BN;
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.k_stages = K / BK;
-  p.groups = K / 64;
-  p.sx = (const __half*)(ws + w.scales);
-  p.sw = (const float*)L->wscales;
   p.bias = L->bias;
   p.Y = (uint16_t*)Y;
   p.acc_dbg = acc_dbg;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
-  const size_t smem = 1024 + (size_t)CONV_STAGES * CONV_BYTES + LR_A + LR_B + (size_t)RAW_STAGES * RAW_BYTES + 256;
   const int grid = p.num_tiles < sm_count_i4(L->device) ? p.num_tiles : sm_count_i4(L->device);
   if (acc_dbg) {
-    if (cudaFuncSetAttribute(k_gemm_int4<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_gemm_int4<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+        cudaSuccess)
       return SVDQ_ERR_CUDA;
-    k_gemm_int4<true><<<grid, THREADS, smem, stream>>>(maps, p);
+    k_gemm_int4<true><<<grid, THREADS, SMEM_BYTES, stream>>>(maps, p);
   } else {
-    if (cudaFuncSetAttribute(k_gemm_int4<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_gemm_int4<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+        cudaSuccess)
       return SVDQ_ERR_CUDA;
-    k_gemm_int4<false><<<grid, THREADS, smem, stream>>>(maps, p);
+    k_gemm_int4<false><<<grid, THREADS, SMEM_BYTES, stream>>>(maps, p);
   }
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }

@@ -105,6 +105,9 @@ float f16_to_f32(uint16_t h) {
   return s ? -v : v;
 }
 
+// The E4M3 byte of a small integer (exact for |v| <= 16).
+uint8_t int_to_e4m3(int v) { return f32_to_e4m3_sat((float)v); }
+
 // E4M3 (OCP FP8), saturating to +-448.
 uint8_t f32_to_e4m3_sat(float f) {
   if (std::isnan(f)) return 0x7F;

@@ -49,6 +49,7 @@ constexpr int kSmemBudget = 220 * 1024;
 
 struct QParams {
   int M, K, xstages, lstages, nslices, nch, katoms;
+  int64_t sld;  // INT4: row stride of the fp16 [K/64, sld] scales
   const float* inv_lambda;
   float g, inv_g, den;  // NVFP4 per-tensor scale, its exact inverse, 6*g
   uint8_t* codes;
@@ -89,6 +90,13 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
   return r & 0xFFu;
+}
+
+// two floats -> two E4M3 bytes, `lo` in bits 0..7
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ float e4m3_value(uint32_t c) {  // c in [0, 0x7E]
@@ -307,26 +315,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
             const float S16 = __half2float(s16);
+            uint32_t qb[4] = {0u, 0u, 0u, 0u};
             if (S16 != 0.f) {
               const float inv = __frcp_rn(S16);
-              uint32_t pk[2] = {0u, 0u};
 #pragma unroll
               for (int e = 0; e < 16; e += 2) {
                 float y0 = v[e], y1 = v[e + 1];
                 mul2(y0, y1, inv, inv);
-                // round half to even on the clamped value: the 4 low bits of
-                // (y + 1.5 * 2^23) are the two's-complement code
+                // clamp, then round half to even: (y + 1.5 * 2^23) - 1.5 * 2^23
+                // is the nearest integer (a +0 for codes of zero), and E4M3
+                // holds every integer of [-8, 7] exactly
                 y0 = fminf(fmaxf(y0, -8.0f), 7.0f);
                 y1 = fminf(fmaxf(y1, -8.0f), 7.0f);
-                const uint32_t c0 = __float_as_uint(__fadd_rn(y0, 12582912.0f)) & 0xFu;
-                const uint32_t c1 = __float_as_uint(__fadd_rn(y1, 12582912.0f)) & 0xFu;
-                pk[e >> 3] |= (c0 | (c1 << 4)) << (4 * (e & 7));
+                y0 = __fsub_rn(__fadd_rn(y0, 12582912.0f), 12582912.0f);
+                y1 = __fsub_rn(__fadd_rn(y1, 12582912.0f), 12582912.0f);
+                qb[e >> 2] |= cvt_e4m3x2(y0, y1) << (8 * (e & 2));
               }
-              packed = make_uint2(pk[0], pk[1]);
             }
-            if ((lane & 3) == 0 && m < p.M) ((__half*)p.scales)[(size_t)(kk0 / 64) * p.M + m] = s16;
+            if ((lane & 3) == 0 && m < p.M) ((__half*)p.scales)[(size_t)(kk0 / 64) * p.sld + m] = s16;
+            if (m < p.M) *(uint4*)(p.codes + (size_t)m * p.K + kk0) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
           }
-          if (m < p.M) *(uint2*)(p.codes + (size_t)m * K2 + kk0 / 2) = packed;
+          if (FMT == SVDQ_NVFP4_G16 && m < p.M) *(uint2*)(p.codes + (size_t)m * K2 + kk0 / 2) = packed;
           if constexpr (RANK > 0) {
             uint32_t b[8];
 #pragma unroll
@@ -475,6 +484,7 @@ int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, 
   p.nch = (int)(L->K / kChunk);
   p.nslices = w.nslices;
   p.katoms = (int)(L->K / 64);
+  p.sld = int4_scale_ld(M);
   p.inv_lambda = L->inv_lambda;
   p.g = L->g_x;
   p.inv_g = 1.0f / L->g_x;  // exact: g_x is a power of two

@@ -52,8 +52,8 @@ Blob blob_layout(int64_t N, int64_t K, int rank, int fmt) {
   o = align_up(o + (size_t)N * rank * 2, kAlign);
   b.bias = o;
   o = align_up(o + (size_t)N * 4, kAlign);
-  b.wcodes = o;
-  o = align_up(o + (size_t)N * K / 2, kAlign);
+  b.wcodes = o;  // NVFP4: packed E2M1 pairs; INT4: one E4M3 byte per code
+  o = align_up(o + (fmt == SVDQ_NVFP4_G16 ? (size_t)N * K / 2 : (size_t)N * K), kAlign);
   b.wscales = o;
   if (fmt == SVDQ_NVFP4_G16) {
     const size_t tiles = (size_t)((N + kNvfp4BN - 1) / kNvfp4BN);
@@ -70,13 +70,13 @@ Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M) {
   Workspace w{};
   size_t o = 0;
   w.codes = o;
-  w.codes_bytes = (size_t)M * K / 2;
+  w.codes_bytes = fmt == SVDQ_NVFP4_G16 ? (size_t)M * K / 2 : (size_t)M * K;
   o = align_up(o + w.codes_bytes, kAlign);
   w.scales = o;
   if (fmt == SVDQ_NVFP4_G16)
     w.scales_bytes = (size_t)((M + kSfAtomRows - 1) / kSfAtomRows) * (size_t)(K / 64) * kSfAtomBytes;
   else
-    w.scales_bytes = (size_t)(K / 64) * M * 2;
+    w.scales_bytes = (size_t)(K / 64) * (size_t)int4_scale_ld(M) * 2;
   o = align_up(o + w.scales_bytes, kAlign);
   w.t = o;
   w.t_bytes = (size_t)M * rank * 2;
@@ -212,7 +212,20 @@ svdq_status svdq_pack(const svdq_canonical* c, void* blob_v, size_t blob_bytes) 
     }
   float* bias = (float*)(blob + b.bias);
   for (int64_t n = 0; n < N; ++n) bias[n] = c->bias ? host::bf16_to_f32(c->bias[n]) : 0.f;
-  std::memcpy(blob + b.wcodes, c->wcodes, (size_t)N * K / 2);
+  if (fmt == SVDQ_NVFP4_G16) {
+    std::memcpy(blob + b.wcodes, c->wcodes, (size_t)N * K / 2);
+  } else {
+    // each two's-complement nibble becomes the E4M3 byte of the same integer,
+    // which the tensor core reads directly (every integer in [-8, 7] is exact)
+    uint8_t lut[16];
+    for (int v = 0; v < 16; ++v) lut[v] = host::int_to_e4m3(v < 8 ? v : v - 16);
+    const size_t nb = (size_t)N * K / 2;
+    uint8_t* d = blob + b.wcodes;
+    for (size_t i = 0; i < nb; ++i) {
+      d[2 * i] = lut[c->wcodes[i] & 15];
+      d[2 * i + 1] = lut[c->wcodes[i] >> 4];
+    }
+  }
   if (fmt == SVDQ_NVFP4_G16) {
     const uint8_t* s = (const uint8_t*)c->wscales;
     const int64_t B = K / 16;
@@ -282,9 +295,9 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   if (fmt == SVDQ_NVFP4_G16)  // 256 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
                        (uint64_t)K / 2, 128, kNvfp4BN, CU_TENSOR_MAP_SWIZZLE_128B);
-  else  // 256 packed codes (128 B) per row per stage, widened to int8 in shared memory
-    e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
-                       (uint64_t)K / 2, 128, kInt4BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  else  // 128 E4M3 codes (128 B) per row per stage, swizzled for the MMA
+    e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K, (uint64_t)N, (uint64_t)K,
+                       128, kInt4BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e == SVDQ_OK && rank > 0) {
     e = encode_tmap_2d(&L->map_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L1t, (uint64_t)K, (uint64_t)rank,
                        (uint64_t)K * 2, 64, (uint32_t)rank, CU_TENSOR_MAP_SWIZZLE_128B);

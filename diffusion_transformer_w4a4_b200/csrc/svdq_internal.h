@@ -47,6 +47,10 @@ struct Blob {  // offsets (bytes) of the packed-weight regions
 };
 Blob blob_layout(int64_t N, int64_t K, int rank, int fmt);
 
+// INT4 activation scales are fp16 [K/64, int4_scale_ld(M)]: each group's row is
+// padded to whole 128-token tiles so the GEMM can stage it with TMA.
+inline int64_t int4_scale_ld(int64_t M) { return (M + kQRows - 1) / kQRows * kQRows; }
+
 // Number of K slices the activation quantizer splits each 128-row block into,
 // so that about one CTA per SM is in flight; partial low-rank sums of the
 // slices are reduced in a fixed order.
@@ -101,6 +105,8 @@ int prepare(const uint16_t* W, const uint16_t* bias, const float* act_absmax, fl
 uint16_t f32_to_bf16(float f);
 float bf16_to_f32(uint16_t h);
 float f16_to_f32(uint16_t h);
+uint8_t f32_to_e4m3_sat(float f);
+uint8_t int_to_e4m3(int v);
 }  // namespace host
 
 // Tensor-map encoding through the driver entry point (no link-time libcuda).

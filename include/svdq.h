@@ -116,11 +116,15 @@ svdq_status svdq_prepare(const uint16_t* W, const uint16_t* bias, const float* a
 svdq_status svdq_packed_size(int64_t N, int64_t K, int rank, int fmt, size_t* bytes);
 
 /* Re-lay canonical weights into the blob the kernels read (a pure permutation
- * plus exact power-of-two rescaling; no rounding).  `blob` is host memory of
+ * plus exact re-encodings; no rounding).  `blob` is host memory of
  * svdq_packed_size bytes; copy it to the device (256-byte aligned) and pass the
  * device pointer to svdq_layer_create.  Layout, each region 1024-byte aligned:
  *   inv_lambda f32 [K] | L1^T bf16 [rank, K] | L2^T bf16 [N, rank] (NVFP4: times
- *   1/(g_x g_w), an exact power of two) | bias f32 [N] | wcodes u8 [N, K/2] |
+ *   1/(g_x g_w), an exact power of two) | bias f32 [N] |
+ *   wcodes: NVFP4 -> the packed E2M1 codes u8 [N, K/2]; INT4 -> one byte per
+ *   code, u8 [N, K], holding the FP8 E4M3 encoding of the code's integer value
+ *   (exact for every integer in [-8, 7]; the tensor cores of CC 10.0 have no
+ *   4-bit integer kind, so INT4 weights are held at one byte per code) |
  *   wscales: NVFP4 -> E4M3 in 192-row tiles of the tensor-core scale-factor
  *   layout, INT4 -> the fp16 group scales widened exactly to f32, [K/64, N]. */
 svdq_status svdq_pack(const svdq_canonical* c, void* blob, size_t blob_bytes);
@@ -143,8 +147,10 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
 void svdq_layer_destroy(svdq_layer* layer);
 
 /* Workspace for M tokens: quantized activations, low-rank t and a status word.
- * layout: offsets/sizes[0] act codes u8 [M, K/2]; [1] act scales (NVFP4: E4M3
- * in the tensor-core scale-factor layout of 128-row tiles; INT4: fp16 [K/64, M]);
+ * layout: offsets/sizes[0] act codes (NVFP4: packed E2M1 u8 [M, K/2]; INT4: one
+ * FP8 E4M3 byte per code holding its integer value, u8 [M, K]); [1] act scales
+ * (NVFP4: E4M3 in the tensor-core scale-factor layout of 128-row tiles; INT4:
+ * fp16 [K/64, M'], M' = M rounded up to a multiple of 128, columns >= M unused);
  * [2] t bf16 [M, rank]; [3] status word int32 (first word of a small control
  * block that also holds the quantizer's split-K counters).  The total size also
  * covers the quantizer's fp32 partial sums of t. */
@@ -192,7 +198,7 @@ svdq_status svdq_read_status(const svdq_layer* layer, int64_t M, const void* ws,
  * device array of 32 MiB, which exists once per GPU that loads the library and
  * stays allocated until the process exits.  Problems whose workspace
  * (svdq_workspace_size) exceeds 32 MiB return SVDQ_ERR_INVALID_ARG (e.g. at
- * K = 12288, rank 32: up to about 4300 tokens).  The first call on a device
+ * K = 12288, rank 32: up to 4480 tokens in NVFP4, 2458 in INT4).  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress), so make that
  * first call before any stream capture.  Each call zeroes the control block;
  * the array keeps the last call's contents otherwise.  All calls share the

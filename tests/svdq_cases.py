@@ -27,6 +27,19 @@ REL_L2 = 1e-3
 MAX_ABS = 2e-2
 
 
+def int4_bytes_to_packed(b: np.ndarray) -> np.ndarray:
+    """Device INT4 codes (one E4M3 byte per code, the byte of the code's
+    integer value) -> canonical packed two's-complement nibbles, element 2i in
+    the low nibble.  A byte that is not the E4M3 encoding of an integer in
+    [-8, 7] (a negative zero included) decodes to an out-of-range marker so the
+    bit-exact comparison fails."""
+    v = oracle.e4m3_to_f32(b.reshape(-1)).reshape(b.shape).astype(np.float64)
+    ok = (v == np.round(v)) & (v >= -8) & (v <= 7) & ~((b & 0x7F) == 0) | (b == 0)
+    assert ok.all(), f"{(~ok).sum()} device INT4 code bytes are not canonical E4M3 integers"
+    n = (v.astype(np.int64) & 15).astype(np.uint8)
+    return (n[:, 0::2] | (n[:, 1::2] << 4)).astype(np.uint8)
+
+
 def bf(h):
     return oracle.bf16_to_f32(h).astype(np.float64)
 
@@ -143,12 +156,15 @@ class GpuLayer:
         ws = self.lin.workspace(M).cpu().numpy()
         off, sz = svdq.svdq_workspace_layout(self.lin.handle, M)
         K, r = self.prep["K"], self.prep["rank"]
-        codes = ws[off[0]:off[0] + sz[0]].reshape(M, K // 2)
+        if self.prep["fmt"] == oracle.NVFP4:
+            codes = ws[off[0]:off[0] + sz[0]].reshape(M, K // 2)
+        else:
+            codes = int4_bytes_to_packed(ws[off[0]:off[0] + sz[0]].reshape(M, K))
         if self.prep["fmt"] == oracle.NVFP4:
             rows, blocks = np.meshgrid(np.arange(M), np.arange(K // 16), indexing="ij")
             scales = ws[off[1]:][sf_offset(rows, blocks, K // 64, 128)]
         else:
-            scales = ws[off[1]:off[1] + sz[1]].view(np.uint16).reshape(K // 64, M).T.copy()
+            scales = ws[off[1]:off[1] + sz[1]].view(np.uint16).reshape(K // 64, -1)[:, :M].T.copy()
         t = ws[off[2]:off[2] + sz[2]].view(np.uint16).reshape(M, r) if r else np.zeros((M, 0), np.uint16)
         return dict(codes=codes.copy(), scales=scales, t=t.copy())
 

@@ -183,7 +183,8 @@ def test_pack_layout(lib, fmt):
         start = o
         o = (o + nbytes + 1023) // 1024 * 1024
         return start
-    o_il, o_l1, o_l2, o_b, o_wc = take(K * 4), take(r * K * 2), take(N * r * 2), take(N * 4), take(N * K // 2)
+    wc_bytes = N * K if fmt == "int4" else N * K // 2
+    o_il, o_l1, o_l2, o_b, o_wc = take(K * 4), take(r * K * 2), take(N * r * 2), take(N * 4), take(wc_bytes)
     o_ws = o
     assert blob.size == (o + (N * K // 64 * 4 if fmt == "int4" else (N + 191) // 192 * (K // 64) * 1024) + 1023) // 1024 * 1024
     assert np.array_equal(blob[o_il:o_il + 4 * K].view(np.float32), c["inv_lambda"])
@@ -192,7 +193,14 @@ def test_pack_layout(lib, fmt):
     scale = 1.0 / (c["g_x"] * c["g_w"]) if fmt == "nvfp4" else 1.0
     assert np.array_equal(l2t, oracle.bf16_to_f32(c["L2"]).T.astype(np.float64) * scale)
     assert np.array_equal(blob[o_b:o_b + 4 * N].view(np.float32), oracle.bf16_to_f32(c["bias"]))
-    assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"])
+    if fmt == "int4":
+        # one E4M3 byte per code, holding the code's integer value exactly
+        wb = blob[o_wc:o_wc + N * K].reshape(N, K)
+        nib = np.stack([c["wcodes"] & 15, c["wcodes"] >> 4], axis=-1).reshape(N, K).astype(np.int64)
+        vals = np.where(nib >= 8, nib - 16, nib).astype(np.float32)
+        assert np.array_equal(wb, oracle.f32_to_e4m3(vals.reshape(-1)).reshape(N, K))
+    else:
+        assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"])
     if fmt == "int4":
         ws = blob[o_ws:o_ws + N * K // 64 * 4].view(np.float32).reshape(K // 64, N)
         assert np.array_equal(ws, c["wscales"].T.view(np.float16).astype(np.float32))
