@@ -13,23 +13,33 @@
 // <= 4096, all exact in binary32, so the accumulator holds acc_g exactly.
 // Because both scales change every 64 columns of K, each group's accumulator is
 // drained by the epilogue warps into an fp32 running sum held in registers,
-// y += (s_x s_w) acc_g, while the tensor core fills the next of four
-// accumulators.  The drain is the kernel's bound: two fp32 operations per
-// output and group against one 128 x 128 x 64 MMA.
+// y += (s_x s_w) acc_g: two fp32 operations per output and group, against one
+// 128 x 128 x 64 MMA.  That drain, not the tensor core, bounds the kernel.  Per
+// 128 x 128 group an SM spends about 256 cycles of FMA-pipe time (128 fp32
+// lanes per clock, packed f32x2 or not), about 256 cycles reading the 64 KiB
+// accumulator out of tensor memory in the 16x256b shape (about 255 B/clk; the
+// 32x32b shape reads about 3x faster but would need 64 weight scales per
+// thread and group from shared memory, which costs more), and about 128
+// cycles of shared-memory traffic for the scales.
 //
 // Persistent, warp-specialized CTA (one per SM), tile 128 x 128:
 //   warp 0      TMA producer: E4M3 codes [128 x 128 B] (128-byte swizzle) for
 //               A and B per 128-column K stage (two groups); the two groups'
 //               scales (f32 s_w [2 x 128], fp16 s_x [2 x 128]) into a ring of
 //               their own; the bf16 t / L2^T chunks of the low-rank branch.
-//   warp 1      owns tensor memory (4 x 128 columns) and issues the MMAs:
-//               kind::f16 for t . L2 (its own accumulator unit, which seeds the
-//               running sum), then 2 x kind::f8f6f4 (K = 32) per group.
-//   warps 2-9   epilogue (two per lane quarter, 64 columns each): tcgen05.ld
-//               each unit; y += (s_x s_w) acc in packed f32x2 arithmetic;
-//               bias, bf16 round-to-nearest-even, 16-byte stores.  With a
-//               debug output pointer it instead writes the group accumulators
-//               as int32 (integer-path parity).
+//   warp 1      owns tensor memory and issues the MMAs.  Accumulator units of
+//               256 columns, double-buffered: one unit per K stage holds its
+//               two groups side by side (2 x kind::f8f6f4, K = 32, per group),
+//               so the MMA and epilogue hand over once per two groups; the
+//               low-rank product t . L2 (kind::f16) is a unit of its own, once
+//               per tile, and seeds the running sum.
+//   warps 2-9   epilogue (two per lane quarter, 64 columns each; a thread holds
+//               4 rows x 16 columns): tcgen05.ld each group, release the unit
+//               once its last group is in registers (one arrival per warp),
+//               y += (s_x s_w) acc in packed f32x2 arithmetic; bias,
+//               bf16 round-to-nearest-even, stores.  With a debug output
+//               pointer it instead writes the group accumulators as int32
+//               (integer-path parity).
 // Every wait is bounded (sm100.cuh); no load uses cluster multicast.
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -59,9 +69,10 @@ constexpr int SC_BYTES = SC_SW + SC_SX;       // 1.5 KiB, a multiple of 128
 constexpr int EPI_WARPS = 8;  // two per tensor-memory lane quarter, 64 columns each
 constexpr int EPI_COLS = BN / 2;
 constexpr int EPI_WARP0 = 2;
-constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;  // 10 warps: up to 200 registers each
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;  // 10 warps: at most 168 registers each
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int NACC = 4;  // accumulator buffers
+constexpr int UNIT_COLS = GPS * BN;  // one accumulator unit: the GPS groups of a K stage
+constexpr int NBUF = 2;              // double-buffered units (all 512 columns)
 constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + LR_A + LR_B + (size_t)SC_SLOTS * SC_BYTES + 256;
@@ -99,21 +110,53 @@ __device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// y[0..31] += (sx * sw[0..31]) * acc[0..31]
-__device__ __forceinline__ void drain32(float* y, const uint32_t (&r)[32], const float* sw, float sx) {
+// Epilogue fragment of one thread (tcgen05.ld 16x256b, one load each for the
+// lanes 32q..32q+15 and 32q+16..32q+31 of its quarter q): rows 32q + t/4 + 8i
+// (i = 0..3) by columns c0 + 8j + e (j = 0..7, e = 0, 1), with
+// c0 = 64 p + 2 (t % 4) for the warp's column half p, held in y[16 i + 2 j + e].
+// (The 32x32b shape reads tensor memory about 3x faster, but gives each thread
+// one row and 64 columns, so every thread would need 64 weight scales per group
+// from shared memory; here a thread needs 16.)
+
+// y += (s_x[row] s_w[col]) acc over the fragment; sw points at s_w[c0], sx[i]
+// is s_x of row i.  Two packed operations per pair of outputs.
+__device__ __forceinline__ void drain_frag(float (&y)[64], const uint32_t (&lo)[32], const uint32_t (&hi)[32],
+                                           const float* sw, const float (&sx)[4]) {
 #pragma unroll
-  for (int j = 0; j < 32; j += 4) {
-    const float4 w4 = *(const float4*)(sw + j);  // the same address in every lane: a broadcast
-    float c0 = w4.x, c1 = w4.y, c2 = w4.z, c3 = w4.w;
-    mul2(c0, c1, sx, sx);  // exact: a product of two fp16 values
-    mul2(c2, c3, sx, sx);
-    fma2(y[j], y[j + 1], c0, c1, __uint_as_float(r[j]), __uint_as_float(r[j + 1]));
-    fma2(y[j + 2], y[j + 3], c2, c3, __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+  for (int j = 0; j < 8; ++j) {
+    const float2 w = *(const float2*)(sw + 8 * j);  // 4 distinct addresses per warp
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t(&r)[32] = i < 2 ? lo : hi;
+      const int k = 4 * j + 2 * (i & 1);
+      float c0 = w.x, c1 = w.y;
+      mul2(c0, c1, sx[i], sx[i]);  // exact: a product of two fp16 values
+      fma2(y[16 * i + 2 * j], y[16 * i + 2 * j + 1], c0, c1, __uint_as_float(r[k]), __uint_as_float(r[k + 1]));
+    }
+  }
+}
+
+// integer-path export of one group's fragment
+__device__ __forceinline__ void export_frag(const I4Params& p, size_t g, int row0, int col0, const uint32_t (&lo)[32],
+                                            const uint32_t (&hi)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = row0 + 8 * i;
+    if (m >= p.M) continue;
+    const uint32_t(&r)[32] = i < 2 ? lo : hi;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int n = col0 + 8 * j;
+      const int k = 4 * j + 2 * (i & 1);
+      if (n < p.N)
+        *(int2*)(p.acc_dbg + (g * p.M + m) * p.N + n) =
+            make_int2(__float2int_rz(__uint_as_float(r[k])), __float2int_rz(__uint_as_float(r[k + 1])));
+    }
   }
 }
 
 template <bool DBG>
-__global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant__ I4Maps maps, const I4Params p) {
+__global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant__ I4Maps maps, const __grid_constant__ I4Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* stages = smem;                             // [STAGES][STAGE_BYTES]  (1024-aligned)
@@ -125,9 +168,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   uint64_t* sc_empty = sc_full + SC_SLOTS;
   uint64_t* lr_full = sc_empty + SC_SLOTS;
   uint64_t* lr_empty = lr_full + 1;
-  uint64_t* acc_full = lr_empty + 1;      // [NACC]
-  uint64_t* acc_empty = acc_full + NACC;  // [NACC]
-  uint64_t* mma_done = acc_empty + NACC;
+  uint64_t* acc_full = lr_empty + 1;      // [NBUF]
+  uint64_t* acc_empty = acc_full + NBUF;  // [NBUF]
+  uint64_t* mma_done = acc_empty + NBUF;
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -145,9 +188,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
     }
     mbar_init(lr_full, 1);
     mbar_init(lr_empty, 1);
-    for (int b = 0; b < NACC; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], EPI_WARPS * 32);
+      mbar_init(&acc_empty[b], EPI_WARPS);  // one arrival per epilogue warp
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -220,8 +263,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         if (p.n_lr > 0) {
-          const int b = unit % NACC;
-          if (!mbar_wait(&acc_empty[b], ((unit / NACC) & 1) ^ 1, wc)) break;
+          const int b = unit % NBUF;
+          if (!mbar_wait(&acc_empty[b], ((unit / NBUF) & 1) ^ 1, wc)) break;
           tc_fence_after();
           uint32_t accum = 0;
           for (int u = 0; u < p.n_lr; ++u, ++lit) {
@@ -235,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
             const uint32_t sbo = 16u * (uint32_t)w;
             const uint32_t a_addr = smem_u32(lrbuf), b_addr = a_addr + LR_A;
             for (int kk = 0; kk < w / 16; ++kk) {
-              mma_bf16(tmem + b * BN, make_sdesc(a_addr + 32 * kk, 16, sbo, layout),
+              mma_bf16(tmem + b * UNIT_COLS, make_sdesc(a_addr + 32 * kk, 16, sbo, layout),
                        make_sdesc(b_addr + 32 * kk, 16, sbo, layout), IDESC_BF16, accum);
               accum = 1;
             }
@@ -253,21 +296,23 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
           }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + s * STAGE_BYTES), b_addr = a_addr + STAGE_A;
-          for (int g = 0; g < GPS; ++g, ++unit) {
-            const int b = unit % NACC;
-            if (!mbar_wait(&acc_empty[b], ((unit / NACC) & 1) ^ 1, wc)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+          const int b = unit % NBUF;
+          if (!mbar_wait(&acc_empty[b], ((unit / NBUF) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int g = 0; g < GPS; ++g) {  // each group into its own 128 columns of the unit
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {  // K = 32 codes (bytes) per instruction
               const uint32_t off = 64 * g + 32 * kk;
-              mma_f8f6f4(tmem + b * BN, make_sdesc(a_addr + off, 16, 1024, LAYOUT_SW128),
+              mma_f8f6f4(tmem + b * UNIT_COLS + g * BN, make_sdesc(a_addr + off, 16, 1024, LAYOUT_SW128),
                          make_sdesc(b_addr + off, 16, 1024, LAYOUT_SW128), IDESC_E4M3, (uint32_t)kk);
             }
-            umma_commit(&acc_full[b]);
           }
+          umma_commit(&acc_full[b]);
+          ++unit;
           umma_commit(&empty[s]);
         }
       }
@@ -277,95 +322,91 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int half = (warp - EPI_WARP0) >> 2;
-    const int row = 32 * q + lane;
+    const int part = (warp - EPI_WARP0) >> 2;
+    const int rq = 32 * q + (lane >> 2);             // fragment rows rq + 8i
+    const int cq = part * EPI_COLS + 2 * (lane & 3);  // fragment columns cq + 8j + e
+    const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(part * EPI_COLS);
+    const uint32_t tq_hi = tq + (16u << 16);
     int it = 0, unit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-      const int m = mt * BM + row;
-      const int n0 = nt * BN + half * EPI_COLS;
-      const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * EPI_COLS);
-      float y[EPI_COLS];
+      const int m0 = mt * BM + rq;
+      const int n0 = nt * BN + cq;
+      float y[64];
 #pragma unroll
-      for (int j = 0; j < EPI_COLS; ++j) y[j] = 0.f;
+      for (int j = 0; j < 64; ++j) y[j] = 0.f;
       if (p.n_lr > 0) {
-        const int b = unit % NACC;
-        if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) break;
+        const int b = unit % NBUF;
+        if (!mbar_wait(&acc_full[b], (unit / NBUF) & 1, wc)) break;
         tc_fence_after();
-        uint32_t r0[32], r1[32];
-        tmem_ld_32x32b_x32(tl + b * BN, r0);
-        tmem_ld_32x32b_x32(tl + b * BN + 32, r1);
-        tmem_ld_wait();
+        uint32_t lo[32], hi[32];
+        tmem_ld_16x256b_x8(tq + b * UNIT_COLS, lo);
+        tmem_ld_16x256b_x8(tq_hi + b * UNIT_COLS, hi);
+        tmem_ld_wait_regs(lo);
+        reg_order(hi);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          y[j] = __uint_as_float(r0[j]);
-          y[32 + j] = __uint_as_float(r1[j]);
-        }
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              y[16 * i + 2 * j + e] = __uint_as_float((i < 2 ? lo : hi)[4 * j + 2 * (i & 1) + e]);
         tc_fence_before();
-        mbar_arrive(&acc_empty[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
         ++unit;
       }
-      for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it) {
+      // One unit per K stage: the accumulators of its GPS groups, drained one
+      // group at a time; the unit is released once its last group is in
+      // registers.
+      for (int ks = 0; ks < p.k_stages && ok; ++ks, ++it, ++unit) {
         const int ss = it % SC_SLOTS;
-        if (!mbar_wait(&sc_full[ss], (it / SC_SLOTS) & 1, wc)) {
+        const int b = unit % NBUF;
+        if (!mbar_wait(&sc_full[ss], (it / SC_SLOTS) & 1, wc) || !mbar_wait(&acc_full[b], (unit / NBUF) & 1, wc)) {
           ok = false;
           break;
         }
+        tc_fence_after();
         const uint8_t* sc = scring + ss * SC_BYTES;
-        for (int g = 0; g < GPS; ++g, ++unit) {
-          const int b = unit % NACC;
-          if (!mbar_wait(&acc_full[b], (unit / NACC) & 1, wc)) {
-            ok = false;
-            break;
+#pragma unroll 1
+        for (int g = 0; g < GPS; ++g) {
+          uint32_t lo[32], hi[32];
+          tmem_ld_16x256b_x8(tq + b * UNIT_COLS + g * BN, lo);
+          tmem_ld_16x256b_x8(tq_hi + b * UNIT_COLS + g * BN, hi);
+          tmem_ld_wait_regs(lo);
+          reg_order(hi);
+          if (g == GPS - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);  // every group of the unit is in registers
           }
-          tc_fence_after();
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(tl + b * BN, r0);
-          tmem_ld_32x32b_x32(tl + b * BN + 32, r1);
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&acc_empty[b]);  // the accumulator is in registers now
           if (DBG) {
-            if (m < p.M) {
-              const int gg = ks * GPS + g;
-#pragma unroll
-              for (int j = 0; j < EPI_COLS; j += 4) {
-                const int n = n0 + j;
-                const uint32_t* rr = j < 32 ? r0 + j : r1 + (j - 32);
-                if (n < p.N)
-                  *(int4*)(p.acc_dbg + ((size_t)gg * p.M + m) * p.N + n) =
-                      make_int4(__float2int_rz(__uint_as_float(rr[0])), __float2int_rz(__uint_as_float(rr[1])),
-                                __float2int_rz(__uint_as_float(rr[2])), __float2int_rz(__uint_as_float(rr[3])));
-              }
-            }
+            export_frag(p, (size_t)(ks * GPS + g), m0, n0, lo, hi);
           } else {
-            const float sx = __half2float(((const __half*)(sc + SC_SW))[g * BM + row]);
-            const float* sw = (const float*)sc + g * BN + half * EPI_COLS;
-            drain32(y, r0, sw, sx);
-            drain32(y + 32, r1, sw + 32, sx);
+            const __half* sxs = (const __half*)(sc + SC_SW) + g * BM + rq;
+            const float sx[4] = {__half2float(sxs[0]), __half2float(sxs[8]), __half2float(sxs[16]),
+                                 __half2float(sxs[24])};
+            drain_frag(y, lo, hi, (const float*)sc + g * BN + cq, sx);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sc_empty[ss]);
       }
       if (!ok) break;
-      if (!DBG && m < p.M) {
+      if (!DBG) {
 #pragma unroll
-        for (int j8 = 0; j8 < EPI_COLS / 8; ++j8) {
-          const int n = n0 + 8 * j8;
-          if (n < p.N) {
-            const float4 b0 = __ldg((const float4*)(p.bias + n));
-            const float4 b1 = __ldg((const float4*)(p.bias + n + 4));
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            uint32_t o[4];
+        for (int j = 0; j < 8; ++j) {
+          const int n = n0 + 8 * j;
+          if (n >= p.N) continue;
+          const float2 bb = __ldg((const float2*)(p.bias + n));
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h =
-                  __floats2bfloat162_rn(y[8 * j8 + 2 * e] + bb[2 * e], y[8 * j8 + 2 * e + 1] + bb[2 * e + 1]);
-              o[e] = *(uint32_t*)&h;
+          for (int i = 0; i < 4; ++i) {
+            const int m = m0 + 8 * i;
+            if (m < p.M) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(y[16 * i + 2 * j] + bb.x, y[16 * i + 2 * j + 1] + bb.y);
+              *(__nv_bfloat162*)(p.Y + (size_t)m * p.N + n) = h;
             }
-            *(uint4*)(p.Y + (size_t)m * p.N + n) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
       }
