@@ -10,8 +10,9 @@
 // Work split: a CTA owns 128 token rows and one slice of K (the K range is cut
 // into enough slices that about one CTA per SM is in flight).  Per 128-column
 // chunk:
-//   warp 8      TMA: the X tile [128 x 128] into a ring that the quantizing
-//               warps release as soon as they have read it;
+//   warp 8      TMA: the X tile [128 x 128], and a bulk copy of the chunk's
+//               128 entries of 1/lambda, into a ring that the quantizing warps
+//               release as soon as they have read it;
 //   warp 10     TMA: the matching L1^T slice [rank x 128] (two 64-column boxes,
 //               128-byte swizzle) into a small ring released by the MMAs;
 //   warps 0-7   quantize 16 rows each (a lane holds 16 consecutive elements:
@@ -43,6 +44,10 @@ constexpr int kMmaWarp = 9;
 constexpr int kL1Warp = 10;
 constexpr int kThreads = 11 * 32;
 constexpr int kXTileBytes = kRows * kChunk * 2;  // 32 KiB
+constexpr int kIlBytes = kChunk * 4;              // the chunk's 1/lambda slice
+constexpr int kXStageBytes = kXTileBytes + kIlBytes;
+// the X ring, padded so the 128-byte-swizzled tiles after it stay 1024-aligned
+__host__ __device__ constexpr int xring_bytes(int xs) { return (xs * kXStageBytes + 1023) & ~1023; }
 constexpr int kAHalfBytes = kRows * 128;         // 64 bf16 columns, 128B-swizzled
 constexpr int kATileBytes = 2 * kAHalfBytes;     // 32 KiB
 constexpr int kSmemBudget = 220 * 1024;
@@ -126,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int XS = p.xstages, LS = p.lstages;
   constexpr int kL1Bytes = RANK * kChunk * 2;  // two boxes of RANK rows x 128 B
-  uint8_t* xring = smem;                          // [XS][kXTileBytes]
-  uint8_t* atile = xring + XS * kXTileBytes;      // [2][kATileBytes] when RANK > 0
+  uint8_t* xring = smem;                          // [XS][X tile | 1/lambda slice]
+  uint8_t* atile = xring + xring_bytes(XS);       // [2][kATileBytes] when RANK > 0 (1024-aligned)
   uint8_t* lring = atile + (RANK > 0 ? 2 * kATileBytes : 0);  // [LS][kL1Bytes]
   float* rtab = (float*)(lring + LS * kL1Bytes);  // [128] 1/e4m3
   uint64_t* full_x = (uint64_t*)(rtab + 128);
@@ -187,8 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < nchunks; ++i) {
         const int s = i % XS;
         if (!mbar_wait(&empty_x[s], ((i / XS) & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&full_x[s], kXTileBytes);
-        tma_load_2d(&map_x, &full_x[s], xring + s * kXTileBytes, (c_begin + i) * kChunk, m0);
+        uint8_t* dst = xring + s * kXStageBytes;
+        mbar_arrive_expect_tx(&full_x[s], kXStageBytes);
+        tma_load_2d(&map_x, &full_x[s], dst, (c_begin + i) * kChunk, m0);
+        bulk_load(dst + kXTileBytes, p.inv_lambda + (size_t)(c_begin + i) * kChunk, kIlBytes, &full_x[s]);
         issued = i + 1;
       }
       if (*abort_flag) {  // drain copies that are still in flight before leaving
@@ -255,13 +262,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&full_x[s], (i / XS) & 1, wc);
       if constexpr (RANK > 0) ok = ok && mbar_wait(&xfree[buf], ((i >> 1) & 1) ^ 1, wc);
       if (ok) {
-        const uint8_t* st = xring + s * kXTileBytes;
+        const uint8_t* st = xring + s * kXStageBytes;
         const int k0 = (c_begin + i) * kChunk;
         const int kk0 = k0 + 16 * j;
         float il[16];
+        const float4* ils = (const float4*)(st + kXTileBytes) + 4 * j;  // staged with the X tile
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float4 t4 = __ldg((const float4*)(p.inv_lambda + kk0 + 4 * q));
+          const float4 t4 = ils[q];
           il[4 * q] = t4.x;
           il[4 * q + 1] = t4.y;
           il[4 * q + 2] = t4.z;
@@ -440,11 +448,10 @@ int launch_rank(const CUtensorMap& mx, const CUtensorMap& ml1, const QParams& p,
   constexpr int kFixed = (RANK > 0 ? 2 * kATileBytes : 0) + 512 + 512;
   QParams q = p;
   q.lstages = RANK > 0 ? (RANK <= 64 ? 3 : 2) : 0;
-  int XS = (kSmemBudget - kFixed - q.lstages * kL1Bytes) / kXTileBytes;
-  if (XS > 5) XS = 5;
-  if (XS < 2) XS = 2;
+  int XS = 5;
+  while (XS > 2 && xring_bytes(XS) + kFixed + q.lstages * kL1Bytes > kSmemBudget) --XS;
   q.xstages = XS;
-  const size_t smem = 1024 + (size_t)XS * kXTileBytes + (size_t)q.lstages * kL1Bytes + kFixed;
+  const size_t smem = 1024 + (size_t)xring_bytes(XS) + (size_t)q.lstages * kL1Bytes + kFixed;
   auto kern = k_quantize<FMT, RANK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;

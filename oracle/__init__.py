@@ -203,6 +203,16 @@ def svd_lowrank_factors(What: np.ndarray, rank: int):
     return Vr * sq[None, :], (Ur * sq[None, :]).T.copy(), S
 
 
+def smoothed_weight(W_bf16: np.ndarray, amax_x: np.ndarray, alpha: float):
+    """Steps 1-2 of prepare: lambda from the channel maxima and W^ = W * lambda
+    (binary64 product of the binary32 lambda).  Returns (W^, (lambda_d, lambda_f,
+    1/lambda_f))."""
+    Wf = bf16_to_f32(np.ascontiguousarray(W_bf16, np.uint16))
+    amax_w = np.abs(Wf).max(axis=0).astype(np.float32)
+    lams = smooth_factors(amax_x, amax_w, alpha)
+    return Wf.astype(np.float64) * lams[1].astype(np.float64)[None, :], lams
+
+
 def prepare(W_bf16: np.ndarray, bias_bf16, amax_x: np.ndarray, alpha: float, rank: int, fmt, svd=None):
     """Offline preparation of one layer ("Суть метода"):
       1. lambda from the activation and weight channel maxima (smoothing),
@@ -213,12 +223,8 @@ def prepare(W_bf16: np.ndarray, bias_bf16, amax_x: np.ndarray, alpha: float, ran
     `svd` may carry a precomputed (L1, L2, S) of the same W^ (same lambda), so
     that several ranks reuse one decomposition; it is truncated to `rank`."""
     fmt = _FMT[fmt]
-    W = np.ascontiguousarray(W_bf16, np.uint16)
-    N, K = W.shape
-    Wf = bf16_to_f32(W)
-    amax_w = np.abs(Wf).max(axis=0).astype(np.float32)
-    lam_d, lam_f, inv_lam = smooth_factors(amax_x, amax_w, alpha)
-    What = Wf.astype(np.float64) * lam_f.astype(np.float64)[None, :]
+    N, K = W_bf16.shape
+    What, (lam_d, lam_f, inv_lam) = smoothed_weight(W_bf16, amax_x, alpha)
     r = int(rank)
     if r > 0:
         if svd is None:
