@@ -13,9 +13,11 @@
 //
 // Persistent, warp-specialized CTA (one per SM), tile 128 x 192:
 //   warp 0      TMA producer: per stage a 128x256 activation-code tile and a
-//               192x256 weight-code tile (128-byte swizzle), plus the matching
-//               E4M3 scale-factor atoms with bulk copies; the t / L2^T chunks of
-//               the low-rank branch ride the same ring first.
+//               192x256 weight-code tile (128-byte swizzle); the t / L2^T chunks
+//               of the low-rank branch ride the same ring first.
+//   warp 10     scale-factor producer: the E4M3 scale-factor atoms of two K
+//               stages per bulk copy (activation and weight side) into a ring of
+//               their own, so they arrive ahead of the codes they scale.
 //   warp 1      owns tensor memory (512 columns: two 192-column fp32
 //               accumulators for ping-pong with the epilogue, and two 48-column
 //               scale-factor buffers); one lane issues tcgen05.mma kind::f16
@@ -23,7 +25,8 @@
 //   warps 6-9   move each stage's E4M3 scale-factor atoms from shared memory
 //               into their tensor-memory lane quarter with tcgen05.st, in the
 //               replicated layout the block-scaled MMA reads, so the transfer
-//               runs beside the tensor pipe instead of inside it.
+//               runs beside the tensor pipe instead of inside it; with their own
+//               ring they finish before the stage's codes land.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, scale, bias,
 //               bf16 round-to-nearest-even into a 128B-swizzled shared-memory
 //               staging tile, written to Y by TMA bulk-tensor stores.
@@ -45,16 +48,20 @@ constexpr int A_BYTES = BM * 128;  // 256 fp4 per row
 constexpr int B_BYTES = BN * 128;
 constexpr int SFA_BYTES = 4 * kSfAtomBytes;      // 4 k-atoms x 128 rows
 constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;  // 4 k-atoms x 256 rows (192 used)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int THREADS = 320;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SF_SLOTS = 2;                                 // scale-factor ring
+constexpr int SF_SLOT_BYTES = 2 * (SFA_BYTES + SFB_BYTES);  // two K stages: [SFA x2 | SFB x2]
+constexpr int SF_WARP = 10;
+constexpr int THREADS = 352;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 2 * BN;  // 384: two buffers of [SFA 16 | SFB 32] columns
 constexpr uint32_t SF_BUF_COLS = 48;
 constexpr int EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 rows x 64 bf16, 128B-swizzled
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 4 * 2 * EPI_STAGE_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + 4 * 2 * EPI_STAGE_BYTES;
 constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(STAGE_BYTES % 1024 == 0 && SF_SLOT_BYTES % 1024 == 0, "stage alignment");
+static_assert(SMEM_BYTES + 1024 + 256 <= 227 * 1024, "shared memory budget");
 static_assert(SF_COL + 2 * SF_BUF_COLS <= TMEM_COLS, "tensor memory budget");
 
 struct GemmMaps {
@@ -79,7 +86,8 @@ __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 
 __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant__ GemmMaps maps, const __grid_constant__ GParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* epi_stage = smem + STAGES * STAGE_BYTES;  // [4 warps][2][EPI_STAGE_BYTES]
+  uint8_t* sfring = smem + STAGES * STAGE_BYTES;                // [SF_SLOTS][SF_SLOT_BYTES]
+  uint8_t* epi_stage = sfring + SF_SLOTS * SF_SLOT_BYTES;       // [4 warps][2][EPI_STAGE_BYTES]
   uint64_t* full = (uint64_t*)(smem + SMEM_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
@@ -87,7 +95,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   uint64_t* mma_done = acc_empty + 2;   // [1]
   uint64_t* sf_ready = mma_done + 1;    // [2]
   uint64_t* sf_free = sf_ready + 2;     // [2]
-  uint32_t* tmem_slot = (uint32_t*)(sf_free + 2);
+  uint64_t* sfs_full = sf_free + 2;     // [SF_SLOTS]
+  uint64_t* sfs_empty = sfs_full + SF_SLOTS;
+  uint32_t* tmem_slot = (uint32_t*)(sfs_empty + SF_SLOTS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -106,6 +116,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sf_ready[b], 4);
       mbar_init(&sf_free[b], 1);
+    }
+    for (int b = 0; b < SF_SLOTS; ++b) {
+      mbar_init(&sfs_full[b], 1);
+      mbar_init(&sfs_empty[b], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -146,10 +160,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
             mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
             tma_load_2d(&maps.a, &full[s], st, ks * 128, mt * BM);
             tma_load_2d(&maps.b, &full[s], st + A_BYTES, ks * 128, nt * BN);
-            bulk_load(st + A_BYTES + B_BYTES, p.sfa + ((size_t)mt * p.katoms + 4 * ks) * kSfAtomBytes, SFA_BYTES,
-                      &full[s]);
-            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES,
-                      p.sfb + ((size_t)nt * p.katoms + 4 * ks) * 2 * kSfAtomBytes, SFB_BYTES, &full[s]);
           }
         }
       }
@@ -213,6 +223,35 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       umma_commit(mma_done);  // every MMA issued above has completed when this fires
       mbar_wait_drain(mma_done, 0, p.limit);
     }
+  } else if (warp == SF_WARP) {
+    // ------------------------------------------------------------ scale-factor producer
+    // Pair j of a tile carries the atoms of K stages 2j and 2j+1 (one stage for
+    // an odd tail): [SFA stage 2j | SFA 2j+1 | SFB stage 2j | SFB 2j+1].
+    if (lane == 0) {
+      int pit = 0;
+      bool ok = true;
+      const int pairs = (p.k_stages + 1) / 2;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        for (int j = 0; j < pairs; ++j, ++pit) {
+          const int slot = pit % SF_SLOTS;
+          if (!mbar_wait(&sfs_empty[slot], ((pit / SF_SLOTS) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
+          uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
+          mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
+          bulk_load(dst, p.sfa + ((size_t)mt * p.katoms + 8 * j) * kSfAtomBytes, ns * SFA_BYTES, &sfs_full[slot]);
+          bulk_load(dst + 2 * SFA_BYTES, p.sfb + ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes, ns * SFB_BYTES,
+                    &sfs_full[slot]);
+        }
+      }
+      if (!ok) {  // drain the copies still in flight
+        for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
+          mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, p.limit);
+      }
+    }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ scale-factor movers
     // Warp q owns tensor-memory lanes 32q..32q+31.  Lane l writes, for every
@@ -220,25 +259,26 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     // scales of rows l, l+32, l+64, l+96 for 4 consecutive K blocks) into 4
     // consecutive columns -- the same bytes in every lane quarter.
     const int q = warp & 3;
-    int it = 0, kst = 0;
+    int kst = 0, pit = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-      for (int u = 0; u < units; ++u, ++it) {
-        if (u < p.n_lr) continue;
-        const int s = it % STAGES, sb = kst & 1;
-        ok = mbar_wait(&full[s], (it / STAGES) & 1, wc) && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+      for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
+        const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
+        const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
+        if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
+        ok = ok && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
         if (!ok) break;
-        const uint8_t* sfa_s = smem + s * STAGE_BYTES + A_BYTES + B_BYTES;
-        const uint8_t* sfb_s = sfa_s + SFA_BYTES;
+        const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
+        const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
         uint32_t ra[16], rb[32];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
           ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + h) * kSfAtomBytes + lane * 16);
-            rb[8 * j + 4 * h] = b4.x; rb[8 * j + 4 * h + 1] = b4.y; rb[8 * j + 4 * h + 2] = b4.z; rb[8 * j + 4 * h + 3] = b4.w;
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + hh) * kSfAtomBytes + lane * 16);
+            rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
           }
         }
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
@@ -247,8 +287,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_ready[sb]);
-        ++kst;
+        if (lane == 0) {
+          mbar_arrive(&sf_ready[sb]);
+          if (last_of_pair) mbar_arrive(&sfs_empty[slot]);  // the slot's atoms are in tensor memory
+        }
+        if (last_of_pair) ++pit;
       }
     }
   } else {
