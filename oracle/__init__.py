@@ -310,3 +310,78 @@ def int4_group_acc(xcodes: np.ndarray, wcodes: np.ndarray) -> np.ndarray:
     acc = np.empty((K // 64, M, N), np.int32)
     lib().orc_int4_group_acc(M, N, K, _p(xcodes), _p(wcodes), _p(acc))
     return acc
+
+
+# ----------------------------------------------------------------------------- awq_w4a16
+# The second runtime layer of the pages ("Hugging Face встроила Nunchaku в
+# Diffusers ...", paragraph on Nunchaku Lite): 4-bit weights with 16-bit
+# activations for precision-sensitive normalization / modulation layers (adaLN in
+# FLUX).  The pages name AWQ and say nothing more; the readings here are:
+#   - activation-aware per-input-channel scale s_j = mean|x_j|^alpha (1 where the
+#     mean is 0), alpha from the grid 0, 0.05, ..., 1 minimising the layer's
+#     output error on its own calibration input (the AWQ form);
+#   - weights W diag(s) quantized with the same INT4 group-64 quantizer as the
+#     svdq_w4a4 residual (symmetric, fp16 scale);
+#   - forward y = (f32(x) * inv_s) . dequant(Q4(W diag(s)))^T + b, the activation
+#     product in binary32 (as in the smoothing step), the rest exact in binary64,
+#     rounded once to bf16.
+AWQ_ALPHAS = tuple(i / 20.0 for i in range(21))
+
+
+def awq_mean_abs(X_bf16: np.ndarray) -> np.ndarray:
+    """Calibration statistic of the activation-aware scale: mean |x| per input channel (binary64)."""
+    return np.abs(bf16_to_f32(X_bf16).astype(np.float64)).mean(axis=0)
+
+
+def awq_channel_scales(mean_abs: np.ndarray, alpha: float):
+    """s_j = mean|x_j|^alpha in binary64 (1 where the mean is 0); returns (s, float32(s), float32(1/float32(s)))."""
+    m = np.asarray(mean_abs, np.float64)
+    s = np.ones_like(m)
+    nz = m > 0
+    s[nz] = m[nz] ** float(alpha)
+    s_f = s.astype(np.float32)
+    inv = (1.0 / s_f.astype(np.float64)).astype(np.float32)
+    return s, s_f, inv
+
+
+def awq_quant_weights(W_bf16: np.ndarray, s_f32: np.ndarray):
+    """Q4(W diag(s)): the scaled weight rounded to binary32, then INT4 groups of 64 (codes, fp16 scales)."""
+    Wf = bf16_to_f32(np.ascontiguousarray(W_bf16, np.uint16)).astype(np.float64)
+    Ws = (Wf * np.asarray(s_f32, np.float32).astype(np.float64)[None, :]).astype(np.float32)
+    return quant_int4(Ws)
+
+
+def awq_forward(X_bf16: np.ndarray, prep: dict, want_f64: bool = False):
+    """y = (f32(x) * inv_s) . (q * S)^T + b in binary64 from the binary32 x^, rounded to bf16."""
+    xhat = smooth_act(X_bf16, prep["inv_s"]).astype(np.float64)
+    deq = dequant(prep["wcodes"], prep["wscales"], INT4)
+    yd = xhat @ deq.T + bf16_to_f32(prep["bias"]).astype(np.float64)[None, :]
+    y = f64_to_bf16(np.ascontiguousarray(yd))
+    return (y, yd) if want_f64 else y
+
+
+def awq_output_error(X_bf16: np.ndarray, W_bf16: np.ndarray, mean_abs: np.ndarray, alpha: float) -> float:
+    """Squared output error sum_mn (x^ . deq^T - x . W^T)^2 (no bias) of one grid point, binary64."""
+    _, s_f, inv = awq_channel_scales(mean_abs, alpha)
+    codes, scales = awq_quant_weights(W_bf16, s_f)
+    xhat = smooth_act(X_bf16, inv).astype(np.float64)
+    ref = bf16_to_f32(X_bf16).astype(np.float64) @ bf16_to_f32(W_bf16).astype(np.float64).T
+    return float(((xhat @ dequant(codes, scales, INT4).T - ref) ** 2).sum())
+
+
+def awq_prepare(W_bf16: np.ndarray, bias_bf16, X_calib_bf16: np.ndarray, alphas=AWQ_ALPHAS):
+    """Activation-aware preparation of one awq_w4a16 layer: the first alpha of the
+    grid with the smallest output error on the calibration input wins."""
+    W = np.ascontiguousarray(W_bf16, np.uint16)
+    N, K = W.shape
+    mabs = awq_mean_abs(X_calib_bf16)
+    best = None
+    for a in alphas:
+        err = awq_output_error(X_calib_bf16, W, mabs, a)
+        if best is None or err < best[1]:
+            best = (a, err)
+    a = best[0]
+    _, s_f, inv = awq_channel_scales(mabs, a)
+    codes, scales = awq_quant_weights(W, s_f)
+    return dict(N=N, K=K, alpha=float(a), err=best[1], s=s_f, inv_s=inv, wcodes=codes, wscales=scales,
+                bias=(np.zeros(N, np.uint16) if bias_bf16 is None else np.ascontiguousarray(bias_bf16, np.uint16)))
