@@ -6,7 +6,8 @@ Argument marshalling only: every step of the layer runs in the CUDA library
 CPU fallback: if libsvdq.so is missing or cannot be loaded, every call raises.
 
 Entry points keep the C names (svdq_prepare, svdq_pack, svdq_layer_create,
-svdq_forward, ...).  `SvdqLinear` bundles them for nn.Linear-style use.
+svdq_forward, ..., and svdq_awq_* for the awq_w4a16 layer).  `SvdqLinear` and
+`AwqLinear` bundle them for nn.Linear-style use.
 """
 from __future__ import annotations
 
@@ -50,6 +51,12 @@ class svdq_canonical(ctypes.Structure):
                 ("wscales", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
 
 
+class svdq_awq_canonical(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64), ("alpha", ctypes.c_float), ("reserved", ctypes.c_float),
+                ("s", ctypes.c_void_p), ("inv_s", ctypes.c_void_p), ("wcodes", ctypes.c_void_p),
+                ("wscales", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+
+
 _lib = None
 _EXPORTS = {
     # name: (restype, argtypes)
@@ -85,6 +92,16 @@ _EXPORTS = {
     "svdq_set_wait_limit": (ctypes.c_int, [ctypes.c_uint64]),
     "svdq_forward_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_void_p]),
+    "svdq_awq_canonical_sizes": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)]),
+    "svdq_awq_prepare": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.POINTER(svdq_awq_canonical)]),
+    "svdq_awq_packed_size": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)]),
+    "svdq_awq_pack": (ctypes.c_int, [ctypes.POINTER(svdq_awq_canonical), ctypes.c_void_p, ctypes.c_size_t]),
+    "svdq_awq_layer_create": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.POINTER(ctypes.c_void_p)]),
+    "svdq_awq_layer_destroy": (None, [ctypes.c_void_p]),
+    "svdq_awq_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                        ctypes.c_void_p]),
 }
 
 
@@ -310,4 +327,104 @@ class SvdqLinear:
         h = getattr(self, "handle", None)
         if h is not None and _lib is not None:
             _lib.svdq_layer_destroy(h)
+            self.handle = None
+
+
+# ----------------------------------------------------------------------------- awq_w4a16
+def svdq_awq_canonical_sizes(N: int, K: int) -> list[int]:
+    sizes = (ctypes.c_size_t * 5)()
+    _check(lib().svdq_awq_canonical_sizes(N, K, sizes), "svdq_awq_canonical_sizes")
+    return list(sizes)
+
+
+def _awq_arrays(N, K):
+    return dict(N=N, K=K, alpha=0.0, s=np.zeros(K, np.float32), inv_s=np.zeros(K, np.float32),
+                wcodes=np.zeros((N, K // 2), np.uint8), wscales=np.zeros((N, K // 64), np.uint16),
+                bias=np.zeros(N, np.uint16))
+
+
+def _awq_struct(c: dict) -> svdq_awq_canonical:
+    st = svdq_awq_canonical()
+    st.N, st.K, st.alpha = int(c["N"]), int(c["K"]), float(c.get("alpha", 0.0))
+    for f in ("s", "inv_s", "wcodes", "wscales", "bias"):
+        arr = c.get(f)
+        setattr(st, f, None if arr is None else arr.ctypes.data)
+    return st
+
+
+def svdq_awq_prepare(W: np.ndarray, bias, X_calib: np.ndarray) -> dict:
+    """Host-side activation-aware preparation of an awq_w4a16 layer.
+    W: bf16 bits [N,K]; bias: bf16 bits [N] or None; X_calib: bf16 bits [M_calib, K]."""
+    W = np.ascontiguousarray(W, np.uint16)
+    X = np.ascontiguousarray(X_calib, np.uint16)
+    N, K = W.shape
+    c = _awq_arrays(N, K)
+    st = _awq_struct(c)
+    b = None if bias is None else np.ascontiguousarray(bias, np.uint16)
+    _check(lib().svdq_awq_prepare(W.ctypes.data, None if b is None else b.ctypes.data, X.ctypes.data, X.shape[0],
+                                  ctypes.byref(st)), "svdq_awq_prepare")
+    c["alpha"] = float(st.alpha)
+    return c
+
+
+def svdq_awq_packed_size(N: int, K: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().svdq_awq_packed_size(N, K, ctypes.byref(n)), "svdq_awq_packed_size")
+    return n.value
+
+
+def svdq_awq_pack(c: dict) -> np.ndarray:
+    c = dict(c)
+    for f, dt in (("s", np.float32), ("inv_s", np.float32), ("wcodes", np.uint8), ("wscales", np.uint16),
+                  ("bias", np.uint16)):
+        if c.get(f) is not None:
+            c[f] = np.ascontiguousarray(c[f], dt)
+    size = svdq_awq_packed_size(c["N"], c["K"])
+    blob = np.zeros(size, np.uint8)
+    _check(lib().svdq_awq_pack(ctypes.byref(_awq_struct(c)), blob.ctypes.data, size), "svdq_awq_pack")
+    return blob
+
+
+def svdq_awq_layer_create(dev_blob, blob_bytes: int, N: int, K: int):
+    h = ctypes.c_void_p()
+    _check(lib().svdq_awq_layer_create(_ptr(dev_blob), blob_bytes, N, K, ctypes.byref(h)), "svdq_awq_layer_create")
+    return h
+
+
+def svdq_awq_layer_destroy(h) -> None:
+    lib().svdq_awq_layer_destroy(h)
+
+
+def svdq_awq_forward(h, X, M: int, Y, stream=None) -> None:
+    _check(lib().svdq_awq_forward(h, _ptr(X), M, _ptr(Y), _stream(stream)), "svdq_awq_forward")
+
+
+class AwqLinear:
+    """One awq_w4a16 layer (4-bit weights, bf16 activations) on the current CUDA
+    device, built from canonical prepared weights (svdq_awq_prepare output or a
+    dict with the same arrays); `forward(x)` maps bf16 [M, K] to bf16 [M, N]."""
+
+    def __init__(self, canonical: dict, device=None):
+        import torch
+
+        self.N, self.K = int(canonical["N"]), int(canonical["K"])
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.blob = torch.from_numpy(svdq_awq_pack(canonical)).to(self.device)
+        self.handle = svdq_awq_layer_create(self.blob, self.blob.numel(), self.N, self.K)
+
+    def forward(self, x, out=None, stream=None):
+        import torch
+
+        assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
+        M = x.numel() // self.K
+        y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        svdq_awq_forward(self.handle, x, M, y, stream)
+        return y
+
+    __call__ = forward
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and _lib is not None:
+            _lib.svdq_awq_layer_destroy(h)
             self.handle = None

@@ -445,5 +445,94 @@ int prepare(const uint16_t* W, const uint16_t* bias, const float* act_absmax, fl
   return SVDQ_OK;
 }
 
+// ------------------------------------------------------------------ awq_w4a16
+// Activation-aware preparation of the 4-bit-weight / 16-bit-activation layer:
+// s_j = mean|x_j|^alpha (1 where the mean is 0) for alpha = 0, 0.05, ..., 1;
+// W diag(s) rounded to binary32 and quantized with the INT4 group-64
+// quantizer above; the grid point with the smallest squared output error
+// sum_mn ((f32(x) * inv_s) . deq^T - x . W^T)^2 on the calibration input (the
+// first one on a tie) is kept.  Errors are summed per output row, then over rows
+// in order, so the choice does not depend on the thread count.
+int awq_prepare(const uint16_t* W, const uint16_t* bias, const uint16_t* X, int64_t Mc, svdq_awq_canonical* c) {
+  const int64_t N = c->N, K = c->K, G = K / 64;
+  for (int64_t i = 0; i < N * K; ++i)
+    if (!std::isfinite(bf16_to_f32(W[i]))) return SVDQ_ERR_NUMERIC;
+  for (int64_t i = 0; i < Mc * K; ++i)
+    if (!std::isfinite(bf16_to_f32(X[i]))) return SVDQ_ERR_NUMERIC;
+  std::vector<double> mabs(K, 0.0);
+  for (int64_t m = 0; m < Mc; ++m)
+    for (int64_t k = 0; k < K; ++k) mabs[k] += std::fabs((double)bf16_to_f32(X[m * K + k]));
+  for (int64_t k = 0; k < K; ++k) mabs[k] /= (double)Mc;
+  std::vector<float> xf(Mc * K);
+  for (int64_t i = 0; i < Mc * K; ++i) xf[i] = bf16_to_f32(X[i]);
+  std::vector<double> ref(Mc * N);
+  parallel_for(N, [&](int64_t n) {
+    for (int64_t m = 0; m < Mc; ++m) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += (double)xf[m * K + k] * (double)bf16_to_f32(W[n * K + k]);
+      ref[m * N + n] = acc;
+    }
+  });
+  auto scales_for = [&](double alpha, std::vector<float>& s_f, std::vector<float>& inv) {
+    for (int64_t k = 0; k < K; ++k) {
+      const double sd = mabs[k] > 0.0 ? std::pow(mabs[k], alpha) : 1.0;
+      s_f[k] = (float)sd;
+      inv[k] = (float)(1.0 / (double)s_f[k]);
+    }
+  };
+  auto quant_row = [&](int64_t n, const std::vector<float>& s_f, std::vector<float>& ws, uint8_t* codes,
+                       uint16_t* sc) {
+    for (int64_t k = 0; k < K; ++k) ws[k] = (float)((double)bf16_to_f32(W[n * K + k]) * (double)s_f[k]);
+    quant_int4_rows(1, K, ws.data(), codes, sc);
+  };
+  std::vector<float> s_f(K), inv(K);
+  double best_err = INFINITY;
+  int best = 0;
+  std::vector<double> err_row(N);
+  for (int i = 0; i <= 20; ++i) {
+    const double alpha = i / 20.0;
+    scales_for(alpha, s_f, inv);
+    std::vector<float> xh(Mc * K);
+    for (int64_t m = 0; m < Mc; ++m)
+      for (int64_t k = 0; k < K; ++k) xh[m * K + k] = xf[m * K + k] * inv[k];  // binary32 product
+    parallel_for(N, [&](int64_t n) {
+      std::vector<float> ws(K);
+      std::vector<uint8_t> codes(K / 2);
+      std::vector<uint16_t> sc(G);
+      quant_row(n, s_f, ws, codes.data(), sc.data());
+      double e = 0.0;
+      for (int64_t m = 0; m < Mc; ++m) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+          const uint8_t b = codes[k / 2];
+          int q = (k & 1) ? (b >> 4) : (b & 15);
+          if (q >= 8) q -= 16;
+          acc += (double)xh[m * K + k] * ((double)q * (double)f16_to_f32(sc[k / 64]));
+        }
+        const double d = acc - ref[m * N + n];
+        e += d * d;
+      }
+      err_row[n] = e;
+    });
+    double err = 0.0;
+    for (int64_t n = 0; n < N; ++n) err += err_row[n];
+    if (err < best_err) {
+      best_err = err;
+      best = i;
+    }
+  }
+  const double alpha = best / 20.0;
+  c->alpha = (float)alpha;
+  scales_for(alpha, s_f, inv);
+  std::memcpy(c->s, s_f.data(), K * 4);
+  std::memcpy(c->inv_s, inv.data(), K * 4);
+  parallel_for(N, [&](int64_t n) {
+    std::vector<float> ws(K);
+    quant_row(n, s_f, ws, c->wcodes + n * (K / 2), c->wscales + n * G);
+  });
+  for (int64_t n = 0; n < N; ++n) c->bias[n] = bias ? bias[n] : 0;
+  return SVDQ_OK;
+}
+
 }  // namespace host
 }  // namespace svdq

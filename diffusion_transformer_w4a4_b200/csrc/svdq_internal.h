@@ -102,6 +102,7 @@ namespace svdq {
 
 namespace host {
 int prepare(const uint16_t* W, const uint16_t* bias, const float* act_absmax, float alpha, svdq_canonical* c);
+int awq_prepare(const uint16_t* W, const uint16_t* bias, const uint16_t* X, int64_t Mc, svdq_awq_canonical* c);
 uint16_t f32_to_bf16(float f);
 float bf16_to_f32(uint16_t h);
 float f16_to_f32(uint16_t h);

@@ -213,6 +213,66 @@ svdq_status svdq_forward_noalloc(const svdq_layer* layer, const void* X, int64_t
  * memory and return.  0 restores the default. */
 svdq_status svdq_set_wait_limit(uint64_t cycles);
 
+/* ------------------------------------------------------------------------ */
+/* awq_w4a16: 4-bit weights, 16-bit activations.                            */
+/* ------------------------------------------------------------------------ */
+/* The second runtime layer of "Hugging Face встроила Nunchaku в Diffusers ..."
+ * (paragraph on Nunchaku Lite): precision-sensitive normalization and
+ * modulation layers (adaLN in FLUX) keep bf16 activations and store only the
+ * weights in 4 bits, prepared activation-aware (AWQ).  The pages name it and
+ * give no arithmetic; this library computes
+ *
+ *     y = (f32(x) * inv_s) . dequant( Q4(W diag(s)) )^T + b
+ *
+ * with s_j = mean|x_j|^alpha (1 where the mean is 0), alpha the first point of
+ * the grid 0, 0.05, ..., 1 with the smallest squared output error on the
+ * calibration input, and Q4 the INT4 group-64 quantizer of the svdq_w4a4
+ * residual (symmetric, fp16 scale amax/7, round-half-even codes clamped to
+ * [-8, 7]).  Shapes: K % 64 == 0, 64 <= K <= 12288, N >= 1; M >= 0. */
+typedef struct svdq_awq_canonical {
+  int64_t N, K;
+  float alpha;       /* the grid point chosen */
+  float reserved;
+  float* s;          /* [K] per-input-channel scale, binary32 */
+  float* inv_s;      /* [K] 1/s rounded to binary32 */
+  uint8_t* wcodes;   /* [N, K/2] packed INT4 codes of W diag(s) */
+  uint16_t* wscales; /* [N, K/64] fp16 group scales */
+  uint16_t* bias;    /* [N] bf16 (zeros when the layer has no bias) */
+} svdq_awq_canonical;
+
+/* Byte sizes of the five arrays in struct order: s, inv_s, wcodes, wscales, bias. */
+svdq_status svdq_awq_canonical_sizes(int64_t N, int64_t K, size_t sizes[5]);
+
+/* Host, synchronous, all cores.  W [N,K] bf16, bias [N] bf16 or NULL, X_calib
+ * [M_calib, K] bf16 (the layer's own inputs; M_calib >= 1).  `out` must have N
+ * and K set and its arrays point at caller memory of svdq_awq_canonical_sizes
+ * bytes.  Errors: INVALID_ARG (shape, pointers), NUMERIC (non-finite W or X). */
+svdq_status svdq_awq_prepare(const uint16_t* W, const uint16_t* bias, const uint16_t* X_calib, int64_t M_calib,
+                             svdq_awq_canonical* out);
+
+/* Device layout ("awq blob"), each region 1024-byte aligned: inv_s f32 [K] |
+ * bias f32 [N] | wscales fp16 [N, G'] with G' = K/64 rounded up to even (the
+ * padding entry is zero) | wcodes u8 [N, K/2] (canonical packing,
+ * kept at 4 bits per weight: the layer is a weight-streaming GEMV at the
+ * batch sizes of modulation layers). */
+svdq_status svdq_awq_packed_size(int64_t N, int64_t K, size_t* bytes);
+svdq_status svdq_awq_pack(const svdq_awq_canonical* c, void* blob, size_t blob_bytes);
+
+typedef struct svdq_awq_layer svdq_awq_layer; /* opaque host-side handle */
+
+/* Bind a device-resident awq blob (256-byte aligned) to a handle; allocates no
+ * device memory; UNSUPPORTED_DEVICE on a device other than CC 10.0. */
+svdq_status svdq_awq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K,
+                                  svdq_awq_layer** out);
+void svdq_awq_layer_destroy(svdq_awq_layer* layer);
+
+/* Y[M,N] = layer(X[M,K]), X and Y device pointers (16-byte aligned), `stream`
+ * a cudaStream_t; asynchronous, returns launch errors only.  Token rows are
+ * processed two at a time: the weights are streamed once per pair of rows, so
+ * the kernel is meant for the small M of modulation layers (the batch size);
+ * it is correct for any M. */
+svdq_status svdq_awq_forward(const svdq_awq_layer* layer, const void* X, int64_t M, void* Y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

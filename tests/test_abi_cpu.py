@@ -219,3 +219,78 @@ def test_pack_rejects_non_power_of_two_scales(lib):
     c["g_x"], c["g_w"] = 0.3, 1.0
     with pytest.raises(svdq.SvdqError):
         svdq.svdq_pack(c)
+
+
+# ----------------------------------------------------------------------------- awq_w4a16
+def test_awq_shape_validation(lib):
+    assert svdq.svdq_awq_packed_size(18432, 3072) > 0
+    for bad in [(16, 100), (0, 64), (16, 32), (16, 12288 + 64)]:
+        with pytest.raises(svdq.SvdqError) as e:
+            svdq.svdq_awq_packed_size(*bad)
+        assert e.value.status == svdq.SVDQ_ERR_INVALID_ARG
+
+
+def test_awq_prepare_rejects_non_finite(lib):
+    W = np.zeros((16, 64), np.uint16)
+    X = np.zeros((2, 64), np.uint16)
+    X[1, 3] = 0x7FC0  # bf16 NaN
+    with pytest.raises(svdq.SvdqError) as e:
+        svdq.svdq_awq_prepare(W, None, X)
+    assert e.value.status == svdq.SVDQ_ERR_NUMERIC
+
+
+@pytest.mark.parametrize("shape", [(2, 256, 48), (64, 512, 96)])
+def test_awq_product_prepare_agrees_with_oracle(lib, shape):
+    """The library's activation-aware preparation picks the oracle's alpha (or
+    one whose error ties it to 1e-9 relative) and then the same codes and scales
+    (its error sums run in another order; the scales use the same pow)."""
+    M, K, N = shape
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[:, rng.choice(K, 3, replace=False)] *= 50.0
+    X = wl.f32_to_bf16_bits(x)
+    W = wl.f32_to_bf16_bits(rng.standard_normal((N, K)).astype(np.float32) * 0.02)
+    b = wl.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32) * 0.01)
+    ours = svdq.svdq_awq_prepare(W, b, X)
+    ref = oracle.awq_prepare(W, b, X)
+    if np.float32(ours["alpha"]) != np.float32(ref["alpha"]):  # the ABI stores alpha as binary32
+        a = min(oracle.AWQ_ALPHAS, key=lambda g: abs(g - ours["alpha"]))
+        e_ours = oracle.awq_output_error(X, W, oracle.awq_mean_abs(X), a)
+        assert abs(e_ours - ref["err"]) <= 1e-9 * ref["err"], (ours["alpha"], ref["alpha"])
+        ref = dict(ref)
+        _, ref["s"], ref["inv_s"] = oracle.awq_channel_scales(oracle.awq_mean_abs(X), a)
+        ref["wcodes"], ref["wscales"] = oracle.awq_quant_weights(W, ref["s"])
+    np.testing.assert_array_equal(ours["s"], ref["s"])
+    np.testing.assert_array_equal(ours["inv_s"], ref["inv_s"])
+    np.testing.assert_array_equal(ours["wcodes"], ref["wcodes"])
+    np.testing.assert_array_equal(ours["wscales"], ref["wscales"])
+    np.testing.assert_array_equal(ours["bias"], b)
+
+
+@pytest.mark.parametrize("K", [192, 256])
+def test_awq_pack_layout(lib, K):
+    N = 40
+    rng = np.random.default_rng(12)
+    c = svdq._awq_arrays(N, K)
+    c["inv_s"][:] = rng.uniform(0.5, 2, K)
+    c["s"][:] = 1.0 / c["inv_s"]
+    c["wcodes"][:] = rng.integers(0, 256, c["wcodes"].shape)
+    c["wscales"][:] = rng.integers(0, 0x7BFF, c["wscales"].shape)
+    c["bias"][:] = oracle.f32_to_bf16(rng.standard_normal(N).astype(np.float32))
+    blob = svdq.svdq_awq_pack(c)
+    o = 0
+    def take(nbytes):
+        nonlocal o
+        start = o
+        o = (o + nbytes + 1023) // 1024 * 1024
+        return start
+    G = K // 64
+    ld = (G + 1) // 2 * 2  # scale rows padded to an even count
+    o_is, o_b, o_ws, o_wc = take(K * 4), take(N * 4), take(N * ld * 2), take(N * K // 2)
+    assert blob.size == o
+    assert np.array_equal(blob[o_is:o_is + 4 * K].view(np.float32), c["inv_s"])
+    assert np.array_equal(blob[o_b:o_b + 4 * N].view(np.float32), oracle.bf16_to_f32(c["bias"]))
+    ws = blob[o_ws:o_ws + N * ld * 2].view(np.uint16).reshape(N, ld)
+    assert np.array_equal(ws[:, :G], c["wscales"])
+    assert np.all(ws[:, G:] == 0)
+    assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"])

@@ -92,6 +92,17 @@ def block_layers(rank: int, M: int = BLOCK_M):
     ]
 
 
+# awq_w4a16 layers: FLUX adaLN modulation linears.  Their input is the per-sample
+# conditioning vector, so M is the batch (2 = the classifier-free-guidance pair);
+# double-stream blocks map 3072 -> 6 x 3072, single-stream blocks 3072 -> 3 x 3072.
+# Same value recipe as the FLUX-style svdq layers (N(0,1), 0.5 % channels x50).
+AWQ = "awq"
+AWQ_LAYERS = {
+    "awq_flux_double_mod_2x3072x18432": _flux(2, 3072, 18432, 0, AWQ, "awq_double_mod", 20),
+    "awq_flux_single_mod_2x3072x9216": _flux(2, 3072, 9216, 0, AWQ, "awq_single_mod", 21),
+}
+
+
 def _rng(seed: int, layer_id: int, stream: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, layer_id, stream])))
 
