@@ -100,6 +100,7 @@ _EXPORTS = {
     "svdq_awq_layer_create": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int64,
                                              ctypes.POINTER(ctypes.c_void_p)]),
     "svdq_awq_layer_destroy": (None, [ctypes.c_void_p]),
+    "svdq_awq_read_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "svdq_awq_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                         ctypes.c_void_p]),
 }
@@ -395,6 +396,12 @@ def svdq_awq_layer_destroy(h) -> None:
     lib().svdq_awq_layer_destroy(h)
 
 
+def svdq_awq_read_status(h) -> int:
+    v = ctypes.c_int()
+    _check(lib().svdq_awq_read_status(h, ctypes.byref(v)), "svdq_awq_read_status")
+    return v.value
+
+
 def svdq_awq_forward(h, X, M: int, Y, stream=None) -> None:
     _check(lib().svdq_awq_forward(h, _ptr(X), M, _ptr(Y), _stream(stream)), "svdq_awq_forward")
 
@@ -422,6 +429,9 @@ class AwqLinear:
         return y
 
     __call__ = forward
+
+    def status(self) -> int:
+        return svdq_awq_read_status(self.handle)
 
     def __del__(self):
         h = getattr(self, "handle", None)

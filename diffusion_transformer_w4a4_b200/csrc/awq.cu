@@ -8,16 +8,20 @@
 // layer is a weight-streaming matrix-vector product, bound by reading the
 // 4-bit weights from HBM, so it runs on CUDA cores and keeps the weights packed.
 //
-// k_awq_gemv: one thread per 32-code (16-byte) chunk of K.  A thread keeps
-// its chunk of x^ = f32(x) * inv_s for up to two token rows in registers and
-// streams the matching 16 bytes of every weight row, eight rows per batch (one
-// load each, all in flight together).  A code u (two's complement nibble n,
-// u = n ^ 8 in [0, 15], value u - 8) is turned into the binary32 1 + u/16 by
-// placing u in the mantissa (byte arithmetic and one byte permute per code), so
-// a chunk's sum is
-//   sum_e (u_e - 8) x^_e = 16 sum_e (1 + u_e/16) x^_e - 24 sum_e x^_e,
-// with the last sum computed once per thread.  The chunk's partial times its
-// group scale is reduced over the CTA (warp shuffles, then shared memory).
+// k_awq_gemv: a thread owns one 32-code (16-byte) chunk of K and keeps that
+// chunk of x^ = f32(x) * inv_s for up to two token rows in registers; it reads
+// the matching 16 bytes of several weight rows from a shared-memory ring that a
+// producer warp fills with bulk copies of consecutive rows.  The device copy of
+// the codes is offset binary (u = n + 8 in [0, 15] for the two's complement
+// nibble n).  A code becomes a binary32 with one logic operation, u masked into
+// the mantissa of 1.0 at bit p, and an exact packed subtraction of 1 leaves
+// u 2^(p-23); the x^ chunk is pre-scaled by 2^(23-p) once, so the packed FMAs
+// accumulate sum_e u_e x^_e directly (no cancelling offset), and a chunk's sum
+// is that minus 8 sum_e x^_e.  The partial times its group scale is reduced over
+// the thread's row group (warp shuffles, then shared memory).  The pre-scaling
+// by at most 2^15 needs |x^| < 2^113.  The decode's integer work (10 logic and
+// shift operations per 8 codes on the half-rate ALU pipe) rather than HBM is
+// the first limit at these shapes.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -35,22 +39,28 @@ struct svdq_awq_layer {
   const float* bias;
   const uint16_t* wscales;
   const uint8_t* wcodes;
+  int* status;
 };
 
 namespace svdq {
 namespace {
 
-constexpr int kAwqRows = 8;  // weight rows per batch
-constexpr int kAwqMaxMB = 2;  // token rows per launch (their x^ chunks live in registers)
-constexpr int kAwqStagesMax = 4;  // weight batches in flight per CTA (2 for the widest K)
+constexpr int kAwqRpt = 4;           // weight rows per row group and batch
+constexpr int kAwqMaxMB = 2;         // token rows per launch (their x^ chunks live in registers)
+constexpr int kAwqMaxStages = 6;     // ring depth bound
+constexpr int kAwqConsumers = 384;   // consumer threads per CTA, at most
+constexpr int kAwqMaxThreads = kAwqConsumers + 32;  // plus the producer warp
+constexpr size_t kAwqRingBudget = 110 * 1024;  // ring bytes per CTA: two CTAs per SM
+// 2^(23 - p) for the mantissa position p at which code k of a 32-bit word is decoded
+__constant__ float kAwqPrescale[8] = {32768.f, 2048.f, 32768.f, 2048.f, 128.f, 32768.f, 2048.f, 128.f};
 
 struct AwqBlob {
-  size_t inv_s, bias, wscales, wcodes, total;
+  size_t inv_s, bias, wscales, wcodes, status, total;
 };
 
-// fp16 group scales per blob row: K/64 rounded up to even, so every row starts
-// 4-byte aligned and a thread's 4-byte scale pair stays inside its row
-__host__ __device__ inline int64_t awq_scale_ld(int64_t K) { return (K / 64 + 1) / 2 * 2; }
+// fp16 group scales per blob row: K/64 rounded up to a multiple of 8, so a run
+// of rows is a whole number of 16-byte units for the bulk copies
+__host__ __device__ inline int64_t awq_scale_ld(int64_t K) { return (K / 64 + 7) / 8 * 8; }
 
 AwqBlob awq_blob_layout(int64_t N, int64_t K) {
   auto up = [](size_t x) { return (x + kAlign - 1) / kAlign * kAlign; };
@@ -64,6 +74,8 @@ AwqBlob awq_blob_layout(int64_t N, int64_t K) {
   o = up(o + (size_t)N * awq_scale_ld(K) * 2);
   b.wcodes = o;
   o = up(o + (size_t)N * (K / 2));
+  b.status = o;  // int32 written by the kernel on a device-side error
+  o = up(o + 16);
   b.total = o;
   return b;
 }
@@ -72,6 +84,12 @@ bool awq_shape_ok(int64_t N, int64_t K) { return N >= 1 && K >= 64 && K % 64 == 
 
 struct AwqParams {
   int M, N, K, m0;
+  int T;       // threads per row group: K/32 rounded up to whole warps
+  int G;       // row groups per CTA (a power of two, at most 8)
+  int stages;  // ring depth
+  int xs_off;  // byte offset of the x^ staging area (the ring's tail, reused once set up)
+  int* status;
+  unsigned long long limit;
   const uint16_t* x;
   const float* inv_s;
   const uint8_t* codes;
@@ -80,161 +98,221 @@ struct AwqParams {
   uint16_t* y;
 };
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+template <int S>
+__device__ __forceinline__ uint32_t shl_b32(uint32_t v) {
+  uint32_t r;
+  asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "n"(S));
+  return r;
 }
-__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+template <int S>
+__device__ __forceinline__ uint32_t shr_b32(uint32_t v) {
+  uint32_t r;
+  asm("shr.b32 %0, %1, %2;" : "=r"(r) : "r"(v), "n"(S));
+  return r;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// binary32 with bits (w & mask) over the encoding of 1.0: one lop3, (a & b) | c
+__device__ __forceinline__ float mant_one(uint32_t w, uint32_t mask) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(mask), "r"(0x3F800000u));
+  return __uint_as_float(r);
 }
 
-// Persistent: a CTA walks batches of kAwqRows weight rows.  Each thread copies
-// its own 16-byte chunk of the batches ahead, and the 4-byte pair of fp16
-// group scales that holds its chunk's scale, into a STG-deep ring in
-// shared memory (cp.async) and reads back only what it copied, so the group
-// wait alone orders the pipeline.
-template <int MB, int STG>
-__global__ void __launch_bounds__(384) k_awq_gemv(const __grid_constant__ AwqParams p) {
-  // [STG][kAwqRows][threads] 16-byte weight chunks, then the same
-  // index space of 4-byte scale pairs
-  extern __shared__ __align__(16) uint8_t awq_smem[];
-  __shared__ float red[12][kAwqRows * MB];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x, nwarps = nthr >> 5;
-  const int nchunk = p.K >> 5;
-  const bool active = tid < nchunk;
-  const int k0 = tid * 32;
+// Persistent and warp-specialized.  The CTA's last warp is the producer: its
+// lane 0 fills a ring of `stages` batches, each R = G * kAwqRpt consecutive
+// weight rows (the rows' packed codes and their scale rows, two bulk copies,
+// both contiguous), completing on per-stage "full" mbarriers.  The other warps
+// form G row groups of T threads: thread t of a group owns the 32-code chunk t
+// of K, with that chunk of x^ = f32(x) * inv_s for each token row in registers,
+// and group g computes rows g*kAwqRpt .. g*kAwqRpt + kAwqRpt - 1 of every batch.
+// A group reduces its partial sums over its warps (shuffles, then shared memory
+// and a named barrier of its own), releases the stage on the stage's "empty"
+// mbarrier (one arrival per group) and its first threads add the bias and store
+// y.  Groups never wait for one another.  Waits are bounded; a group whose
+// wait fails leaves as a whole (the named barrier reduces the outcome), the
+// producer drains its copies, and the status word records the error.
+template <int MB>
+__global__ void __launch_bounds__(kAwqMaxThreads) k_awq_gemv(const __grid_constant__ AwqParams p) {
+  extern __shared__ __align__(128) uint8_t awq_smem[];  // [stages][R scale rows] then [stages][R rows of codes]
+  __shared__ float red[2][kAwqConsumers / 32][kAwqRpt * MB];  // per-warp partials, by batch parity
+  __shared__ uint64_t full[kAwqMaxStages], empty[kAwqMaxStages];
+  __shared__ uint64_t xs_free;  // every consumer warp has its x^ chunk in registers
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int T = p.T, G = p.G, S = p.stages;
+  const int R = G * kAwqRpt;
+  const int nbatch = (p.N + R - 1) / R;
+  const size_t row_bytes = (size_t)p.K / 2, ld = (size_t)awq_scale_ld(p.K);
+  const size_t wstage = (size_t)R * row_bytes, sstage = (size_t)R * ld * 2;
+  uint8_t* sring = awq_smem;
+  uint8_t* wring = awq_smem + (size_t)S * sstage;
+  WaitCtl wc{&abort_flag, p.status, p.limit};
 
-  const size_t row_bytes = (size_t)p.K / 2, row_groups = (size_t)awq_scale_ld(p.K);
-  const int stride = gridDim.x * kAwqRows;
-  const size_t nslots = (size_t)STG * kAwqRows * nthr;
-  auto slot = [&](int st, int r) -> size_t { return ((size_t)st * kAwqRows + r) * nthr + tid; };
-  auto wslot = [&](int st, int r) -> uint8_t* { return awq_smem + slot(st, r) * 16; };
-  auto sslot = [&](int st, int r) -> uint8_t* { return awq_smem + nslots * 16 + slot(st, r) * 4; };
-  auto issue = [&](int nb, int st) {
-#pragma unroll
-    for (int r = 0; r < kAwqRows; ++r) {
-      const int n = nb + r;
-      if (active && n < p.N) {
-        cp_async16(wslot(st, r), p.codes + (size_t)n * row_bytes + 16 * (size_t)tid);
-        // groups 2(tid/4) and 2(tid/4)+1: a 4-byte-aligned pair holding this chunk's group tid/2
-        cp_async4(sslot(st, r), p.scales + (size_t)n * row_groups + 2 * (tid >> 2));
+  if (tid == 0) {
+    for (int j = 0; j < S; ++j) {
+      mbar_init(&full[j], 1);
+      mbar_init(&empty[j], G);
+    }
+    mbar_init(&xs_free, (G * T) >> 5);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (tid >= G * T) {  // ---------------------------------------- producer
+    if (lane != 0) return;
+    int s = 0, j = 0;
+    uint32_t ph = 0;  // parity of the current fill of stage s
+    const size_t xs_lo = (size_t)p.xs_off;
+    for (int b = blockIdx.x; b < nbatch; b += gridDim.x, ++j) {
+      if (j >= S && !mbar_wait(&empty[s], ph ^ 1, wc)) break;  // the previous fill's batch is released
+      if (j < S && S * sstage + (s + 1) * wstage > xs_lo &&
+          !mbar_wait(&xs_free, 0, wc))
+        break;  // a first fill that overwrites the x^ staging area waits until it is read
+      const int rows = (p.N - b * R) < R ? (p.N - b * R) : R;
+      mbar_arrive_expect_tx(&full[s], (uint32_t)(rows * (row_bytes + ld * 2)));
+      bulk_load(wring + s * wstage, p.codes + (size_t)b * R * row_bytes, (uint32_t)(rows * row_bytes), &full[s]);
+      bulk_load(sring + s * sstage, p.scales + (size_t)b * R * ld, (uint32_t)(rows * ld * 2), &full[s]);
+      if (++s == S) {
+        s = 0;
+        ph ^= 1;
       }
     }
-  };
-
-  const int nb0 = blockIdx.x * kAwqRows;
-#pragma unroll
-  for (int j = 0; j < STG - 1; ++j) {  // prologue: the first batches in flight
-    issue(nb0 + j * stride, j);
-    cp_async_commit();
-  }
-
-  // this thread's 32 activations of each token row, times 1/s (while the
-  // first weight batches are on their way)
-  float xh[MB][32];
-  float xsum[MB];
-#pragma unroll
-  for (int m = 0; m < MB; ++m) {
-    xsum[m] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) xh[m][e] = 0.f;
-  }
-  if (active) {
-    float is[32];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 v = __ldg((const float4*)(p.inv_s + k0) + q);
-      is[4 * q] = v.x;
-      is[4 * q + 1] = v.y;
-      is[4 * q + 2] = v.z;
-      is[4 * q + 3] = v.w;
+    if (abort_flag) {  // the ring must not be left with copies in flight
+      for (int st = 0; st < S && st < j; ++st) mbar_wait_drain(&full[st], ((j - 1 - st) / S) & 1, p.limit);
     }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int g = tid / T, t = tid - g * T;
+  const int warp = tid >> 5, wbase = g * (T >> 5);
+  const int nchunk = p.K >> 5;
+  const bool active = t < nchunk;
+
+  // x^ = f32(x) * inv_s for the CTA's token rows, computed once with coalesced
+  // loads into the ring's tail; float4 q of chunk c of token m sits at unit
+  // m*K/4 + c*8 + (q ^ (c & 7)), so that each thread's reads of its own chunk
+  // are free of bank conflicts
+  {
+    float4* xs = (float4*)(awq_smem + p.xs_off);
+    const int kq = p.K >> 2;
+    for (int i = tid; i < MB * kq; i += G * T) {
+      const int m = i / kq, w = i - m * kq;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (p.m0 + m < p.M) {
+        const float4 is = __ldg((const float4*)p.inv_s + w);
+        const uint2 xv = __ldg((const uint2*)(p.x + (size_t)(p.m0 + m) * p.K) + w);
+        o.x = __uint_as_float(xv.x << 16) * is.x;  // binary32 products, as in the smoothing step
+        o.y = __uint_as_float(xv.x & 0xFFFF0000u) * is.y;
+        o.z = __uint_as_float(xv.y << 16) * is.z;
+        o.w = __uint_as_float(xv.y & 0xFFFF0000u) * is.w;
+      }
+      const int c = w >> 3, q = w & 7;
+      xs[m * kq + c * 8 + (q ^ (c & 7))] = o;
+    }
+  }
+  named_bar_sync(9, G * T);  // the consumers only (barriers 1..8 belong to the row groups)
+  float2 xh[MB][16];  // pairs (x^_2j, x^_2j+1) of the chunk, pre-scaled for the decode
+  float xsum[MB];
+  {
+    const float4* xs = (const float4*)(awq_smem + p.xs_off);
+    const int kq = p.K >> 2;
 #pragma unroll
     for (int m = 0; m < MB; ++m) {
-      if (p.m0 + m >= p.M) continue;
-      const uint4* xr = (const uint4*)(p.x + (size_t)(p.m0 + m) * p.K + k0);
+      xsum[m] = 0.f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = __ldg(xr + q);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int e = 8 * q + 2 * h;
-          xh[m][e] = __uint_as_float(w[h] << 16) * is[e];  // binary32 product, as in the smoothing step
-          xh[m][e + 1] = __uint_as_float(w[h] & 0xFFFF0000u) * is[e + 1];
-        }
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = active ? xs[m * kq + t * 8 + (q ^ (t & 7))] : make_float4(0.f, 0.f, 0.f, 0.f);
+        xsum[m] += v.x;
+        xsum[m] += v.y;
+        xsum[m] += v.z;
+        xsum[m] += v.w;
+        // pre-scale by 2^(23 - p) for the mantissa position p of each code's
+        // nibble in the decode below (exact: powers of two)
+        xh[m][2 * q] = make_float2(v.x * kAwqPrescale[(4 * q) & 7], v.y * kAwqPrescale[(4 * q + 1) & 7]);
+        xh[m][2 * q + 1] = make_float2(v.z * kAwqPrescale[(4 * q + 2) & 7], v.w * kAwqPrescale[(4 * q + 3) & 7]);
       }
-#pragma unroll
-      for (int e = 0; e < 32; ++e) xsum[m] += xh[m][e];
     }
   }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&xs_free);
 
-  int it = 0;
-  for (int nb = nb0; nb < p.N; nb += stride, ++it) {
-    issue(nb + (STG - 1) * stride, (it + STG - 1) % STG);
-    cp_async_commit();
-    cp_async_wait<STG - 1>();  // this batch's own copies have landed
-    const int st = it % STG;
-    float part[kAwqRows][MB];
+  const int fr = t / MB, fm = t - (t / MB) * MB;  // finishing thread t: group row fr, token fm
+  int s = 0, j = 0;
+  uint32_t ph = 0;
+  for (int b = blockIdx.x; b < nbatch; b += gridDim.x, ++j) {
+    const int n0 = b * R + g * kAwqRpt;  // this group's first row
+    float bias_v = 0.f;
+    if (t < kAwqRpt * MB && n0 + fr < p.N) bias_v = __ldg(p.bias + n0 + fr);
+    const bool ok = mbar_wait(&full[s], ph, wc);
+    float part[kAwqRpt][MB];
 #pragma unroll
-    for (int r = 0; r < kAwqRows; ++r) {
-      uint4 wv = make_uint4(0u, 0u, 0u, 0u);
-      float sc = 0.f;
-      if (active && nb + r < p.N) {
-        wv = *(const uint4*)wslot(st, r);
-        const uint32_t pair = *(const uint32_t*)sslot(st, r);
-        sc = __half2float(__ushort_as_half((unsigned short)(((tid >> 1) & 1) ? (pair >> 16) : (pair & 0xFFFFu))));
-      }
-      const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
-      float acc[MB];
+    for (int r = 0; r < kAwqRpt; ++r)
 #pragma unroll
-      for (int m = 0; m < MB; ++m) acc[m] = 0.f;
+      for (int m = 0; m < MB; ++m) part[r][m] = 0.f;
+    if (ok) {
+      const uint8_t* ws = wring + s * wstage + (size_t)g * kAwqRpt * row_bytes;
+      const uint16_t* ss = (const uint16_t*)(sring + s * sstage) + (size_t)g * kAwqRpt * ld;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // offset-binary codes u = n ^ 8; each byte of te / to becomes the third
-        // byte 0x80 | u << 3 of the binary32 1 + u/16 for the even / odd code of
-        // that byte, and one byte permute per code adds the top byte 0x3F
-        const uint32_t v = wr[j] ^ 0x88888888u;
-        const uint32_t te = ((v << 3) & 0x78787878u) | 0x80808080u;
-        const uint32_t to = ((v >> 1) & 0x78787878u) | 0x80808080u;
+      for (int r = 0; r < kAwqRpt; ++r) {
+        if (!active || n0 + r >= p.N) continue;
+        const uint4 wv = *(const uint4*)(ws + r * row_bytes + 16 * t);
+        const float sc = __half2float(__ushort_as_half(ss[r * ld + (t >> 1)]));
+        const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+        float2 acc[MB];  // even- and odd-position codes, one packed FMA per pair
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float fe = __uint_as_float(__byte_perm(te, 0x3F000000u, 0x7054u | (i << 8)));
-          const float fo = __uint_as_float(__byte_perm(to, 0x3F000000u, 0x7054u | (i << 8)));
+        for (int m = 0; m < MB; ++m) acc[m] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // code k of word q (bits 4k..4k+3, offset binary u) is masked into the
+          // mantissa of 1.0 at bit p = 8, 12, 8, 12, 16, 8, 12, 16 (from the word
+          // shifted left by 8 for k < 2, as is for k = 2..4, shifted right by 12
+          // for k > 4): one logic operation makes 1 + u 2^(p-23), and subtracting
+          // 1 leaves u 2^(p-23) exactly, which meets the pre-scaled x^
+          // (written as explicit shifts and 3-input logic operations, so that the
+          // shifted words are computed once rather than re-derived per code)
+          const uint32_t v = wr[q], a = shl_b32<8>(v), c = shr_b32<12>(v);
+          const float2 m1 = make_float2(-1.f, -1.f);
+          const float2 g01 = __fadd2_rn(make_float2(mant_one(a, 0x00F00u), mant_one(a, 0x0F000u)), m1);
+          const float2 g23 = __fadd2_rn(make_float2(mant_one(v, 0x00F00u), mant_one(v, 0x0F000u)), m1);
+          const float2 g45 = __fadd2_rn(make_float2(mant_one(v, 0xF0000u), mant_one(c, 0x00F00u)), m1);
+          const float2 g67 = __fadd2_rn(make_float2(mant_one(c, 0x0F000u), mant_one(c, 0xF0000u)), m1);
 #pragma unroll
           for (int m = 0; m < MB; ++m) {
-            acc[m] = fmaf(fe, xh[m][8 * j + 2 * i], acc[m]);
-            acc[m] = fmaf(fo, xh[m][8 * j + 2 * i + 1], acc[m]);
+            acc[m] = __ffma2_rn(g01, xh[m][4 * q], acc[m]);
+            acc[m] = __ffma2_rn(g23, xh[m][4 * q + 1], acc[m]);
+            acc[m] = __ffma2_rn(g45, xh[m][4 * q + 2], acc[m]);
+            acc[m] = __ffma2_rn(g67, xh[m][4 * q + 3], acc[m]);
           }
         }
-      }
+        // sum_e (u_e - 8) x^_e = sum_e u_e x^_e - 8 sum_e x^_e
 #pragma unroll
-      for (int m = 0; m < MB; ++m) part[r][m] = sc * fmaf(16.f, acc[m], -24.f * xsum[m]);
+        for (int m = 0; m < MB; ++m) part[r][m] = sc * fmaf(-8.f, xsum[m], acc[m].x + acc[m].y);
+      }
     }
 #pragma unroll
-    for (int r = 0; r < kAwqRows; ++r)
+    for (int r = 0; r < kAwqRpt; ++r)
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
         float v = part[r][m];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[warp][r * MB + m] = v;
+        if (lane == 0) red[j & 1][warp][r * MB + m] = v;
       }
-    __syncthreads();
-    if (tid < kAwqRows * MB) {
-      const int r = tid / MB, m = tid % MB, n = nb + r;
+    if (!named_bar_and(1 + g, T, ok)) break;  // the group's reads of stage s and its partials are done
+    if (t == 0) mbar_arrive(&empty[s]);
+    if (t < kAwqRpt * MB) {
       float v = 0.f;
-      for (int wi = 0; wi < nwarps; ++wi) v += red[wi][tid];
-      if (n < p.N && p.m0 + m < p.M)
-        p.y[(size_t)(p.m0 + m) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v + p.bias[n]));
+      for (int w = 0; w < (T >> 5); ++w) v += red[j & 1][wbase + w][t];
+      const int n = n0 + fr;
+      if (n < p.N && p.m0 + fm < p.M)
+        p.y[(size_t)(p.m0 + fm) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v + bias_v));
     }
-    __syncthreads();
+    if (++s == S) {
+      s = 0;
+      ph ^= 1;
+    }
   }
-  cp_async_wait<0>();  // no copy may still target shared memory when the CTA exits
 }
 
 int awq_sm_count(int dev) {
@@ -248,36 +326,48 @@ int awq_sm_count(int dev) {
   return cache[dev];
 }
 
-// Shared memory of one CTA: STG stages of kAwqRows 16-byte chunks and 4-byte
-// scale pairs per thread.
-constexpr size_t awq_smem_bytes(int stg, int threads) { return (size_t)stg * kAwqRows * threads * 20; }
+// Launch shape for a K: row groups, ring depth and dynamic shared memory.
+struct AwqShape {
+  int T, G, stages, xs_off;
+  size_t smem;
+};
+AwqShape awq_shape(int K, int MB) {
+  AwqShape a{};
+  a.T = ((K / 32) + 31) / 32 * 32;
+  a.G = 1;
+  while (a.G < 8 && 2 * a.G * a.T <= kAwqConsumers) a.G *= 2;
+  const size_t stage = (size_t)a.G * kAwqRpt * ((size_t)K / 2 + (size_t)awq_scale_ld(K) * 2);
+  size_t st = kAwqRingBudget / stage;
+  a.stages = (int)(st < 2 ? 2 : (st > (size_t)kAwqMaxStages ? (size_t)kAwqMaxStages : st));
+  const size_t ring = (size_t)a.stages * stage, xs = (size_t)MB * K * 4;
+  a.xs_off = ring >= xs ? (int)((ring - xs) / 128 * 128) : 0;
+  a.smem = ring > (size_t)a.xs_off + xs ? ring : (size_t)a.xs_off + xs;
+  return a;
+}
 
-// CTAs per SM for one kernel variant and block size, found once per device and
-// cached (the attribute call and the occupancy query cost microseconds of host
-// time that would otherwise precede every launch)
-// The largest block a variant is launched with: four stages up to 256 threads
-// (K <= 8192), two stages up to 384.  The dynamic shared-memory attribute belongs
-// to the kernel, not to a block size, so it is set once to this largest need.
-constexpr int awq_max_threads(int stg) { return stg == kAwqStagesMax ? 256 : 384; }
-
-template <int MB, int STG>
-int awq_blocks_per_sm(int dev, int threads) {
+// CTAs per SM for one kernel variant and K, found once per device and cached:
+// the attribute call and the occupancy query cost microseconds of host time
+// that would otherwise precede every launch.  The dynamic shared-memory
+// attribute belongs to the kernel, not to a launch, so it is set once to the
+// ring budget, which bounds every K's ring.
+template <int MB>
+int awq_blocks_per_sm(int dev, const AwqShape& a, int K) {
   static std::mutex mu;
-  static int cache[64][13] = {};  // [device][threads / 32]
+  static int cache[64][12288 / 64 + 1] = {};  // [device][K / 64]
   static bool attr_set[64] = {};
-  if (dev < 0 || dev >= 64 || threads < 32 || threads > awq_max_threads(STG)) return -1;
+  if (dev < 0 || dev >= 64 || K < 64 || K > 12288 || a.smem > kAwqRingBudget) return -1;
   std::lock_guard<std::mutex> lock(mu);
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(k_awq_gemv<MB, STG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)awq_smem_bytes(STG, awq_max_threads(STG))) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_awq_gemv<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAwqRingBudget) !=
+        cudaSuccess)
       return -1;
     attr_set[dev] = true;
   }
-  int& c = cache[dev][threads / 32];
+  int& c = cache[dev][K / 64];
   if (c == 0) {
-    const size_t smem = awq_smem_bytes(STG, threads);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_awq_gemv<MB, STG>, threads, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_awq_gemv<MB>, a.G * a.T + 32, a.smem) !=
+            cudaSuccess ||
         per_sm < 1)
       return -1;
     c = per_sm;
@@ -285,27 +375,21 @@ int awq_blocks_per_sm(int dev, int threads) {
   return c;
 }
 
-template <int MB, int STG>
-int launch_awq_stg(const AwqParams& p, int dev, int threads, cudaStream_t stream) {
-  const int per_sm = awq_blocks_per_sm<MB, STG>(dev, threads);
-  if (per_sm < 1) return SVDQ_ERR_CUDA;
-  // enough CTAs to fill the SMs, but each walking several batches so that its
-  // ring reaches steady state (a CTA's setup and first round trip are not hidden)
-  const int batches = (p.N + kAwqRows - 1) / kAwqRows;
-  const int sms = awq_sm_count(dev);
-  int grid = sms * per_sm;
-  const int by_work = batches / STG;
-  if (grid > by_work) grid = by_work > sms ? by_work : sms;
-  if (grid > batches) grid = batches;
-  k_awq_gemv<MB, STG><<<grid, threads, awq_smem_bytes(STG, threads), stream>>>(p);
-  return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
-}
-
 template <int MB>
-int launch_awq(const AwqParams& p, int dev, cudaStream_t stream) {
-  const int threads = ((p.K / 32) + 31) / 32 * 32;
-  if (threads <= awq_max_threads(kAwqStagesMax)) return launch_awq_stg<MB, kAwqStagesMax>(p, dev, threads, stream);
-  return launch_awq_stg<MB, 2>(p, dev, threads, stream);
+int launch_awq(AwqParams p, int dev, cudaStream_t stream) {
+  const AwqShape a = awq_shape(p.K, MB);
+  p.T = a.T;
+  p.xs_off = a.xs_off;
+  p.G = a.G;
+  p.stages = a.stages;
+  const int per_sm = awq_blocks_per_sm<MB>(dev, a, p.K);
+  if (per_sm < 1) return SVDQ_ERR_CUDA;
+  const int R = a.G * kAwqRpt;
+  const int nbatch = (p.N + R - 1) / R;
+  int grid = awq_sm_count(dev) * per_sm;
+  if (grid > nbatch) grid = nbatch;
+  k_awq_gemv<MB><<<grid, a.G * a.T + 32, a.smem, stream>>>(p);
+  return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
 }  // namespace
@@ -355,7 +439,10 @@ svdq_status svdq_awq_pack(const svdq_awq_canonical* c, void* blob_v, size_t blob
   for (int64_t n = 0; n < N; ++n) bias[n] = c->bias ? host::bf16_to_f32(c->bias[n]) : 0.f;
   const int64_t G = K / 64, ld = awq_scale_ld(K);
   for (int64_t n = 0; n < N; ++n) std::memcpy(blob + b.wscales + (size_t)n * ld * 2, c->wscales + n * G, (size_t)G * 2);
-  std::memcpy(blob + b.wcodes, c->wcodes, (size_t)N * (K / 2));
+  // offset binary on the device: nibble n -> n ^ 8 = n + 8 (mod 16), per nibble
+  const uint8_t* src = c->wcodes;
+  uint8_t* dst = blob + b.wcodes;
+  for (size_t i = 0, e = (size_t)N * (K / 2); i < e; ++i) dst[i] = src[i] ^ 0x88u;
   return SVDQ_OK;
 }
 
@@ -383,11 +470,20 @@ svdq_status svdq_awq_layer_create(const void* dev_blob, size_t blob_bytes, int64
   L->bias = (const float*)(base + b.bias);
   L->wscales = (const uint16_t*)(base + b.wscales);
   L->wcodes = base + b.wcodes;
+  L->status = (int*)(base + b.status);
   *out = L;
   return SVDQ_OK;
 }
 
 void svdq_awq_layer_destroy(svdq_awq_layer* layer) { delete layer; }
+
+svdq_status svdq_awq_read_status(const svdq_awq_layer* L, int* device_status) {
+  if (!L || !device_status) return SVDQ_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaMemcpy(&v, L->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
+  *device_status = v;
+  return SVDQ_OK;
+}
 
 svdq_status svdq_awq_forward(const svdq_awq_layer* L, const void* X, int64_t M, void* Y, void* stream) {
   if (!L || M < 0) return SVDQ_ERR_INVALID_ARG;
@@ -403,6 +499,8 @@ svdq_status svdq_awq_forward(const svdq_awq_layer* L, const void* X, int64_t M, 
   p.scales = L->wscales;
   p.bias = L->bias;
   p.y = (uint16_t*)Y;
+  p.status = L->status;
+  p.limit = wait_limit_cycles();
   cudaStream_t s = (cudaStream_t)stream;
   for (int64_t m0 = 0; m0 < M; m0 += kAwqMaxMB) {
     p.m0 = (int)m0;

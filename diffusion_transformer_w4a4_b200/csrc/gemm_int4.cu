@@ -96,20 +96,6 @@ struct I4Params {
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
 
-__device__ __forceinline__ void mul2(float& a0, float& a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
-      "mul.rn.f32x2 z, x, y;\n\tmov.b64 {%0, %1}, z;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(b0), "f"(b1));
-}
-// (y0, y1) += (a0, a1) * (b0, b1), one rounding each
-__device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %5};\n\tmov.b64 z, {%0, %1};\n\t"
-      "fma.rn.f32x2 z, x, y, z;\n\tmov.b64 {%0, %1}, z;\n\t}"
-      : "+f"(y0), "+f"(y1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // Epilogue fragment of one thread (tcgen05.ld 16x256b, one load each for the
 // lanes 32q..32q+15 and 32q+16..32q+31 of its quarter q): rows 32q + t/4 + 8i
 // (i = 0..3) by columns c0 + 8j + e (j = 0..7, e = 0, 1), with

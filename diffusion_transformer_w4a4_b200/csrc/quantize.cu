@@ -79,18 +79,6 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
   return out;
 }
 
-// (a0, a1) * (b0, b1) with one packed instruction; each product is an ordinary
-// binary32 round-to-nearest multiply.
-__device__ __forceinline__ void mul2(float& a0, float& a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 x, y, z;\n\t"
-      "mov.b64 x, {%0, %1};\n\t"
-      "mov.b64 y, {%2, %3};\n\t"
-      "mul.rn.f32x2 z, x, y;\n\t"
-      "mov.b64 {%0, %1}, z;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(b0), "f"(b1));
-}
-
 __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));

@@ -251,10 +251,12 @@ svdq_status svdq_awq_prepare(const uint16_t* W, const uint16_t* bias, const uint
                              svdq_awq_canonical* out);
 
 /* Device layout ("awq blob"), each region 1024-byte aligned: inv_s f32 [K] |
- * bias f32 [N] | wscales fp16 [N, G'] with G' = K/64 rounded up to even (the
- * padding entry is zero) | wcodes u8 [N, K/2] (canonical packing,
- * kept at 4 bits per weight: the layer is a weight-streaming GEMV at the
- * batch sizes of modulation layers). */
+ * bias f32 [N] | wscales fp16 [N, G'] with G' = K/64 rounded up to a multiple of
+ * 8 (padding entries zero; a run of rows is then a whole number of 16-byte
+ * units) | wcodes u8 [N, K/2] (the canonical packing with every nibble in
+ * offset binary, n + 8 = n ^ 8, kept at 4 bits per weight: the layer is a
+ * weight-streaming GEMV at the batch sizes of modulation layers) | status int32 (zero in a packed blob; the kernel writes a nonzero
+ * code there when one of its bounded waits expires). */
 svdq_status svdq_awq_packed_size(int64_t N, int64_t K, size_t* bytes);
 svdq_status svdq_awq_pack(const svdq_awq_canonical* c, void* blob, size_t blob_bytes);
 
@@ -265,6 +267,11 @@ typedef struct svdq_awq_layer svdq_awq_layer; /* opaque host-side handle */
 svdq_status svdq_awq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K,
                                   svdq_awq_layer** out);
 void svdq_awq_layer_destroy(svdq_awq_layer* layer);
+
+/* Synchronous read of the blob's status word: 0, or SVDQ_ERR_TIMEOUT after a
+ * kernel gave up waiting for its weight copies (the outputs of that call are
+ * then incomplete).  The word is sticky until the blob is re-uploaded. */
+svdq_status svdq_awq_read_status(const svdq_awq_layer* layer, int* device_status);
 
 /* Y[M,N] = layer(X[M,K]), X and Y device pointers (16-byte aligned), `stream`
  * a cudaStream_t; asynchronous, returns launch errors only.  Token rows are

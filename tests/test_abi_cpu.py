@@ -285,12 +285,13 @@ def test_awq_pack_layout(lib, K):
         o = (o + nbytes + 1023) // 1024 * 1024
         return start
     G = K // 64
-    ld = (G + 1) // 2 * 2  # scale rows padded to an even count
-    o_is, o_b, o_ws, o_wc = take(K * 4), take(N * 4), take(N * ld * 2), take(N * K // 2)
+    ld = (G + 7) // 8 * 8  # scale rows padded to a multiple of 8 entries
+    o_is, o_b, o_ws, o_wc, o_st = take(K * 4), take(N * 4), take(N * ld * 2), take(N * K // 2), take(16)
     assert blob.size == o
+    assert np.all(blob[o_st:] == 0)
     assert np.array_equal(blob[o_is:o_is + 4 * K].view(np.float32), c["inv_s"])
     assert np.array_equal(blob[o_b:o_b + 4 * N].view(np.float32), oracle.bf16_to_f32(c["bias"]))
     ws = blob[o_ws:o_ws + N * ld * 2].view(np.uint16).reshape(N, ld)
     assert np.array_equal(ws[:, :G], c["wscales"])
     assert np.all(ws[:, G:] == 0)
-    assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"])
+    assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"] ^ 0x88)  # offset binary nibbles

@@ -40,6 +40,7 @@ def _run(layer):
     x = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).view(torch.bfloat16).to("cuda:0")
     y = lin.forward(x)
     torch.cuda.synchronize()
+    assert lin.status() == 0
     got = y.view(torch.int16).cpu().numpy().view(np.uint16)
     ref, yd = oracle.awq_forward(X, prep, want_f64=True)
     g, o = oracle.bf16_to_f32(got).astype(np.float64), oracle.bf16_to_f32(ref).astype(np.float64)
