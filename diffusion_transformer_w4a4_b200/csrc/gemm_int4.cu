@@ -106,8 +106,8 @@ __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 
 
 // y += (s_x[row] s_w[col]) acc over the fragment; sw points at s_w[c0], sx[i]
 // is s_x of row i.  Two packed operations per pair of outputs.
-__device__ __forceinline__ void drain_frag(float (&y)[64], const uint32_t (&lo)[32], const uint32_t (&hi)[32],
-                                           const float* sw, const float (&sx)[4]) {
+__device__ __forceinline__ void drain_frag(float2 (&y)[32], const uint32_t (&lo)[32], const uint32_t (&hi)[32],
+                                           const float* sw, const float2 (&sx)[4]) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float2 w = *(const float2*)(sw + 8 * j);  // 4 distinct addresses per warp
@@ -115,9 +115,8 @@ __device__ __forceinline__ void drain_frag(float (&y)[64], const uint32_t (&lo)[
     for (int i = 0; i < 4; ++i) {
       const uint32_t(&r)[32] = i < 2 ? lo : hi;
       const int k = 4 * j + 2 * (i & 1);
-      float c0 = w.x, c1 = w.y;
-      mul2(c0, c1, sx[i], sx[i]);  // exact: a product of two fp16 values
-      fma2(y[16 * i + 2 * j], y[16 * i + 2 * j + 1], c0, c1, __uint_as_float(r[k]), __uint_as_float(r[k + 1]));
+      const float2 c = __fmul2_rn(w, sx[i]);  // exact: products of two fp16 values
+      y[8 * i + j] = __ffma2_rn(c, make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), y[8 * i + j]);
     }
   }
 }
@@ -319,9 +318,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
       const int m0 = mt * BM + rq;
       const int n0 = nt * BN + cq;
-      float y[64];
+      float2 y[32];  // y[8i + j] = columns 8j, 8j + 1 of row 8i (of this thread's fragment)
 #pragma unroll
-      for (int j = 0; j < 64; ++j) y[j] = 0.f;
+      for (int j = 0; j < 32; ++j) y[j] = make_float2(0.f, 0.f);
       if (p.n_lr > 0) {
         const int b = unit % NBUF;
         if (!mbar_wait(&acc_full[b], (unit / NBUF) & 1, wc)) break;
@@ -334,10 +333,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-              y[16 * i + 2 * j + e] = __uint_as_float((i < 2 ? lo : hi)[4 * j + 2 * (i & 1) + e]);
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t(&r)[32] = i < 2 ? lo : hi;
+            y[8 * i + j] = make_float2(__uint_as_float(r[4 * j + 2 * (i & 1)]), __uint_as_float(r[4 * j + 2 * (i & 1) + 1]));
+          }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[b]);
@@ -371,8 +370,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
             export_frag(p, (size_t)(ks * GPS + g), m0, n0, lo, hi);
           } else {
             const __half* sxs = (const __half*)(sc + SC_SW) + g * BM + rq;
-            const float sx[4] = {__half2float(sxs[0]), __half2float(sxs[8]), __half2float(sxs[16]),
-                                 __half2float(sxs[24])};
+            float2 sx[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sx[i].x = sx[i].y = __half2float(sxs[8 * i]);
             drain_frag(y, lo, hi, (const float*)sc + g * BN + cq, sx);
           }
         }
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
           for (int i = 0; i < 4; ++i) {
             const int m = m0 + 8 * i;
             if (m < p.M) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(y[16 * i + 2 * j] + bb.x, y[16 * i + 2 * j + 1] + bb.y);
+              __nv_bfloat162 h = __floats2bfloat162_rn(y[8 * i + j].x + bb.x, y[8 * i + j].y + bb.y);
               *(__nv_bfloat162*)(p.Y + (size_t)m * p.N + n) = h;
             }
           }
