@@ -269,15 +269,27 @@ def lowrank_down(xhat: np.ndarray, L1: np.ndarray) -> np.ndarray:
     return t
 
 
+def act_tensor_scale(xhat: np.ndarray) -> float:
+    """Dynamic per-tensor NVFP4 activation scale: pow2_scale of the largest |x^|
+    of the tensor being quantized (a first pass over the whole activation, then
+    the block quantizer with that scale).  The static scale of prepare is the
+    same formula applied to the calibration statistic instead."""
+    return pow2_scale(float(np.abs(np.asarray(xhat, np.float32)).max()) if np.size(xhat) else 0.0)
+
+
 def quantize_act(X_bf16: np.ndarray, prep: dict):
     """Activation side of the layer: smoothing, 4-bit group quantization and the
-    low-rank down-projection t = bf16(bf16(x^) L1).  Returns dict(xhat, codes, scales, t)."""
+    low-rank down-projection t = bf16(bf16(x^) L1).  Returns dict(xhat, codes,
+    scales, t, g_x); g_x is the activation per-tensor scale used (NVFP4: the
+    prepared static one, or, when prep["g_x"] is 0, the dynamic one of this X)."""
     xhat = smooth_act(X_bf16, prep["inv_lambda"])
     if prep["fmt"] == INT4:
+        g = 1.0
         codes, scales = quant_int4(xhat)
     else:
-        codes, scales = quant_nvfp4(xhat, prep["g_x"])
-    return dict(xhat=xhat, codes=codes, scales=scales, t=lowrank_down(xhat, prep["L1"]))
+        g = prep["g_x"] if prep["g_x"] != 0 else act_tensor_scale(xhat)
+        codes, scales = quant_nvfp4(xhat, g)
+    return dict(xhat=xhat, codes=codes, scales=scales, t=lowrank_down(xhat, prep["L1"]), g_x=g)
 
 
 def forward_from_act(act: dict, prep: dict, want_f64: bool = False):
@@ -293,7 +305,7 @@ def forward_from_act(act: dict, prep: dict, want_f64: bool = False):
     lib().orc_forward_out(M, N, K, r, prep["fmt"], _p(codes), _p(np.ascontiguousarray(act["scales"], sc_dtype)),
                           _p(np.ascontiguousarray(prep["wcodes"], np.uint8)),
                           _p(np.ascontiguousarray(prep["wscales"], sc_dtype)),
-                          float(prep["g_x"]), float(prep["g_w"]), _p(t), _p(L2), _p(prep["bias"]),
+                          float(act.get("g_x", prep["g_x"])), float(prep["g_w"]), _p(t), _p(L2), _p(prep["bias"]),
                           _p(yd) if want_f64 else None, _p(y))
     return (y, yd) if want_f64 else y
 

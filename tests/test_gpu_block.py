@@ -59,7 +59,7 @@ def _check_layer(gl, X, prep, rows):
     np.testing.assert_array_equal(got["codes"], ref["codes"])
     np.testing.assert_array_equal(got["scales"], ref["scales"])
     st = assert_t_close(got["t"], ref["t"], ref, prep)
-    sub = {k: v[rows] for k, v in ref.items()}
+    sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
     sy = assert_y_close(y[rows], oracle.forward_from_act(sub, prep), sub, prep)
     return y, dict(sy, **st)
 
