@@ -64,7 +64,9 @@ extern "C" svdq_status svdq_forward_noalloc(const svdq_layer* L, const void* X, 
   // the control block (status word, split-K counters) must start at zero; the
   // rest is fully rewritten by the kernels
   if (cudaMemsetAsync(ws + w.status, 0, w.ctrl_bytes, s) != cudaSuccess) return SVDQ_ERR_CUDA;
-  int st = launch_quantize(L, X, M, ws, w, s);
+  int st = L->dyn_gx ? launch_act_amax(L, X, M, ws, w, s) : SVDQ_OK;
+  if (st != SVDQ_OK) return (svdq_status)st;
+  st = launch_quantize(L, X, M, ws, w, s);
   if (st != SVDQ_OK) return (svdq_status)st;
   if (L->fmt == SVDQ_NVFP4_G16) return (svdq_status)launch_gemm_nvfp4(L, M, Y, ws, w, s);
   return (svdq_status)launch_gemm_int4(L, M, Y, ws, w, nullptr, s);

@@ -76,7 +76,9 @@ struct GParams {
   const uint8_t* sfb;
   const float* bias;
   uint16_t* Y;
-  float out_scale;
+  float out_scale;       // g_x g_w (static activation scale)
+  const float* gx_dev;   // dynamic activation scale: g_x left by the quantizer (else null)
+  float g_w;
   int* status;
   unsigned long long limit;
 };
@@ -296,6 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;  // exact: powers of two
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     uint8_t* stg = epi_stage + (warp - 2) * 2 * EPI_STAGE_BYTES;
     int local = 0, sbuf = 0;
@@ -335,8 +338,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = 8 * k + 2 * e;
-              const float y0 = fmaf(__uint_as_float(r[j]), p.out_scale, bb[j]);
-              const float y1 = fmaf(__uint_as_float(r[j + 1]), p.out_scale, bb[j + 1]);
+              const float y0 = fmaf(__uint_as_float(r[j]), out_scale, bb[j]);
+              const float y1 = fmaf(__uint_as_float(r[j + 1]), out_scale, bb[j + 1]);
               __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
               o[e] = *(uint32_t*)&hv;
             }
@@ -419,6 +422,8 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
   p.bias = L->bias;
   p.Y = (uint16_t*)Y;
   p.out_scale = L->g_x * L->g_w;
+  p.g_w = L->g_w;
+  p.gx_dev = L->dyn_gx ? (const float*)(ws + w.status + 4) : nullptr;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
   st = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 32,

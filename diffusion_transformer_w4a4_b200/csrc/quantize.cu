@@ -57,6 +57,11 @@ struct QParams {
   int64_t sld;  // INT4: row stride of the fp16 [K/64, sld] scales
   const float* inv_lambda;
   float g, inv_g, den;  // NVFP4 per-tensor scale, its exact inverse, 6*g
+  // dynamic per-tensor scale: the first pass's per-CTA maxima of |x^| (else null),
+  // and where this kernel leaves the resulting g_x for the GEMM
+  const float* amax_slots;
+  int nslots;
+  float* g_out;
   uint8_t* codes;
   uint8_t* scales;
   uint16_t* t;
@@ -110,6 +115,24 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 template <int RANK>
 __host__ __device__ constexpr uint32_t tmem_cols() {
   return RANK <= 32 ? 32u : (RANK <= 64 ? 64u : 128u);
+}
+
+// bf16 t times a power of two (1 for the static scale): exact in binary32, and
+// the product has the bf16 value's significand, so the rounding back is exact
+__device__ __forceinline__ __nv_bfloat162 scale_t(__nv_bfloat162 h, float s) {
+  return __floats2bfloat162_rn(__low2float(h) * s, __high2float(h) * s);
+}
+
+// The per-tensor NVFP4 scale for a tensor maximum: the smallest power of two g
+// with 6 * 448 * g >= amax (1 for an all-zero tensor); every comparison is exact.
+__device__ __forceinline__ float nvfp4_tensor_scale_dev(float amax) {
+  if (!(amax > 0.f)) return 1.f;
+  int e;
+  frexpf(amax, &e);
+  int k = e - 12;  // 2688 = 0.65625 * 2^12
+  while (ldexpf(2688.f, k) < amax) ++k;
+  while (ldexpf(2688.f, k - 1) >= amax) --k;
+  return ldexpf(1.f, k);
 }
 
 template <int FMT, int RANK>
@@ -171,6 +194,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+
+  // NVFP4 per-tensor scale: the prepared static one, or the dynamic one from the
+  // first pass's maxima (then t is stored as t / g_x, an exact power-of-two
+  // scaling, because the packed L2 carries only 1/g_w)
+  float gs = p.g, inv_gs = p.inv_g, dens = p.den, tsc = 1.f;
+  if (FMT == SVDQ_NVFP4_G16 && p.amax_slots != nullptr) {
+    __shared__ float dred[kThreads / 32];
+    float m = 0.f;
+    for (int i = threadIdx.x; i < p.nslots; i += kThreads) m = fmaxf(m, p.amax_slots[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) dred[warp] = m;
+    __syncthreads();
+    m = dred[0];
+#pragma unroll
+    for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, dred[i]);
+    gs = nvfp4_tensor_scale_dev(m);
+    inv_gs = 1.0f / gs;  // exact: a power of two
+    dens = 6.0f * gs;
+    tsc = inv_gs;
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = gs;
+  }
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ X producer
@@ -283,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
           uint2 packed = make_uint2(0u, 0u);
           if (FMT == SVDQ_NVFP4_G16) {
-            const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, p.den));
+            const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, dens));
             if (sb != 0) {
               // 1 / (e4m3(sb) * g) exactly: g is a power of two
-              const float inv = rtab[sb] * p.inv_g;
+              const float inv = rtab[sb] * inv_gs;
               float q0[8], q1[8];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -379,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m < p.M) {
 #pragma unroll
               for (int j = 0; j < RANK; j += 2) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+                __nv_bfloat162 h = scale_t(__floats2bfloat162_rn(acc[j], acc[j + 1]), tsc);
                 *(uint32_t*)(p.t + (size_t)m * RANK + j) = *(uint32_t*)&h;
               }
             }
@@ -407,8 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sum.z += v.z;
                     sum.w += v.w;
                   }
-                  __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
-                  __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                  __nv_bfloat162 h0 = scale_t(__floats2bfloat162_rn(sum.x, sum.y), tsc);
+                  __nv_bfloat162 h1 = scale_t(__floats2bfloat162_rn(sum.z, sum.w), tsc);
                   *(uint2*)(p.t + (size_t)m * RANK + j) = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
                 }
               }
@@ -484,6 +529,14 @@ int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, 
   p.g = L->g_x;
   p.inv_g = 1.0f / L->g_x;  // exact: g_x is a power of two
   p.den = 6.0f * L->g_x;
+  if (L->dyn_gx) {  // the first pass (k_act_amax) ran just before on this stream
+    int gx = 0, gy = 0;
+    act_amax_grid(M, L->K, &gx, &gy);
+    p.amax_slots = (const float*)(ws + w.amax);
+    p.nslots = gx * gy;
+    p.g_out = (float*)(ws + w.status + 4);
+    p.g = p.inv_g = p.den = 0.f;  // set in the kernel
+  }
   p.codes = ws + w.codes;
   p.scales = ws + w.scales;
   p.t = (uint16_t*)(ws + w.t);

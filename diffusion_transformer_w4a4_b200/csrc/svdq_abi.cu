@@ -81,9 +81,11 @@ Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M) {
   w.t = o;
   w.t_bytes = (size_t)M * rank * 2;
   o = align_up(o + w.t_bytes, kAlign);
-  // control block: status word, then one arrival counter per 128-row block
+  // control block: status word and per-call g_x, one arrival counter per
+  // 128-row block, then the slots of the dynamic activation-scale pass
   w.status = o;
-  w.ctrl_bytes = 16 + 4 * (size_t)((M + kQRows - 1) / kQRows);
+  w.amax = o + align_up(16 + 4 * (size_t)((M + kQRows - 1) / kQRows), 16);
+  w.ctrl_bytes = (w.amax - o) + 4 * (size_t)kAmaxSlots;
   o = align_up(o + w.ctrl_bytes, kAlign);
   // fp32 partial low-rank sums of the quantizer's K slices
   w.nslices = quant_slices(M, K);
@@ -196,10 +198,11 @@ svdq_status svdq_pack(const svdq_canonical* c, void* blob_v, size_t blob_bytes) 
   for (int64_t k = 0; k < K; ++k)
     for (int j = 0; j < r; ++j) L1t[(int64_t)j * K + k] = c->L1[k * r + j];
   // NVFP4: L2 / (g_x g_w), a power of two, so the low-rank product accumulates in
-  // the units of the 4-bit block-scaled product.
+  // the units of the 4-bit block-scaled product.  With the dynamic activation
+  // scale (g_x = 0) only 1/g_w is folded here; the quantizer stores t / g_x.
   float l2_scale = 1.0f;
   if (fmt == SVDQ_NVFP4_G16) {
-    const float gg = c->g_x * c->g_w;
+    const float gg = (c->g_x == 0.f ? 1.0f : c->g_x) * c->g_w;
     int e;
     if (!(gg > 0.f) || std::frexp(gg, &e) != 0.5f) return SVDQ_ERR_INVALID_ARG;  // must be a power of two
     l2_scale = 1.0f / gg;
@@ -263,9 +266,10 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   if (!dev_blob || !shape_ok(N, K, rank, fmt) || ((uintptr_t)dev_blob & 255)) return SVDQ_ERR_INVALID_ARG;
   const Blob b = blob_layout(N, K, rank, fmt);
   if (blob_bytes < b.total) return SVDQ_ERR_INVALID_ARG;
-  if (fmt == SVDQ_NVFP4_G16) {
+  if (fmt == SVDQ_NVFP4_G16) {  // g_x == 0 selects the dynamic activation scale
     int e;
-    if (!(g_x > 0.f) || !(g_w > 0.f) || std::frexp(g_x * g_w, &e) != 0.5f) return SVDQ_ERR_INVALID_ARG;
+    if (!(g_x >= 0.f) || !(g_w > 0.f) || std::frexp((g_x == 0.f ? 1.0f : g_x) * g_w, &e) != 0.5f)
+      return SVDQ_ERR_INVALID_ARG;
   }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -282,6 +286,7 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   L->fmt = fmt;
   L->g_x = fmt == SVDQ_NVFP4_G16 ? g_x : 1.0f;
   L->g_w = fmt == SVDQ_NVFP4_G16 ? g_w : 1.0f;
+  L->dyn_gx = fmt == SVDQ_NVFP4_G16 && g_x == 0.f;
   L->device = dev;
   L->blob = (const uint8_t*)dev_blob;
   L->off = b;
@@ -364,6 +369,10 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!X || ((uintptr_t)X & 15)) return SVDQ_ERR_INVALID_ARG;
+  if (L->dyn_gx) {  // first pass: the tensor's largest |x^|
+    const int e = launch_act_amax(L, X, M, (uint8_t*)ws, w, (cudaStream_t)stream);
+    if (e != SVDQ_OK) return (svdq_status)e;
+  }
   return (svdq_status)launch_quantize(L, X, M, (uint8_t*)ws, w, (cudaStream_t)stream);
 }
 

@@ -24,6 +24,7 @@ constexpr int kQRows = 128;   // activation quantizer: token rows per CTA (= tcg
 constexpr int kQChunk = 128;  // activation quantizer: K columns per pipeline chunk
 constexpr int kQSmCount = 148;  // SM count the quantizer's K-split is sized for (fixed, so sizes are device-free)
 constexpr size_t kAlign = 1024;
+constexpr int kAmaxSlots = 1024;  // per-CTA maxima of the dynamic activation-scale pass
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -64,7 +65,10 @@ inline int quant_slices(int64_t M, int64_t K) {
 }
 
 struct Workspace {
-  size_t codes, scales, t, status, tpart, total;
+  // status: control block = [0] status word, [4] the per-call activation scale
+  // g_x (dynamic layers), [16, ...) split-K counters, then at `amax` the
+  // kAmaxSlots per-CTA maxima of the dynamic-scale pass
+  size_t codes, scales, t, status, amax, tpart, total;
   size_t codes_bytes, scales_bytes, t_bytes, ctrl_bytes, tpart_bytes;
   int nslices;
 };
@@ -83,7 +87,8 @@ LowRankChunks lowrank_chunks(int rank);
 struct svdq_layer {
   int64_t N, K;
   int rank, fmt;
-  float g_x, g_w;
+  float g_x, g_w;  // g_x == 0: NVFP4 activation scale computed per call (dynamic)
+  bool dyn_gx;
   int device;
   const uint8_t* blob;
   svdq::Blob off;
@@ -117,6 +122,11 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
 unsigned long long wait_limit_cycles();
 
 // Kernel launchers (return svdq_status).
+// dynamic activation scale: grid of the amax pass (its CTA count is the number
+// of valid slots) and its launch
+void act_amax_grid(int64_t M, int64_t K, int* gx, int* gy);
+int launch_act_amax(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
+                    cudaStream_t stream);
 int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
                     cudaStream_t stream);
 int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w,

@@ -77,7 +77,8 @@ typedef struct svdq_canonical {
   int32_t rank;      /* low-rank branch width r */
   int32_t fmt;       /* svdq_format */
   float alpha;       /* smoothing migration strength used */
-  float g_x;         /* NVFP4 activation per-tensor scale (1 for INT4) */
+  float g_x;         /* NVFP4 activation per-tensor scale (1 for INT4); 0 selects the
+                        dynamic scale: computed per call from the input's largest |x^| */
   float g_w;         /* NVFP4 weight per-tensor scale (1 for INT4) */
   float reserved;
   float* lambda;     /* [K]  smoothing factors, binary32 */
@@ -141,7 +142,14 @@ typedef struct svdq_layer svdq_layer; /* opaque host-side handle */
 
 /* Bind a device-resident packed blob (from svdq_pack) to a host handle.  No
  * device memory is allocated; the blob must outlive the handle.  Fails with
- * UNSUPPORTED_DEVICE on a device other than CC 10.0 (current device). */
+ * UNSUPPORTED_DEVICE on a device other than CC 10.0 (current device).
+ * NVFP4: g_w and g_x must be powers of two, or g_x = 0 for the dynamic
+ * activation scale (the blob must then have been packed with g_x = 0 too: its
+ * L2 carries 1/g_w only).  A dynamic layer's svdq_quantize_act runs a first pass
+ * over X for its largest |x^| = |fl32(x * inv_lambda)| (per-CTA maxima in the
+ * workspace), takes g_x = the smallest power of two >= that / (6 * 448) (1 for
+ * an all-zero X), quantizes with it, stores t / g_x (exact) as the workspace's
+ * t, and leaves g_x in word 1 of the control block for svdq_gemm. */
 svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K, int rank, int fmt,
                               float g_x, float g_w, svdq_layer** out);
 void svdq_layer_destroy(svdq_layer* layer);
@@ -151,9 +159,11 @@ void svdq_layer_destroy(svdq_layer* layer);
  * FP8 E4M3 byte per code holding its integer value, u8 [M, K]); [1] act scales
  * (NVFP4: E4M3 in the tensor-core scale-factor layout of 128-row tiles; INT4:
  * fp16 [K/64, M'], M' = M rounded up to a multiple of 128, columns >= M unused);
- * [2] t bf16 [M, rank]; [3] status word int32 (first word of a small control
- * block that also holds the quantizer's split-K counters).  The total size also
- * covers the quantizer's fp32 partial sums of t. */
+ * [2] t bf16 [M, rank] (t / g_x for a dynamic-scale layer); [3] status word
+ * int32, the first word of a control block that also holds the per-call g_x of a
+ * dynamic-scale layer (word 1, float), the quantizer's split-K counters and the
+ * first pass's per-CTA maxima.  The total size also covers the quantizer's fp32
+ * partial sums of t. */
 svdq_status svdq_workspace_size(const svdq_layer* layer, int64_t M, size_t* bytes);
 svdq_status svdq_workspace_layout(const svdq_layer* layer, int64_t M, size_t offsets[4], size_t sizes[4]);
 

@@ -166,7 +166,13 @@ class GpuLayer:
         else:
             scales = ws[off[1]:off[1] + sz[1]].view(np.uint16).reshape(K // 64, -1)[:, :M].T.copy()
         t = ws[off[2]:off[2] + sz[2]].view(np.uint16).reshape(M, r) if r else np.zeros((M, 0), np.uint16)
-        return dict(codes=codes.copy(), scales=scales, t=t.copy())
+        g_x = self.prep["g_x"]
+        if self.prep["fmt"] == oracle.NVFP4 and g_x == 0:
+            # dynamic activation scale: the quantizer leaves g_x in the control block
+            # (word 1) and stores t / g_x; undo the exact power-of-two scaling
+            g_x = float(ws[off[3] + 4:off[3] + 8].view(np.float32)[0])
+            t = oracle.f32_to_bf16(oracle.bf16_to_f32(t) * np.float32(g_x))
+        return dict(codes=codes.copy(), scales=scales, t=t.copy(), g_x=g_x)
 
     def forward(self, X):
         torch = self.torch

@@ -214,6 +214,33 @@ def test_pack_layout(lib, fmt):
         assert np.all(blob[o_ws:][~used] == 0)
 
 
+def test_pack_dynamic_activation_scale_folds_only_the_weight_scale(lib):
+    """g_x = 0 selects the per-call activation scale: the packed L2 carries
+    1/g_w only (the quantizer stores t / g_x), everything else is unchanged."""
+    N, K, r = 208, 256, 16
+    rng = np.random.default_rng(4)
+    c = svdq._canonical_arrays(N, K, r, "nvfp4")
+    c["inv_lambda"][:] = rng.uniform(0.5, 2, K)
+    c["L1"][:] = oracle.f32_to_bf16(rng.standard_normal((K, r)).astype(np.float32))
+    c["L2"][:] = oracle.f32_to_bf16(rng.standard_normal((r, N)).astype(np.float32))
+    c["wcodes"][:] = rng.integers(0, 256, c["wcodes"].shape)
+    c["wscales"][:] = rng.integers(0, 0x7E, c["wscales"].shape)
+    c["g_x"], c["g_w"] = 0.0, 2.0**-11
+    dyn = svdq.svdq_pack(c)
+    c["g_x"] = 1.0
+    st = svdq.svdq_pack(c)
+    assert np.array_equal(dyn, st)  # with g_x = 1 the static fold is the same 1/g_w
+    c["g_x"] = 2.0**-3
+    st3 = svdq.svdq_pack(c)
+    l2_off = (K * 4 + 1023) // 1024 * 1024 + (r * K * 2 + 1023) // 1024 * 1024
+    l2d = oracle.bf16_to_f32(dyn[l2_off:l2_off + 2 * N * r].view(np.uint16))
+    l23 = oracle.bf16_to_f32(st3[l2_off:l2_off + 2 * N * r].view(np.uint16))
+    assert np.array_equal(l23, l2d * np.float32(8.0))
+    c["g_x"] = -1.0
+    with pytest.raises(svdq.SvdqError):
+        svdq.svdq_pack(c)
+
+
 def test_pack_rejects_non_power_of_two_scales(lib):
     c = svdq._canonical_arrays(32, 256, 16, "nvfp4")
     c["g_x"], c["g_w"] = 0.3, 1.0

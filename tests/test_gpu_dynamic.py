@@ -1,0 +1,89 @@
+"""GPU parity of the dynamic per-tensor NVFP4 activation scale (layers prepared
+with g_x = 0: a first pass takes the tensor's largest |x^|, the quantizer derives
+g_x from it, stores t / g_x, and the GEMM scales by g_x g_w).
+
+The inputs are the calibration inputs times a factor that is not a power of
+two, so the per-call scale differs from the one calibration would give.  Bar:
+g_x, activation codes and scales bit-exact; t within its bound; bf16 Y within
+rel-L2 1e-3 and the elementwise bound of svdq_cases (sampled rows at the
+FLUX-sized shape)."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+from svdq_cases import GpuLayer, assert_t_close, assert_y_close, oracle_layer
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+    from diffusion_transformer_w4a4_b200 import build
+
+    build.build()
+    assert torch.cuda.is_available()
+    assert svdq.svdq_device_check(0) == svdq.SVDQ_OK, "needs an sm_100a device"
+    torch.cuda.set_device(0)
+
+
+def _dynamic_case(layer, factor):
+    X, W, b, prep = oracle_layer(layer)
+    dyn = dict(prep)
+    dyn["g_x"] = 0.0
+    Xs = wl.f32_to_bf16_bits(oracle.bf16_to_f32(X) * np.float32(factor))
+    return Xs, dyn
+
+
+@pytest.mark.parametrize("M,K,N,rank,factor", [(1, 256, 192, 16, 3.0), (37, 512, 400, 32, 0.3),
+                                               (300, 768, 576, 48, 7.5), (128, 1024, 384, 0, 1.7),
+                                               (257, 256, 208, 64, 40.0), (513, 2048, 1152, 128, 0.05)])
+def test_dynamic_scale_parity(M, K, N, rank, factor):
+    layer = wl.small_layer(M, K, N, rank, "nvfp4", layer_id=3 * M + K)
+    X, dyn = _dynamic_case(layer, factor)
+    gl = GpuLayer(dyn)
+    y = gl.forward(X)
+    assert gl.status(M) == 0
+    got = gl.read_act(M)
+    ref = oracle.quantize_act(X, dyn)
+    assert got["g_x"] == ref["g_x"]
+    np.testing.assert_array_equal(got["codes"], ref["codes"])
+    np.testing.assert_array_equal(got["scales"], ref["scales"])
+    if rank:
+        assert_t_close(got["t"], ref["t"], ref, dyn)
+    assert_y_close(y, oracle.forward_from_act(ref, dyn), ref, dyn)
+
+
+def test_dynamic_scale_flux_shape_sampled_rows():
+    layer = wl.WORKLOADS["c2_nvfp4_1024x3072x3072_r32"][0]
+    X, dyn = _dynamic_case(layer, 6.0)
+    gl = GpuLayer(dyn)
+    M = layer.M
+    y = gl.forward(X)
+    assert gl.status(M) == 0
+    got = gl.read_act(M)
+    ref = oracle.quantize_act(X, dyn)
+    assert got["g_x"] == ref["g_x"]
+    np.testing.assert_array_equal(got["codes"], ref["codes"])
+    np.testing.assert_array_equal(got["scales"], ref["scales"])
+    assert_t_close(got["t"], ref["t"], ref, dyn)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], np.random.default_rng(3).choice(M, 40, replace=False)]))
+    sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
+    assert_y_close(y[rows], oracle.forward_from_act(sub, dyn), sub, dyn)
+
+
+def test_dynamic_scale_follows_the_input_from_call_to_call():
+    """One layer, two calls on inputs 2^5 apart: the second call's g_x is 2^5
+    times the first one's and its codes and scales are the same."""
+    layer = wl.small_layer(200, 512, 256, 32, "nvfp4", layer_id=99)
+    X, dyn = _dynamic_case(layer, 1.0)
+    gl = GpuLayer(dyn)
+    a = gl.quantize(X)
+    b = gl.quantize(wl.f32_to_bf16_bits(oracle.bf16_to_f32(X) * np.float32(32.0)))
+    assert gl.status(200) == 0
+    assert b["g_x"] == 32.0 * a["g_x"]
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    np.testing.assert_array_equal(a["scales"], b["scales"])
