@@ -285,6 +285,49 @@ def awq_measure(dev, hbm_peak):
             "gpu_launches": reps * AWQ_SET}
 
 
+def dynamic_measure(dev, canons, xs, steps=20):
+    """The same two layers with the dynamic per-tensor activation scale (g_x = 0):
+    per step, for each layer, the amax pass + quantizer and the GEMM, L2 flushed
+    between steps like the main measurement.  The amax pass is HBM-bound (one read
+    of X); its cost is the difference of the quantize times."""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    lins = []
+    for c in canons:
+        d = dict(c)
+        d["g_x"] = 0.0
+        lins.append(svdq.SvdqLinear(d, device=dev))
+    xd = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in xs]
+    ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in LAYERS]
+    wss = [lin.workspace(l.M) for lin, l in zip(lins, LAYERS)]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps + 3)]
+    for k in range(steps + 3):
+        flush.zero_()
+        for i, (lin, l) in enumerate(zip(lins, LAYERS)):
+            evs[k][2 * i].record(stream)
+            svdq.svdq_quantize_act(lin.handle, xd[i], l.M, wss[i], sp)
+            evs[k][2 * i + 1].record(stream)
+            svdq.svdq_gemm(lin.handle, l.M, ys[i], wss[i], sp)
+        evs[k][4].record(stream)
+    torch.cuda.synchronize()
+    for lin, l in zip(lins, LAYERS):
+        assert lin.status(l.M) == 0, "kernel reported an error (dynamic scale)"
+    ev = evs[3:]
+    step = statistics.median([e[0].elapsed_time(e[4]) for e in ev]) * 1e3
+    q = statistics.median([e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev]) * 1e3
+    amax_bytes = sum(2 * l.M * l.K + 4 * l.K for l in LAYERS)
+    del lins
+    return {"step_us": step, "quantize_with_amax_pass_us": q, "amax_pass_bytes_per_step": amax_bytes,
+            "kernels": ["k_act_amax", "k_quantize", "k_gemm_nvfp4"],
+            "note": "layers prepared like the main line, then g_x = 0 (per-call scale); "
+                    "compare quantize_with_amax_pass_us with per_layer_us.quantize_both"}
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -402,6 +445,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clk.summary(),
     }
     out["awq_w4a16"] = awq_measure(dev, hbm)
+    out["dynamic_act_scale"] = dynamic_measure(dev, canons, xs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(canons, xs)
     if rank == 0:
