@@ -397,3 +397,59 @@ def awq_prepare(W_bf16: np.ndarray, bias_bf16, X_calib_bf16: np.ndarray, alphas=
     codes, scales = awq_quant_weights(W, s_f)
     return dict(N=N, K=K, alpha=float(a), err=best[1], s=s_f, inv_s=inv, wcodes=codes, wscales=scales,
                 bias=(np.zeros(N, np.uint16) if bias_bf16 is None else np.ascontiguousarray(bias_bf16, np.uint16)))
+
+
+# ----------------------------------------------------------------------------- int8 tensorwise W8A8
+# The INT8 tensorwise W8A8 layer the Krea page ("SVDQuant ускоряет Krea 2 вдвое ...",
+# section "Решение: INT8 и W4A4") compares with W4A4: symmetric 8-bit codes with one
+# scale per tensor, for the weight (fixed at preparation) and for the activation
+# (taken from the tensor being quantized at every call: a first pass for its
+# largest |x|, then the quantizer).  No smoothing and no low-rank branch.
+W8_QMAX = 127
+
+
+def w8_tensor_scale(v: np.ndarray) -> np.float32:
+    """s = fl32(max|v| / 127) (0 for an all-zero tensor)."""
+    v = np.asarray(v, np.float32)
+    amax = np.float32(np.abs(v).max()) if v.size else np.float32(0.0)
+    return np.float32(amax / np.float32(W8_QMAX))
+
+
+def quant_w8(v: np.ndarray, s: np.float32) -> np.ndarray:
+    """Codes clamp(rne(v * fl32(1/s)), -127, 127) as int8, the product in binary32
+    (all zero when s is 0)."""
+    v = np.asarray(v, np.float32)
+    if s == 0:
+        return np.zeros(v.shape, np.int8)
+    inv = np.float32(np.float32(1.0) / np.float32(s))
+    q = np.rint((v * inv).astype(np.float32))
+    return np.clip(q, -W8_QMAX, W8_QMAX).astype(np.int8)
+
+
+def w8a8_prepare(W_bf16: np.ndarray, bias_bf16=None) -> dict:
+    W = np.ascontiguousarray(W_bf16, np.uint16)
+    N, K = W.shape
+    w = bf16_to_f32(W)
+    s_w = w8_tensor_scale(w)
+    return dict(N=N, K=K, s_w=s_w, wcodes=quant_w8(w, s_w),
+                bias=(np.zeros(N, np.uint16) if bias_bf16 is None else np.ascontiguousarray(bias_bf16, np.uint16)))
+
+
+def w8a8_quantize_act(X_bf16: np.ndarray) -> dict:
+    x = bf16_to_f32(np.ascontiguousarray(X_bf16, np.uint16))
+    s_x = w8_tensor_scale(x)
+    return dict(codes=quant_w8(x, s_x), s_x=s_x)
+
+
+def w8a8_forward_from_act(act: dict, prep: dict, want_f64: bool = False):
+    """y = bf16(s_x s_w (qx . qw^T) + b): the integer product exactly (int64), the
+    rest in binary64."""
+    acc = act["codes"].astype(np.int64) @ prep["wcodes"].astype(np.int64).T
+    yd = float(act["s_x"]) * float(prep["s_w"]) * acc.astype(np.float64) + \
+        bf16_to_f32(prep["bias"]).astype(np.float64)[None, :]
+    y = f64_to_bf16(np.ascontiguousarray(yd))
+    return (y, yd) if want_f64 else y
+
+
+def w8a8_forward(X_bf16: np.ndarray, prep: dict, want_f64: bool = False):
+    return w8a8_forward_from_act(w8a8_quantize_act(X_bf16), prep, want_f64)
