@@ -328,6 +328,53 @@ def dynamic_measure(dev, canons, xs, steps=20):
                     "compare quantize_with_amax_pass_us with per_layer_us.quantize_both"}
 
 
+def w8a8_measure(dev, xs, steps=20):
+    """INT8 tensorwise W8A8 layers at the same FLUX MLP shapes (weights from the
+    same seeded generator, prepared by the library): per step, for each layer,
+    the max|x| pass + quantizer and the int8 tensor-core GEMM, L2 flushed between
+    steps like the main measurement."""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    lins = []
+    for l in LAYERS:
+        _, W, b = wl.make_layer_inputs(l, 0)
+        codes, s_w = svdq.svdq_w8a8_prepare(W)
+        lins.append(svdq.W8A8Linear(codes, s_w, b, device=dev))
+    xd = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev) for x in xs]
+    ys = [torch.empty(l.M, l.N, dtype=torch.bfloat16, device=dev) for l in LAYERS]
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps + 3)]
+    for k in range(steps + 3):
+        flush.zero_()
+        for i, (lin, l) in enumerate(zip(lins, LAYERS)):
+            evs[k][2 * i].record(stream)
+            lin.quantize_act(xd[i], l.M)
+            evs[k][2 * i + 1].record(stream)
+            lin.gemm(l.M, ys[i])
+        evs[k][4].record(stream)
+    torch.cuda.synchronize()
+    for lin, l in zip(lins, LAYERS):
+        assert lin.status(l.M) == 0, "w8a8 kernel reported an error"
+    ev = evs[3:]
+    step = statistics.median([e[0].elapsed_time(e[4]) for e in ev]) * 1e3
+    q = statistics.median([e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev]) * 1e3
+    g = statistics.median([e[1].elapsed_time(e[2]) + e[3].elapsed_time(e[4]) for e in ev]) * 1e3
+    flops = sum(2.0 * l.M * l.N * l.K for l in LAYERS)
+    _, bf16, _, src = _peaks()
+    i8_peak = 2.0 * bf16  # measured bf16 dense x nominal int8:bf16 ratio (4.5 / 2.25)
+    gemm_tops = flops / (g * 1e-6) / 1e12
+    del lins
+    return {"metric": "W8A8 linear TOPS (2*M*N*K per layer)", "value": flops / (step * 1e-6) / 1e12, "unit": "TOPS",
+            "step_us": step, "quantize_us": q, "gemm_us": g,
+            "gemm_roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": i8_peak, "unit": "TOPS",
+                              "frac": gemm_tops / i8_peak, "kernel": "k_gemm_w8a8",
+                              "peak_source": f"{src} bf16 {bf16} TFLOP/s (burst) x 2 (nominal int8/bf16)"},
+            "gpu_launches": 6 * steps}
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -446,6 +493,7 @@ def run_ours(args, world, rank, local):
     }
     out["awq_w4a16"] = awq_measure(dev, hbm)
     out["dynamic_act_scale"] = dynamic_measure(dev, canons, xs)
+    out["w8a8"] = w8a8_measure(dev, xs)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(canons, xs)
     if rank == 0:

@@ -103,6 +103,23 @@ _EXPORTS = {
     "svdq_awq_read_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "svdq_awq_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                         ctypes.c_void_p]),
+    "svdq_w8a8_prepare": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.POINTER(ctypes.c_float)]),
+    "svdq_w8a8_packed_size": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)]),
+    "svdq_w8a8_pack": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_size_t]),
+    "svdq_w8a8_layer_create": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int64,
+                                              ctypes.c_float, ctypes.POINTER(ctypes.c_void_p)]),
+    "svdq_w8a8_layer_destroy": (None, [ctypes.c_void_p]),
+    "svdq_w8a8_workspace_size": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)]),
+    "svdq_w8a8_quantize_act": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                              ctypes.c_size_t, ctypes.c_void_p]),
+    "svdq_w8a8_gemm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                      ctypes.c_size_t, ctypes.c_void_p]),
+    "svdq_w8a8_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "svdq_w8a8_read_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t,
+                                             ctypes.POINTER(ctypes.c_int)]),
 }
 
 
@@ -437,4 +454,128 @@ class AwqLinear:
         h = getattr(self, "handle", None)
         if h is not None and _lib is not None:
             _lib.svdq_awq_layer_destroy(h)
+            self.handle = None
+
+
+# ----------------------------------------------------------------------------- int8 tensorwise W8A8
+def svdq_w8a8_prepare(W):
+    """Host: W [N,K] bf16 bits -> (int8 codes [N,K], s_w)."""
+    W = np.ascontiguousarray(W, np.uint16)
+    N, K = W.shape
+    codes = np.empty((N, K), np.int8)
+    s = ctypes.c_float()
+    _check(lib().svdq_w8a8_prepare(W.ctypes.data, N, K, codes.ctypes.data, ctypes.byref(s)), "svdq_w8a8_prepare")
+    return codes, float(s.value)
+
+
+def svdq_w8a8_packed_size(N: int, K: int) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().svdq_w8a8_packed_size(N, K, ctypes.byref(v)), "svdq_w8a8_packed_size")
+    return v.value
+
+
+def svdq_w8a8_pack(wcodes, bias=None) -> np.ndarray:
+    wcodes = np.ascontiguousarray(wcodes, np.int8)
+    N, K = wcodes.shape
+    size = svdq_w8a8_packed_size(N, K)
+    blob = np.zeros(size, np.uint8)
+    b = None if bias is None else np.ascontiguousarray(bias, np.uint16)
+    _check(lib().svdq_w8a8_pack(N, K, wcodes.ctypes.data, None if b is None else b.ctypes.data, blob.ctypes.data,
+                                size), "svdq_w8a8_pack")
+    return blob
+
+
+def svdq_w8a8_layer_create(dev_blob, blob_bytes: int, N: int, K: int, s_w: float):
+    h = ctypes.c_void_p()
+    _check(lib().svdq_w8a8_layer_create(_ptr(dev_blob), blob_bytes, N, K, s_w, ctypes.byref(h)),
+           "svdq_w8a8_layer_create")
+    return h
+
+
+def svdq_w8a8_layer_destroy(h) -> None:
+    lib().svdq_w8a8_layer_destroy(h)
+
+
+def svdq_w8a8_workspace_size(h, M: int) -> int:
+    v = ctypes.c_size_t()
+    _check(lib().svdq_w8a8_workspace_size(h, M, ctypes.byref(v)), "svdq_w8a8_workspace_size")
+    return v.value
+
+
+def svdq_w8a8_quantize_act(h, X, M: int, ws, stream=None) -> None:
+    _check(lib().svdq_w8a8_quantize_act(h, _ptr(X), M, _ptr(ws), ws.numel(), _stream(stream)),
+           "svdq_w8a8_quantize_act")
+
+
+def svdq_w8a8_gemm(h, M: int, Y, ws, stream=None) -> None:
+    _check(lib().svdq_w8a8_gemm(h, M, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)), "svdq_w8a8_gemm")
+
+
+def svdq_w8a8_forward(h, X, M: int, Y, ws, stream=None) -> None:
+    _check(lib().svdq_w8a8_forward(h, _ptr(X), M, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
+           "svdq_w8a8_forward")
+
+
+def svdq_w8a8_read_status(h, M: int, ws) -> int:
+    v = ctypes.c_int()
+    _check(lib().svdq_w8a8_read_status(h, M, _ptr(ws), ws.numel(), ctypes.byref(v)), "svdq_w8a8_read_status")
+    return v.value
+
+
+class W8A8Linear:
+    """One INT8 tensorwise W8A8 layer on the current CUDA device, from prepared
+    int8 weight codes [N,K], the weight scale s_w and an optional bf16 bias;
+    `forward(x)` maps bf16 [M, K] to bf16 [M, N]."""
+
+    def __init__(self, wcodes, s_w: float, bias=None, device=None):
+        import torch
+
+        self.N, self.K = int(wcodes.shape[0]), int(wcodes.shape[1])
+        self.s_w = float(s_w)
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.blob = torch.from_numpy(svdq_w8a8_pack(wcodes, bias)).to(self.device)
+        self.handle = svdq_w8a8_layer_create(self.blob, self.blob.numel(), self.N, self.K, self.s_w)
+        self._ws = {}
+
+    def workspace_size(self, M: int) -> int:
+        return svdq_w8a8_workspace_size(self.handle, M)
+
+    def workspace(self, M: int):
+        import torch
+
+        if M not in self._ws:
+            self._ws[M] = torch.empty(self.workspace_size(M), dtype=torch.uint8, device=self.device)
+        return self._ws[M]
+
+    def quantize_act(self, x, M: int, stream=None):
+        svdq_w8a8_quantize_act(self.handle, x, M, self.workspace(M), stream)
+
+    def gemm(self, M: int, y, stream=None):
+        svdq_w8a8_gemm(self.handle, M, y, self.workspace(M), stream)
+
+    def forward(self, x, out=None, stream=None):
+        import torch
+
+        assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
+        M = x.numel() // self.K
+        y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        svdq_w8a8_forward(self.handle, x, M, y, self.workspace(M), stream)
+        return y
+
+    __call__ = forward
+
+    def status(self, M: int) -> int:
+        return svdq_w8a8_read_status(self.handle, M, self.workspace(M))
+
+    def read_act(self, M: int):
+        """Activation codes int8 [M, K] and s_x from the workspace (after quantize_act)."""
+        ws = self.workspace(M).cpu().numpy()
+        ctrl = (M * self.K + 1023) // 1024 * 1024
+        return dict(codes=ws[:M * self.K].view(np.int8).reshape(M, self.K).copy(),
+                    s_x=np.float32(ws[ctrl + 4:ctrl + 8].view(np.float32)[0]))
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and _lib is not None:
+            _lib.svdq_w8a8_layer_destroy(h)
             self.handle = None

@@ -22,13 +22,18 @@ namespace {
 constexpr int kAmaxThreads = 256;
 constexpr int kUnroll = 4;
 
+// SMOOTH: |fl32(x * inv_lambda)|; else |x| (the INT8 tensorwise layer)
+template <bool SMOOTH>
 __global__ void __launch_bounds__(kAmaxThreads) k_act_amax(const uint4* __restrict__ x, const float4* __restrict__ il,
                                                          int M, int kv, float* __restrict__ slots) {
   const int c = blockIdx.y * kAmaxThreads + threadIdx.x;  // column vector
   float m = 0.f;
   if (c < kv) {
-    const float4 a = __ldg(il + 2 * c), b = __ldg(il + 2 * c + 1);
-    const float s[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    float s[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+    if constexpr (SMOOTH) {
+      const float4 a = __ldg(il + 2 * c), b = __ldg(il + 2 * c + 1);
+      s[0] = a.x, s[1] = a.y, s[2] = a.z, s[3] = a.w, s[4] = b.x, s[5] = b.y, s[6] = b.z, s[7] = b.w;
+    }
     auto fold = [&](const uint4 v) {
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -75,13 +80,22 @@ void act_amax_grid(int64_t M, int64_t K, int* gx, int* gy) {
   *gy = y;
 }
 
+int launch_act_amax_raw(const void* X, int64_t M, int64_t K, const float* inv_lambda, float* slots,
+                        cudaStream_t stream) {
+  int gx = 0, gy = 0;
+  act_amax_grid(M, K, &gx, &gy);
+  if (inv_lambda)
+    k_act_amax<true><<<dim3(gx, gy), kAmaxThreads, 0, stream>>>((const uint4*)X, (const float4*)inv_lambda, (int)M,
+                                                               (int)(K / 8), slots);
+  else
+    k_act_amax<false><<<dim3(gx, gy), kAmaxThreads, 0, stream>>>((const uint4*)X, nullptr, (int)M, (int)(K / 8),
+                                                                slots);
+  return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
 int launch_act_amax(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
                     cudaStream_t stream) {
-  int gx = 0, gy = 0;
-  act_amax_grid(M, L->K, &gx, &gy);
-  k_act_amax<<<dim3(gx, gy), kAmaxThreads, 0, stream>>>((const uint4*)X, (const float4*)L->inv_lambda, (int)M,
-                                                       (int)(L->K / 8), (float*)(ws + w.amax));
-  return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+  return launch_act_amax_raw(X, M, L->K, L->inv_lambda, (float*)(ws + w.amax), stream);
 }
 
 }  // namespace svdq

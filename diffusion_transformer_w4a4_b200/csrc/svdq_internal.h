@@ -127,6 +127,9 @@ unsigned long long wait_limit_cycles();
 void act_amax_grid(int64_t M, int64_t K, int* gx, int* gy);
 int launch_act_amax(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
                     cudaStream_t stream);
+// the same pass for any bf16 [M, K] tensor, with (inv_lambda) or without smoothing
+int launch_act_amax_raw(const void* X, int64_t M, int64_t K, const float* inv_lambda, float* slots,
+                        cudaStream_t stream);
 int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
                     cudaStream_t stream);
 int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w,

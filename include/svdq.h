@@ -290,6 +290,54 @@ svdq_status svdq_awq_read_status(const svdq_awq_layer* layer, int* device_status
  * it is correct for any M. */
 svdq_status svdq_awq_forward(const svdq_awq_layer* layer, const void* X, int64_t M, void* Y, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* INT8 tensorwise W8A8 layer: the 8-bit variant that "SVDQuant ускоряет      */
+/* Krea 2 вдвое ..." (section "Решение: INT8 и W4A4") compares with W4A4.     */
+/*   s = fl32(max|v| / 127) per tensor, q = clamp(rne(v * fl32(1/s)), +-127); */
+/*   the weight's s_w is fixed at preparation, the activation's s_x is taken   */
+/*   from each input (a first pass for max|x|);                              */
+/*   Y = bf16(s_x s_w (qx . qw^T) + b).  No smoothing, no low-rank branch.     */
+/* Shapes: N >= 8 and N % 8 == 0, K >= 128 and K % 128 == 0.                  */
+/* ------------------------------------------------------------------------ */
+typedef struct svdq_w8a8_layer svdq_w8a8_layer; /* opaque host-side handle */
+
+/* Host, synchronous.  W [N,K] bf16 -> wcodes int8 [N,K] (row-major) and *s_w.
+ * Errors: INVALID_ARG (shape, pointers), NUMERIC (non-finite W). */
+svdq_status svdq_w8a8_prepare(const uint16_t* W, int64_t N, int64_t K, int8_t* wcodes, float* s_w);
+
+/* Device layout ("w8a8 blob"), regions 1024-byte aligned: bias f32 [N] | wcodes
+ * int8 [N, K] row-major.  bias bf16 [N] or NULL (zeros). */
+svdq_status svdq_w8a8_packed_size(int64_t N, int64_t K, size_t* bytes);
+svdq_status svdq_w8a8_pack(int64_t N, int64_t K, const int8_t* wcodes, const uint16_t* bias, void* blob,
+                           size_t blob_bytes);
+
+/* Bind a device-resident w8a8 blob (256-byte aligned) to a handle with the
+ * weight scale s_w (finite, >= 0); allocates no device memory.
+ * UNSUPPORTED_DEVICE on a device other than CC 10.0. */
+svdq_status svdq_w8a8_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K, float s_w,
+                                   svdq_w8a8_layer** out);
+void svdq_w8a8_layer_destroy(svdq_w8a8_layer* layer);
+
+/* Workspace for M tokens (caller device memory, 256-byte aligned): activation
+ * codes int8 [M, K] at offset 0 | at the next 1024-byte boundary a control
+ * block: int32 status, float s_x of the last quantized input, 8 bytes unused,
+ * then the first pass's per-CTA maxima (1024 floats).  Needs no initialisation. */
+svdq_status svdq_w8a8_workspace_size(const svdq_w8a8_layer* layer, int64_t M, size_t* bytes);
+
+/* Asynchronous on `stream`; launch errors only.  X [M,K] bf16 and Y [M,N] bf16
+ * are device pointers (16-byte aligned).  quantize_act runs the max|x| pass and
+ * the quantizer; gemm the int8 tensor-core product with the scale and bias. */
+svdq_status svdq_w8a8_quantize_act(const svdq_w8a8_layer* layer, const void* X, int64_t M, void* ws,
+                                   size_t ws_bytes, void* stream);
+svdq_status svdq_w8a8_gemm(const svdq_w8a8_layer* layer, int64_t M, void* Y, void* ws, size_t ws_bytes,
+                           void* stream);
+svdq_status svdq_w8a8_forward(const svdq_w8a8_layer* layer, const void* X, int64_t M, void* Y, void* ws,
+                              size_t ws_bytes, void* stream);
+/* Synchronous read of the workspace status word (SVDQ_ERR_TIMEOUT after a wait
+ * ran past its limit). */
+svdq_status svdq_w8a8_read_status(const svdq_w8a8_layer* layer, int64_t M, const void* ws, size_t ws_bytes,
+                                  int* device_status);
+
 #ifdef __cplusplus
 }
 #endif

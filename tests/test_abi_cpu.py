@@ -322,3 +322,44 @@ def test_awq_pack_layout(lib, K):
     assert np.array_equal(ws[:, :G], c["wscales"])
     assert np.all(ws[:, G:] == 0)
     assert np.array_equal(blob[o_wc:o_wc + N * K // 2].reshape(N, K // 2), c["wcodes"] ^ 0x88)  # offset binary nibbles
+
+
+# ----------------------------------------------------------------------------- int8 tensorwise W8A8
+def test_w8a8_shape_validation(lib):
+    assert svdq.svdq_w8a8_packed_size(3072, 12288) > 0
+    for bad in [(12, 128), (0, 128), (16, 64), (16, 200)]:
+        with pytest.raises(svdq.SvdqError):
+            svdq.svdq_w8a8_packed_size(*bad)
+
+
+@pytest.mark.parametrize("shape", [(24, 128), (200, 384)])
+def test_w8a8_product_prepare_agrees_with_oracle(lib, shape):
+    N, K = shape
+    rng = np.random.default_rng(31)
+    w = rng.standard_normal((N, K)).astype(np.float32) * 0.02
+    w[3, 5] = 0.5  # a large entry sets the scale
+    W = wl.f32_to_bf16_bits(w)
+    codes, s_w = svdq.svdq_w8a8_prepare(W)
+    ref = oracle.w8a8_prepare(W)
+    assert np.float32(s_w) == ref["s_w"]
+    np.testing.assert_array_equal(codes, ref["wcodes"])
+
+
+def test_w8a8_prepare_rejects_non_finite(lib):
+    W = wl.f32_to_bf16_bits(np.ones((8, 128), np.float32))
+    W[2, 3] = 0x7F80  # +inf
+    with pytest.raises(svdq.SvdqError):
+        svdq.svdq_w8a8_prepare(W)
+
+
+def test_w8a8_pack_layout(lib):
+    N, K = 40, 256
+    rng = np.random.default_rng(32)
+    codes = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    b = oracle.f32_to_bf16(rng.standard_normal(N).astype(np.float32))
+    blob = svdq.svdq_w8a8_pack(codes, b)
+    o_wc = (N * 4 + 1023) // 1024 * 1024
+    assert blob.size == (o_wc + N * K + 1023) // 1024 * 1024
+    assert np.array_equal(blob[:4 * N].view(np.float32), oracle.bf16_to_f32(b))
+    assert np.array_equal(blob[o_wc:o_wc + N * K].view(np.int8).reshape(N, K), codes)
+    assert np.all(svdq.svdq_w8a8_pack(codes)[:4 * N] == 0)  # no bias: zeros
