@@ -145,7 +145,7 @@ const char* svdq_status_string(int status) {
   }
 }
 
-int svdq_abi_version(void) { return 1; }
+int svdq_abi_version(void) { return SVDQ_ABI_VERSION; }
 
 svdq_status svdq_canonical_sizes(int64_t N, int64_t K, int rank, int fmt, size_t sizes[7]) {
   if (!sizes || !shape_ok(N, K, rank, fmt)) return SVDQ_ERR_INVALID_ARG;

@@ -66,7 +66,11 @@ typedef enum svdq_format { SVDQ_INT4_G64 = 1, SVDQ_NVFP4_G16 = 2 } svdq_format;
 /* Human-readable name of a status code (static string, never NULL). */
 const char* svdq_status_string(int status);
 
-/* ABI version of this header (increments on incompatible change). */
+/* ABI version of this header (increments on incompatible change).
+ * 2: the svdq workspace control block holds the per-call g_x and the first
+ *    pass's maxima; the awq blob's scale rows are padded to 8 entries, its codes
+ *    are offset binary and it ends in a status word; the W8A8 layer. */
+#define SVDQ_ABI_VERSION 2
 int svdq_abi_version(void);
 
 /* ------------------------------------------------------------------------ */

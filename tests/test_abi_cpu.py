@@ -49,7 +49,7 @@ def test_status_strings(lib):
     assert svdq.svdq_status_string(0) == "SVDQ_OK"
     assert "sm_100a" in svdq.svdq_status_string(svdq.SVDQ_ERR_UNSUPPORTED_DEVICE)
     assert svdq.svdq_status_string(99).startswith("SVDQ_ERR")
-    assert svdq.svdq_abi_version() == 1
+    assert svdq.svdq_abi_version() == 2
 
 
 def test_shape_validation(lib):
