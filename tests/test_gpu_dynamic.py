@@ -57,8 +57,10 @@ def test_dynamic_scale_parity(M, K, N, rank, factor):
     assert_y_close(y, oracle.forward_from_act(ref, dyn), ref, dyn)
 
 
-def test_dynamic_scale_flux_shape_sampled_rows():
-    layer = wl.WORKLOADS["c2_nvfp4_1024x3072x3072_r32"][0]
+@pytest.mark.parametrize("name,idx", [("c2_nvfp4_1024x3072x3072_r32", 0), ("c4_mlp_4608x3072x12288_r32", 0),
+                                      ("c4_mlp_4608x3072x12288_r32", 1)], ids=["c2", "c4_up", "c4_down"])
+def test_dynamic_scale_flux_shape_sampled_rows(name, idx):
+    layer = wl.WORKLOADS[name][idx]
     X, dyn = _dynamic_case(layer, 6.0)
     gl = GpuLayer(dyn)
     M = layer.M
