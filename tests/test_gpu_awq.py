@@ -28,13 +28,15 @@ def _device():
     torch.cuda.set_device(0)
 
 
-def _run(layer):
+def _run(layer, x_scale=1.0):
     import torch
 
     import diffusion_transformer_w4a4_b200 as svdq
 
     X, W, b = wl.make_layer_inputs(layer)
     prep = oracle.awq_prepare(W, b, X)
+    if x_scale != 1.0:  # run on inputs far from the calibration ones
+        X = wl.f32_to_bf16_bits(oracle.bf16_to_f32(X) * np.float32(x_scale))
     lin = svdq.AwqLinear(dict(N=prep["N"], K=prep["K"], alpha=prep["alpha"], s=prep["s"], inv_s=prep["inv_s"],
                               wcodes=prep["wcodes"], wscales=prep["wscales"], bias=prep["bias"]), device="cuda:0")
     x = torch.from_numpy(np.ascontiguousarray(X).view(np.int16)).view(torch.bfloat16).to("cuda:0")
@@ -79,3 +81,10 @@ def test_awq_empty_and_arguments():
     with pytest.raises(svdq.SvdqError) as e:
         svdq.svdq_awq_forward(lin.handle, None, 2, y)
     assert e.value.status == svdq.SVDQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("x_scale", [2.0 ** 60, 2.0 ** -60])
+def test_awq_extreme_activation_magnitudes(x_scale):
+    """Activations 2^60 above or below the calibration ones (far beyond any real
+    layer, inside the kernel's |x^| < 2^113 domain for its pre-scaled decode)."""
+    print(x_scale, _run(wl.small_layer(2, 1024, 136, 0, wl.AWQ, layer_id=17), x_scale))

@@ -89,3 +89,17 @@ def test_dynamic_scale_follows_the_input_from_call_to_call():
     assert b["g_x"] == 32.0 * a["g_x"]
     np.testing.assert_array_equal(a["codes"], b["codes"])
     np.testing.assert_array_equal(a["scales"], b["scales"])
+
+
+def test_dynamic_scale_all_zero_input():
+    """max|x^| = 0: g_x = 1, every code and block scale 0, t = 0, and Y = bias."""
+    layer = wl.small_layer(130, 512, 256, 32, "nvfp4", layer_id=5)
+    X, dyn = _dynamic_case(layer, 1.0)
+    X = np.zeros_like(X)
+    gl = GpuLayer(dyn)
+    y = gl.forward(X)
+    assert gl.status(130) == 0
+    got = gl.read_act(130)
+    assert got["g_x"] == 1.0
+    assert not got["codes"].any() and not got["scales"].any() and not got["t"].any()
+    np.testing.assert_array_equal(y, oracle.forward(X, dyn))
