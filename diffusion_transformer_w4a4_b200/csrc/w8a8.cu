@@ -332,12 +332,18 @@ int launch_w8_gemm(const svdq_w8a8_layer* L, int64_t M, void* Y, uint8_t* ws, cu
   p.Y = (uint16_t*)Y;
   p.status = (int*)(ws + w.ctrl);
   p.limit = wait_limit_cycles();
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(k_gemm_w8a8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-  });
-  if (attr != cudaSuccess) return SVDQ_ERR_CUDA;
+  {  // the shared-memory attribute belongs to the kernel on each device: set it once per device
+    static std::mutex mu;
+    static bool attr_set[64] = {};
+    if (L->device < 0 || L->device >= 64) return SVDQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[L->device]) {
+      if (cudaFuncSetAttribute(k_gemm_w8a8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+          cudaSuccess)
+        return SVDQ_ERR_CUDA;
+      attr_set[L->device] = true;
+    }
+  }
   const int sms = w8_sm_count(L->device);
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   k_gemm_w8a8<<<grid, THREADS, SMEM_BYTES, stream>>>(maps, p);
