@@ -14,6 +14,11 @@ paragraph "Суть метода" (smoothing, 16-bit low-rank branch from the we
 4-bit residual, W4A4), and the paragraph after it (svdq_w4a4 in INT4 and NVFP4
 variants); "SVDQuant ускоряет Krea 2 вдвое ..." (ainews.so), section
 "Решение: INT8 и W4A4" (no calibration dataset; low-rank branches compensate).
+Beyond the svdq_w4a4 layer: the awq_w4a16 runtime layer the same iitog.ru page
+names for normalization / modulation layers (awq_*), the per-call (dynamic)
+per-tensor NVFP4 activation scale (act_tensor_scale, selected by g_x = 0), and
+the INT8 tensorwise W8A8 layer the ainews.so section compares (w8a8_*), each
+pinned in its own tests/test_oracle_*.py.
 """
 from __future__ import annotations
 
