@@ -9,18 +9,18 @@
 //
 // Work split: a CTA owns 128 token rows and one slice of K (the K range is cut
 // into enough slices that about one CTA per SM is in flight).  Per 128-column
-// chunk:
-//   warp 8      TMA: the X tile [128 x 128], and a bulk copy of the chunk's
+// chunk, with C quantizing warps (16, or 8 for ranks above 80):
+//   warp C      TMA: the X tile [128 x 128], and a bulk copy of the chunk's
 //               128 entries of 1/lambda, into a ring that the quantizing warps
 //               release as soon as they have read it;
-//   warp 10     TMA: the matching L1^T slice [rank x 128] (two 64-column boxes,
+//   warp C+2    TMA: the matching L1^T slice [rank x 128] (two 64-column boxes,
 //               128-byte swizzle) into a small ring released by the MMAs;
-//   warps 0-7   quantize 16 rows each (a lane holds 16 consecutive elements:
-//               one NVFP4 block, or a quarter of a 64-element INT4 group whose
-//               maximum takes two warp shuffles; products in packed f32x2),
-//               store codes and scales, and write bf16(x^) into a
+//   warps 0..C-1 quantize 128/C rows each (a lane holds 16 consecutive
+//               elements: one NVFP4 block, or a quarter of a 64-element INT4
+//               group whose maximum takes two warp shuffles; products in packed
+//               f32x2), store codes and scales, and write bf16(x^) into a
 //               128-byte-swizzled K-major tile;
-//   warp 9      issues tcgen05.mma kind::f16 (M = 128 tokens, N = rank, K = 16)
+//   warp C+1    issues tcgen05.mma kind::f16 (M = 128 tokens, N = rank, K = 16)
 //               on that tile and the L1^T slice, accumulating the slice's part of
 //               t in tensor memory.
 // At the end the slice's fp32 partial of t leaves tensor memory; the last CTA of
@@ -38,11 +38,18 @@ namespace {
 
 constexpr int kRows = kQRows;    // 128
 constexpr int kChunk = kQChunk;  // 128
-constexpr int kConsumerWarps = 8;
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kL1Warp = 10;
-constexpr int kThreads = 11 * 32;
+// Quantizing warps per CTA: 16 (8 rows each) where the registers allow it, 8
+// (16 rows each) for ranks above 80, whose fp32 partial of t takes a register per
+// rank column; the three role warps follow them.
+template <int RANK>
+struct Roles {
+  static constexpr int kConsumerWarps = RANK <= 80 ? 16 : 8;
+  static constexpr int kRowsPerWarp = 128 / kConsumerWarps;
+  static constexpr int kTmaWarp = kConsumerWarps;
+  static constexpr int kMmaWarp = kConsumerWarps + 1;
+  static constexpr int kL1Warp = kConsumerWarps + 2;
+  static constexpr int kThreads = (kConsumerWarps + 3) * 32;
+};
 constexpr int kXTileBytes = kRows * kChunk * 2;  // 32 KiB
 constexpr int kIlBytes = kChunk * 4;              // the chunk's 1/lambda slice
 constexpr int kXStageBytes = kXTileBytes + kIlBytes;
@@ -136,10 +143,13 @@ __device__ __forceinline__ float nvfp4_tensor_scale_dev(float amax) {
 }
 
 template <int FMT, int RANK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
     k_quantize(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1, QParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  constexpr int kConsumerWarps = Roles<RANK>::kConsumerWarps, kTmaWarp = Roles<RANK>::kTmaWarp;
+  constexpr int kMmaWarp = Roles<RANK>::kMmaWarp, kL1Warp = Roles<RANK>::kL1Warp, kThreads = Roles<RANK>::kThreads;
+  constexpr int kRowsPerWarp = Roles<RANK>::kRowsPerWarp;
   const int XS = p.xstages, LS = p.lstages;
   constexpr int kL1Bytes = RANK * kChunk * 2;  // two boxes of RANK rows x 128 B
   uint8_t* xring = smem;                          // [XS][X tile | 1/lambda slice]
@@ -310,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* at = atile + buf * kATileBytes + (j >> 2) * kAHalfBytes;
 #pragma unroll 2
-        for (int it = 0; it < 4; ++it) {
-          const int row = warp * 16 + 4 * it + rsub;
+        for (int it = 0; it < kRowsPerWarp / 4; ++it) {
+          const int row = warp * kRowsPerWarp + 4 * it + rsub;
           const int m = m0 + row;
           const uint4 r0 = *(const uint4*)(st + row * (kChunk * 2) + 32 * j);
           const uint4 r1 = *(const uint4*)(st + row * (kChunk * 2) + 32 * j + 16);
@@ -489,7 +499,7 @@ int launch_rank(const CUtensorMap& mx, const CUtensorMap& ml1, const QParams& p,
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   const dim3 grid((unsigned)((M + kRows - 1) / kRows), (unsigned)p.nslices);
-  kern<<<grid, kThreads, smem, stream>>>(mx, ml1, q);
+  kern<<<grid, Roles<RANK>::kThreads, smem, stream>>>(mx, ml1, q);
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
