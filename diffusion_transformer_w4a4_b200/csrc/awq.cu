@@ -158,8 +158,19 @@ __global__ void __launch_bounds__(kAwqMaxThreads) k_awq_gemv(const __grid_consta
   }
   __syncthreads();
 
+  if (tid == 0) pdl_launch_dependents();  // the next layer's CTAs may start as SMs free up
+
   if (tid >= G * T) {  // ---------------------------------------- producer
     if (lane != 0) return;
+    // This kernel may start before the previous one on the stream has finished
+    // (programmatic dependent launch): warm L2 with the first batches' weights,
+    // which is only a hint, then wait for the previous kernel before copying.
+    for (int b = blockIdx.x, jj = 0; b < nbatch && jj < S; b += gridDim.x, ++jj) {
+      const int rows = (p.N - b * R) < R ? (p.N - b * R) : R;
+      prefetch_l2_bulk(p.codes + (size_t)b * R * row_bytes, (uint32_t)(rows * row_bytes));
+      prefetch_l2_bulk(p.scales + (size_t)b * R * ld, (uint32_t)(rows * ld * 2));
+    }
+    pdl_wait();
     int s = 0, j = 0;
     uint32_t ph = 0;  // parity of the current fill of stage s
     const size_t xs_lo = (size_t)p.xs_off;
@@ -189,6 +200,7 @@ __global__ void __launch_bounds__(kAwqMaxThreads) k_awq_gemv(const __grid_consta
   const int nchunk = p.K >> 5;
   const bool active = t < nchunk;
 
+  pdl_wait();  // x and y belong to the stream's order
   // x^ = f32(x) * inv_s for the CTA's token rows, computed once with coalesced
   // loads into the ring's tail; float4 q of chunk c of token m sits at unit
   // m*K/4 + c*8 + (q ^ (c & 7)), so that each thread's reads of its own chunk
@@ -388,7 +400,17 @@ int launch_awq(AwqParams p, int dev, cudaStream_t stream) {
   const int nbatch = (p.N + R - 1) / R;
   int grid = awq_sm_count(dev) * per_sm;
   if (grid > nbatch) grid = nbatch;
-  k_awq_gemv<MB><<<grid, a.G * a.T + 32, a.smem, stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(a.G * a.T + 32);
+  cfg.dynamicSmemBytes = a.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see pdl_wait in the kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_awq_gemv<MB>, p) != cudaSuccess) return SVDQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 

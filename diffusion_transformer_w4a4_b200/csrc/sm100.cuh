@@ -117,6 +117,16 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel on the stream start its
+// prologue while this one runs, and wait for the previous kernel's completion
+// (and the visibility of its writes) before touching what it produced.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Hint: bring `bytes` (a multiple of 16) at a 16-byte-aligned global address into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Hint: bring a tile of a tensor into L2 ahead of its load (no completion, no
 // shared memory).
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
