@@ -18,11 +18,12 @@ import workloads as wl
 #    is within gamma_K * sum|terms| of the exact sum (gamma_K ~ K u, u = 2^-24;
 #    taken as K 2^-23 to cover truncating accumulators), plus one bf16 ulp of
 #    the final rounding.
-# Y: the stated gates rel-L2 <= 1e-3 and max-abs 2e-2.  Elementwise, 2e-2 is
-#    widened by one bf16 ulp of the oracle value (two correct accumulation
-#    orders round to neighbouring bf16 values once |y| >= 4) and by the forward
-#    error of the fp32 arithmetic: the t bound carried through L2, and the fp32
-#    accumulation bound of the main product.
+# Y: the stated gates rel-L2 <= 1e-3 and max-abs 2e-2, with the elementwise
+#    bound widened by exactly one bf16 ulp of the oracle value: two correct fp32
+#    accumulation orders of the same exact sum round to neighbouring bf16 values
+#    once |y| >= 4, where one bf16 ulp (1/32) already exceeds 2e-2.  Nothing
+#    else widens the gate; the fp32 forward-error bound of the arithmetic
+#    (y_error_bound) is reported beside it as a diagnostic only.
 REL_L2 = 1e-3
 MAX_ABS = 2e-2
 
@@ -76,23 +77,38 @@ def y_error_bound(act: dict, prep: dict):
     return bound
 
 
-def y_stats(y_gpu_bits, y_orc_bits, extra=None):
+def y_stats(y_gpu_bits, y_orc_bits, diag=None):
     g, o = bf(y_gpu_bits), bf(y_orc_bits)
     d = np.abs(g - o)
-    lim = MAX_ABS + bf16_ulp(o) + (0.0 if extra is None else extra)
-    return dict(rel_l2=float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30)), max_abs=float(d.max()),
-                n_over_abs=int(np.sum(d > MAX_ABS)), n_over_abs_ulp=int(np.sum(d > MAX_ABS + bf16_ulp(o))),
-                n_flip=int(np.sum(g != o)), worst_excess=float(np.max(d - lim)),
-                nonfinite=int(np.sum(~np.isfinite(g))))
+    lim = MAX_ABS + bf16_ulp(o)
+    s = dict(rel_l2=float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30)), max_abs=float(d.max()),
+             n_over_abs=int(np.sum(d > MAX_ABS)), n_over_abs_ulp=int(np.sum(d > lim)),
+             n_flip=int(np.sum(g != o)), worst_excess=float(np.max(d - lim)),
+             nonfinite=int(np.sum(~np.isfinite(g))))
+    if diag is not None:  # how much of the fp32 forward-error allowance the result uses
+        s["max_err_over_fp32_bound"] = float(np.max(np.maximum(d - bf16_ulp(o), 0.0) / np.maximum(diag, 1e-300)))
+    return s
 
 
 def assert_y_close(y_gpu_bits, y_orc_bits, act=None, prep=None):
-    extra = y_error_bound(act, prep) if act is not None else None
-    s = y_stats(y_gpu_bits, y_orc_bits, extra)
+    """rel-L2 <= 1e-3 and |dy| <= 2e-2 + 1 bf16 ulp(|y_oracle|) on every element."""
+    diag = y_error_bound(act, prep) if act is not None else None
+    s = y_stats(y_gpu_bits, y_orc_bits, diag)
     assert s["nonfinite"] == 0, s
     assert s["rel_l2"] <= REL_L2, s
-    assert s["worst_excess"] <= 0.0, s
+    assert s["n_over_abs_ulp"] == 0, s
     return s
+
+
+def tile_rows(M, seed, spread=40, tile=128):
+    """Sampled output rows: one seeded row inside every 128-row M tile (the ragged
+    last tile included), the first/last rows of the first two tiles and of the
+    tail, and a seeded spread."""
+    rng = np.random.default_rng(seed)
+    starts = np.arange(0, M, tile)
+    per_tile = starts + rng.integers(0, np.minimum(tile, M - starts))
+    fixed = [r for r in (0, 1, 127, 128, 255, M - 129, M - 128, M - 1) if 0 <= r < M]
+    return np.unique(np.concatenate([fixed, per_tile, rng.choice(M, min(M, spread), replace=False)]))
 
 
 def assert_t_close(t_gpu, t_orc, act=None, prep=None):

@@ -3,8 +3,11 @@ the oracle, through the C ABI, on the FLUX modulation shapes and on small shapes
 with ragged N, several passes over token rows, tiny K and M = 0.
 
 Bar: bf16 Y within rel-L2 1e-3 and, elementwise, 2e-2 + one bf16 ulp of the
-oracle value + the forward error of binary32 accumulation (K 2^-22 times the sum
-of |x^| |w|), the same reading of the tolerance as for svdq_w4a4."""
+oracle value, the same gate as for svdq_w4a4.  On inputs scaled by 2^k away
+from the calibration the output scales by 2^k, and so does the absolute part of
+the gate (2e-2 * 2^k): the stated max-abs is read in the layer's own units.  The
+forward error of binary32 accumulation (K 2^-22 times the sum of |x^| |w|) is
+reported as a diagnostic only."""
 import numpy as np
 import pytest
 
@@ -48,13 +51,16 @@ def _run(layer, x_scale=1.0):
     g, o = oracle.bf16_to_f32(got).astype(np.float64), oracle.bf16_to_f32(ref).astype(np.float64)
     xh = np.abs(oracle.smooth_act(X, prep["inv_s"]).astype(np.float64))
     wabs = np.abs(oracle.dequant(prep["wcodes"], prep["wscales"], oracle.INT4))
-    bound = MAX_ABS + bf16_ulp(o) + prep["K"] * 2.0 ** -22 * (xh @ wabs.T)
+    fp32_bound = prep["K"] * 2.0 ** -22 * (xh @ wabs.T)
+    bound = MAX_ABS * x_scale + bf16_ulp(o)
     d = np.abs(g - o)
     rel = float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30))
     assert np.all(np.isfinite(g))
     assert rel <= REL_L2, rel
-    assert np.all(d <= bound), float(np.max(d - bound))
-    return dict(rel_l2=rel, max_abs=float(d.max()), n_flip=int(np.sum(got != ref)), alpha=prep["alpha"])
+    assert np.all(d <= bound), (int(np.sum(d > bound)), float(np.max(d - bound)))
+    used = float(np.max(np.maximum(d - bf16_ulp(o), 0.0) / np.maximum(fp32_bound, 1e-300)))
+    return dict(rel_l2=rel, max_abs=float(d.max()), n_flip=int(np.sum(got != ref)), alpha=prep["alpha"],
+                max_err_over_fp32_bound=used)
 
 
 @pytest.mark.parametrize("name", list(wl.AWQ_LAYERS))

@@ -22,7 +22,7 @@ import pytest
 
 import oracle
 import workloads as wl
-from svdq_cases import GpuLayer, assert_t_close, assert_y_close
+from svdq_cases import GpuLayer, assert_t_close, assert_y_close, tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -44,9 +44,9 @@ def _device():
 
 
 def _rows(M):
-    """First/last rows of the first two 128-row tiles and of the tail, plus a seeded spread."""
-    fixed = [0, 1, 127, 128, 255, M - 129, M - 128, M - 1]
-    return np.unique(np.concatenate([fixed, np.random.default_rng(7).choice(M, 40, replace=False)]))
+    """One seeded row in every 128-row tile, the edges of the first two tiles and of
+    the tail, and a seeded spread."""
+    return tile_rows(M, 7)
 
 
 def _check_layer(gl, X, prep, rows):

@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 import workloads as wl
-from svdq_cases import GpuLayer, assert_t_close, assert_y_close, oracle_layer
+from svdq_cases import GpuLayer, assert_t_close, assert_y_close, oracle_layer, tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -72,7 +72,7 @@ def test_dynamic_scale_flux_shape_sampled_rows(name, idx):
     np.testing.assert_array_equal(got["codes"], ref["codes"])
     np.testing.assert_array_equal(got["scales"], ref["scales"])
     assert_t_close(got["t"], ref["t"], ref, dyn)
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], np.random.default_rng(3).choice(M, 40, replace=False)]))
+    rows = tile_rows(M, 3)
     sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
     assert_y_close(y[rows], oracle.forward_from_act(sub, dyn), sub, dyn)
 

@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 import workloads as wl
-from svdq_cases import GpuLayer, assert_t_close, assert_y_close, oracle_layer, y_stats
+from svdq_cases import GpuLayer, assert_t_close, assert_y_close, oracle_layer, tile_rows, y_stats
 
 pytestmark = pytest.mark.gpu
 
@@ -89,7 +89,7 @@ def test_flux_workloads_nvfp4(name):
     np.testing.assert_array_equal(got["scales"], ref["scales"])
     st = assert_t_close(got["t"], ref["t"], ref, prep)
     # sampled output rows: first/last tile rows and a seeded spread
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], np.random.default_rng(1).choice(M, 40, replace=False)]))
+    rows = tile_rows(M, 1)
     sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
     y_ref = oracle.forward_from_act(sub, prep)
     s = assert_y_close(y[rows], y_ref, sub, prep)
@@ -167,7 +167,7 @@ def test_flux_workloads_int4(name):
     np.testing.assert_array_equal(got["codes"], ref["codes"])
     np.testing.assert_array_equal(got["scales"], ref["scales"])
     st = assert_t_close(got["t"], ref["t"], ref, prep)
-    rows = np.unique(np.concatenate([[0, 1, M // 2, M - 1], np.random.default_rng(2).choice(M, min(M, 40), replace=False)]))
+    rows = tile_rows(M, 2)
     sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
     s = assert_y_close(y[rows], oracle.forward_from_act(sub, prep), sub, prep)
     print(name, s, st)

@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 import workloads as wl
+from svdq_cases import tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -86,7 +87,7 @@ def test_w8a8_flux_mlp_sampled_rows(K, N):
     ref = oracle.w8a8_quantize_act(X)
     assert got["s_x"] == ref["s_x"]
     np.testing.assert_array_equal(got["codes"], ref["codes"])
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], np.random.default_rng(9).choice(M, 40, replace=False)]))
+    rows = tile_rows(M, 9)
     print(K, N, _check_y(y, ref, prep, rows))
 
 
