@@ -18,7 +18,8 @@ Beyond the svdq_w4a4 layer: the awq_w4a16 runtime layer the same iitog.ru page
 names for normalization / modulation layers (awq_*), the per-call (dynamic)
 per-tensor NVFP4 activation scale (act_tensor_scale, selected by g_x = 0), and
 the INT8 tensorwise W8A8 layer the ainews.so section compares (w8a8_*), each
-pinned in its own tests/test_oracle_*.py.
+pinned in its own tests/test_oracle_*.py, and the GELU between a block's MLP
+linears (gelu_bf16, for the fused MLP pair; pinned in test_oracle_gelu.py).
 """
 from __future__ import annotations
 
@@ -114,6 +115,22 @@ def e2m1_to_f32(x): return _vec("orc_vec_e2m1_to_f32", x, np.uint8, np.float32)
 
 def bf16_to_f32(h):
     return (np.asarray(h, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ----------------------------------------------------------------------------- GELU
+def gelu_f64(h: np.ndarray) -> np.ndarray:
+    """GELU in its erf form, h/2 (1 + erf(h / sqrt 2)), in binary64 (the
+    activation between a diffusion transformer block's MLP linears)."""
+    from scipy.special import erf
+
+    h = np.asarray(h, np.float64)
+    return 0.5 * h * (1.0 + erf(h / math.sqrt(2.0)))
+
+
+def gelu_bf16(h_bits: np.ndarray) -> np.ndarray:
+    """bf16 bits -> bf16 bits of GELU(h), computed in binary64 and rounded once
+    (round to nearest even)."""
+    return f64_to_bf16(np.ascontiguousarray(gelu_f64(bf16_to_f32(h_bits))))
 
 
 # ----------------------------------------------------------------------------- smoothing
