@@ -200,14 +200,41 @@ def _prepare_layers(seed=0):
     return canons, xs
 
 
-def run_reference(args, world, rank):
-    if rank != 0:
-        return
-    canons, xs = _prepare_layers()
+def _config(world):
+    return {"workload": WORKLOAD + "_nvfp4", "layers": [f"{l.M}x{l.K}->{l.N}" for l in LAYERS],
+            "rank": LAYERS[0].rank, "l2": "flushed between steps (256 MiB write)",
+            "parallelism": f"replicas x{world}"}
+
+
+def _oracle_prepare_layers(seed=0):
+    """Oracle-side preparation (binary64 SVD, the oracle's own quantizers) of both
+    layers, from the same seeded inputs as the product side."""
     import oracle
 
-    preps = [_oracle_prep(c) for c in canons]
-    rows = 4
+    preps, xs = [], []
+    for l in LAYERS:
+        X, W, b = wl.make_layer_inputs(l, seed)
+        preps.append(oracle.prepare(W, b, oracle.calib_absmax(X), 0.5, l.rank, l.fmt))
+        xs.append(X)
+    return preps, xs
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, on the host cores, on the bench's workload: each
+    step quantizes and multiplies a sample of token rows of both layers, sized
+    from two probes so that the oracle's fixed per-call cost (decoding every
+    weight code) is amortized and the whole run takes about two minutes."""
+    if rank != 0:
+        return
+    import oracle
+
+    preps, xs = _oracle_prepare_layers()
+    _, t2 = oracle_sample(preps, xs, 2)
+    _, t34 = oracle_sample(preps, xs, 34)
+    per_row = max((t34 - t2) / 32.0, 1e-4)
+    fixed = max(t2 - 2 * per_row, 0.0)
+    per_step = 120.0 / max(args.steps + args.warmup, 1)
+    rows = int(max(32, min(LAYERS[0].M, (per_step - fixed) / per_row)))
     for _ in range(args.warmup):
         oracle_sample(preps, xs, rows)
     tot_f, tot_t = 0.0, 0.0
@@ -216,12 +243,13 @@ def run_reference(args, world, rank):
         tot_f += f
         tot_t += t
     val = tot_f / tot_t / 1e12
-    sample = f"{rows} token rows of each MLP layer per step (full layer is {LAYERS[0].M} rows)"
+    sample = (f"{rows} token rows of each MLP layer per step (full layer is {LAYERS[0].M} rows); "
+              f"fixed per-call cost {fixed:.2f} s, {per_row * 1e3:.2f} ms per row pair")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD + "_nvfp4", "sample": sample},
+        "config": _config(world),
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
@@ -378,6 +406,217 @@ def w8a8_measure(dev, xs, steps=20):
             "gpu_launches": 6 * steps}
 
 
+def fused_mlp_measure(dev, lins, xs, steps=20):
+    """The same MLP pair with cross-layer fusion: per step the up layer's
+    quantizer, the up GEMM whose epilogue applies GELU and writes the down layer's
+    quantized input (codes, scales, t') instead of y_up, and the down GEMM; L2
+    flushed between steps like the main line.  (The unfused line's down input is
+    its own seeded tensor, so the two lines time the same kernels' work except
+    that the fused one also computes the GELU.)"""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    up, dn = lins
+    if svdq.svdq_mlp_fusable(up.handle, dn.handle) != svdq.SVDQ_OK:
+        return {"unavailable": "layer pair not fusable"}
+    l_up, l_dn = LAYERS
+    M = l_up.M
+    x = torch.from_numpy(xs[0].view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.empty(M, l_dn.N, dtype=torch.bfloat16, device=dev)
+    ws_up, ws_dn = up.workspace(M), dn.workspace(M)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps + 3)]
+    for e in evs:
+        flush.zero_()
+        e[0].record(stream)
+        svdq.svdq_quantize_act(up.handle, x, M, ws_up, sp)
+        e[1].record(stream)
+        svdq.svdq_gemm_gelu_quantize(up.handle, dn.handle, M, ws_up, ws_dn, None, sp)
+        e[2].record(stream)
+        svdq.svdq_gemm(dn.handle, M, y, ws_dn, sp)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    assert up.status(M) == 0 and dn.status(M) == 0, "kernel reported an error (fused MLP)"
+    ev = evs[3:]
+    med = lambda a, b: statistics.median([e[a].elapsed_time(e[b]) for e in ev]) * 1e3
+    step = med(0, 3)
+    flops = sum(_layer_flops(l) for l in LAYERS)
+    return {"step_us": step, "quantize_up_us": med(0, 1), "fused_gemm_gelu_quantize_us": med(1, 2),
+            "gemm_down_us": med(2, 3), "tops": flops / (step * 1e-6) / 1e12,
+            "kernels": ["k_quantize", "k_gemm_gelu_quant", "k_gemm_nvfp4_pair"], "gpu_launches": 3 * steps,
+            "note": "compare step_us with ms_per_step of the main line (unfused: two quantizers, two GEMMs)"}
+
+
+def _random_canonical(N, K, r, fmt, rng):
+    """Valid prepared weights with seeded random codes and scales.  The kernels'
+    run time does not depend on the weight values, so the per-config timings use
+    these instead of a host SVD of every shape (the main line above uses the
+    product's own preparation of the seeded FLUX weights)."""
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    c = svdq._canonical_arrays(N, K, r, fmt)
+    c["inv_lambda"][:] = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    c["lambda_"][:] = (1.0 / c["inv_lambda"].astype(np.float64)).astype(np.float32)
+    c["L1"][:] = wl.f32_to_bf16_bits(rng.standard_normal((K, r)).astype(np.float32) * 0.05)
+    c["L2"][:] = wl.f32_to_bf16_bits(rng.standard_normal((r, N)).astype(np.float32) * 0.05)
+    c["wcodes"][:] = rng.integers(0, 256, c["wcodes"].shape)
+    if fmt == wl.NVFP4:
+        c["wscales"][:] = rng.integers(0x20, 0x60, c["wscales"].shape)
+        c["g_x"], c["g_w"] = 2.0 ** -6, 2.0 ** -12
+    else:
+        c["wscales"][:] = rng.integers(0x1000, 0x2400, c["wscales"].shape)
+    c["bias"][:] = wl.f32_to_bf16_bits(rng.standard_normal(N).astype(np.float32) * 0.01)
+    return c
+
+
+def _peak_for(fmt):
+    _, bf16, _, src = _peaks()
+    if fmt == wl.NVFP4:
+        return 4.0 * bf16, f"{src} bf16 {bf16} TFLOP/s (burst) x 4 (nominal fp4/bf16)"
+    return 2.0 * bf16, f"{src} bf16 {bf16} TFLOP/s (burst) x 2 (nominal int8/bf16; INT4 runs on 8-bit tensor cores)"
+
+
+def _time_layer(lin, x, y, M, flush, reps=20):
+    """Median quantize / GEMM / layer times (us) with L2 flushed before every rep."""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    ws = lin.workspace(M)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps + 3)]
+    for ev in evs:
+        flush.zero_()
+        ev[0].record(stream)
+        svdq.svdq_quantize_act(lin.handle, x, M, ws, sp)
+        ev[1].record(stream)
+        svdq.svdq_gemm(lin.handle, M, y, ws, sp)
+        ev[2].record(stream)
+    torch.cuda.synchronize()
+    assert lin.status(M) == 0, "kernel reported an error"
+    ev = evs[3:]
+    q = statistics.median([e[0].elapsed_time(e[1]) for e in ev]) * 1e3
+    g = statistics.median([e[1].elapsed_time(e[2]) for e in ev]) * 1e3
+    t = statistics.median([e[0].elapsed_time(e[2]) for e in ev]) * 1e3
+    return q, g, t
+
+
+def _graph_times(lin, x, y, M, flush, n=40):
+    """us per forward from CUDA graphs: back to back with the weights warm in L2,
+    and with an L2 flush before each forward (a graph of flushes alone subtracted)."""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    ws = lin.workspace(M)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graphs = {}
+    with torch.cuda.stream(side):
+        for kind in ("warm", "cold", "flush"):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(n):
+                    if kind != "warm":
+                        flush.zero_()
+                    if kind != "flush":
+                        svdq.svdq_forward(lin.handle, x, M, y, ws, side.cuda_stream)
+            graphs[kind] = g
+    torch.cuda.current_stream().wait_stream(side)
+    out = {}
+    for kind, g in graphs.items():
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3 / n)
+        out[kind] = statistics.median(ts)
+    assert lin.status(M) == 0, "kernel reported an error (graph)"
+    del graphs
+    return {"graph_warm_l2_us": out["warm"], "graph_cold_l2_us": max(out["cold"] - out["flush"], 0.0)}
+
+
+def configs_measure(dev):
+    """Every other configuration of the workload list, one entry each: the
+    128-token INT4 layer and the 1024-token NVFP4 layer (eager with L2 flushed,
+    and from CUDA graphs), the FLUX QKV projection and MLP pair in both formats,
+    and the batch-2 block's four linears at ranks 16/32/64/128 (NVFP4)."""
+    import torch
+
+    import diffusion_transformer_w4a4_b200 as svdq
+
+    rng = np.random.default_rng(4321)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    xcache = {}
+
+    def xdev(M, K):
+        if (M, K) not in xcache:
+            xcache[(M, K)] = torch.randn(M, K, device=dev).to(torch.bfloat16)
+        return xcache[(M, K)]
+
+    def one(M, K, N, r, fmt, graphs=False):
+        lin = svdq.SvdqLinear(_random_canonical(N, K, r, fmt, rng), device=dev)
+        x = xdev(M, K)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        q, g, t = _time_layer(lin, x, y, M, flush)
+        peak, src = _peak_for(fmt)
+        flops = 2.0 * M * N * K
+        e = {"shape": f"{M}x{K}->{N}", "rank": r, "fmt": fmt, "quantize_us": q, "gemm_us": g, "layer_us": t,
+             "layer_tops": flops / (t * 1e-6) / 1e12,
+             "gemm_roofline": {"bound": "tensor", "achieved": flops / (g * 1e-6) / 1e12, "peak": peak,
+                               "unit": "TFLOP/s" if fmt == wl.NVFP4 else "TOPS",
+                               "frac": flops / (g * 1e-6) / 1e12 / peak, "peak_source": src}}
+        if graphs:
+            e.update(_graph_times(lin, x, y, M, flush))
+        del lin
+        return e
+
+    out = {"timing": "CUDA events, median of 20 with L2 flushed before each; weights are seeded random valid "
+                     "codes and scales (run time does not depend on their values); X ~ N(0,1) bf16"}
+    out["c1_int4_128x1024x1024_r32"] = one(128, 1024, 1024, 32, wl.INT4, graphs=True)
+    out["c2_nvfp4_1024x3072x3072_r32"] = one(1024, 3072, 3072, 32, wl.NVFP4, graphs=True)
+    for fmt in (wl.NVFP4, wl.INT4):
+        out[f"c3_qkv_4608x3072x9216_r32_{fmt}"] = one(4608, 3072, 9216, 32, fmt)
+    up, dn = one(4608, 3072, 12288, 32, wl.INT4), one(4608, 12288, 3072, 32, wl.INT4)
+    flops = 2 * 2.0 * 4608 * 3072 * 12288
+    peak, src = _peak_for(wl.INT4)
+    gsum = up["gemm_us"] + dn["gemm_us"]
+    out["c4_mlp_4608x3072x12288_r32_int4"] = {
+        "up": up, "down": dn, "step_us": up["layer_us"] + dn["layer_us"],
+        "tops": flops / ((up["layer_us"] + dn["layer_us"]) * 1e-6) / 1e12,
+        "gemm_roofline": {"bound": "tensor", "achieved": flops / (gsum * 1e-6) / 1e12, "peak": peak, "unit": "TOPS",
+                          "frac": flops / (gsum * 1e-6) / 1e12 / peak, "peak_source": src}}
+    xcache.clear()
+    M = wl.BLOCK_M
+    peak, src = _peak_for(wl.NVFP4)
+    for r in wl.BLOCK_RANKS:
+        lay = {}
+        for name, (K, N) in (("qkv", (3072, 9216)), ("out", (3072, 3072)), ("up", (3072, 12288)),
+                             ("down", (12288, 3072))):
+            lay[name] = one(M, K, N, r, wl.NVFP4)
+        tot = sum(v["layer_us"] for v in lay.values())
+        gsum = sum(v["gemm_us"] for v in lay.values())
+        flops = sum(2.0 * M * int(v["shape"].split("x")[1].split("->")[0]) * int(v["shape"].split("->")[1])
+                    for v in lay.values())
+        out[f"c5_block_9216_nvfp4_r{r}"] = {
+            "linears": lay, "block_us": tot, "tops": flops / (tot * 1e-6) / 1e12,
+            "gemm_roofline": {"bound": "tensor", "achieved": flops / (gsum * 1e-6) / 1e12, "peak": peak,
+                              "unit": "TFLOP/s", "frac": flops / (gsum * 1e-6) / 1e12 / peak, "peak_source": src}}
+        xcache.clear()
+    del flush
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -515,9 +754,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales) + bf16 low-rank, f32 accumulate", "data": "synthetic",
-        "config": {"workload": WORKLOAD + "_nvfp4", "layers": [f"{l.M}x{l.K}->{l.N}" for l in LAYERS],
-                   "rank": LAYERS[0].rank, "l2": "flushed between steps (256 MiB write)",
-                   "parallelism": f"replicas x{world}"},
+        "config": _config(world),
         "roofline": roofline, "quantize_roofline": quant,
         "per_layer_us": {"gemm_up": statistics.median(g_up) * 1e3, "gemm_down": statistics.median(g_dn) * 1e3,
                          "quantize_both": statistics.median(q_ms) * 1e3,
@@ -527,6 +764,9 @@ def run_ours(args, world, rank, local):
     out["awq_w4a16"] = awq_measure(dev, hbm)
     out["dynamic_act_scale"] = dynamic_measure(dev, canons, xs)
     out["w8a8"] = w8a8_measure(dev, xs)
+    out["fused_mlp"] = fused_mlp_measure(dev, lins, xs)
+    if not args.no_configs:
+        out["configs"] = configs_measure(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(canons, xs)
     if rank == 0:
@@ -541,6 +781,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-config timings")
     args = ap.parse_args()
     world, rank, local = _dist_init()
     try:

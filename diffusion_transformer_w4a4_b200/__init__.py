@@ -92,6 +92,13 @@ _EXPORTS = {
     "svdq_set_wait_limit": (ctypes.c_int, [ctypes.c_uint64]),
     "svdq_forward_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_void_p]),
+    "svdq_mlp_fusable": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "svdq_gemm_gelu_quantize": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                               ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                               ctypes.c_void_p]),
+    "svdq_mlp_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                        ctypes.c_size_t, ctypes.c_void_p]),
     "svdq_awq_canonical_sizes": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)]),
     "svdq_awq_prepare": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                         ctypes.POINTER(svdq_awq_canonical)]),
@@ -282,14 +289,34 @@ def svdq_int4_group_acc(h, M: int, ws, acc, stream=None) -> None:
 
 
 def svdq_read_status(h, M: int, ws) -> int:
+    """Status word of a caller workspace, or (ws=None) of the last
+    svdq_forward_noalloc call for M tokens on the current device."""
     v = ctypes.c_int()
-    _check(lib().svdq_read_status(h, M, _ptr(ws), ws.numel(), ctypes.byref(v)), "svdq_read_status")
+    nbytes = ws.numel() if ws is not None else 0
+    _check(lib().svdq_read_status(h, M, _ptr(ws), nbytes, ctypes.byref(v)), "svdq_read_status")
     return int(v.value)
 
 
 def svdq_forward_noalloc(h, X, M: int, Y, stream=None) -> None:
     """Forward without a caller workspace (library-owned 32 MiB scratch per GPU)."""
     _check(lib().svdq_forward_noalloc(h, _ptr(X), M, _ptr(Y), _stream(stream)), "svdq_forward_noalloc")
+
+
+def svdq_mlp_fusable(up, down) -> int:
+    """SVDQ_OK when the pair (up, down) can run as one fused MLP (see svdq_mlp_forward)."""
+    return int(lib().svdq_mlp_fusable(up, down))
+
+
+def svdq_gemm_gelu_quantize(up, down, M: int, ws_up, ws_dn, H=None, stream=None) -> None:
+    """The up layer's GEMM with GELU and the down layer's quantizer in its epilogue."""
+    _check(lib().svdq_gemm_gelu_quantize(up, down, M, _ptr(ws_up), ws_up.numel(), _ptr(ws_dn), ws_dn.numel(),
+                                         _ptr(H), _stream(stream)), "svdq_gemm_gelu_quantize")
+
+
+def svdq_mlp_forward(up, down, X, M: int, Y, ws_up, ws_dn, stream=None) -> None:
+    """Y = down(GELU(up(X))) with the cross-layer fused GEMM in the middle."""
+    _check(lib().svdq_mlp_forward(up, down, _ptr(X), M, _ptr(Y), _ptr(ws_up), ws_up.numel(), _ptr(ws_dn),
+                                  ws_dn.numel(), _stream(stream)), "svdq_mlp_forward")
 
 
 def svdq_set_wait_limit(cycles: int) -> None:

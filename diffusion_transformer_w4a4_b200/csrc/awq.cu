@@ -524,6 +524,7 @@ svdq_status svdq_awq_forward(const svdq_awq_layer* L, const void* X, int64_t M, 
   p.status = L->status;
   p.limit = wait_limit_cycles();
   cudaStream_t s = (cudaStream_t)stream;
+  NvtxRange range("svdq/awq_gemv");
   for (int64_t m0 = 0; m0 < M; m0 += kAwqMaxMB) {
     p.m0 = (int)m0;
     const int64_t mb = (M - m0) < kAwqMaxMB ? (M - m0) : kAwqMaxMB;

@@ -1,0 +1,742 @@
+// K8: the MLP up-projection GEMM with the down-projection's activation
+// quantizer fused into its epilogue (cross-layer fusion of the MLP pair).
+//
+//   h  = bf16( g_x g_w [ sum_blocks (s_x s_w)(qx . qw) + t . L2/(g_x g_w) ] + b )   (the up layer's y)
+//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) in binary32
+//   x^' = f32(x') * inv_lambda'                                                     (the down layer's input)
+//   codes', E4M3 block scales'  of x^' (blocks of 16, static g_x'),  t' = bf16( bf16(x^') . L1' )
+//
+// "Hugging Face встроила Nunchaku в Diffusers ..." (iitog.ru), paragraph on
+// Nunchaku Lite: the original engine's speed comes from fused, model-specific
+// kernels.  Here the up layer's output never goes to memory: each epilogue
+// thread owns one token row of the tile, so the 16-column blocks of the down
+// layer's quantizer need no cross-thread step, and the up layer's N columns
+// are the down layer's K columns.  The low-rank sum t' runs over all N columns
+// of a row; each tile contributes bf16(x^'_tile) . L1'[tile columns] with a
+// pair MMA into a 32-column tensor-memory accumulator that persists across the
+// tiles of a work unit (one 256-row M tile times one of S contiguous groups of
+// N tiles), and the S partial sums of a row are added in a fixed order by the
+// unit that finishes last (counter per 128-row block), as the standalone
+// quantizer does for its K slices.
+//
+// Same main loop as the CTA-pair NVFP4 GEMM (k_gemm_nvfp4_pair: 256 x 192 tile,
+// cta_group::2, no multicast loads).  Roles per CTA (512 threads):
+//   warp 0      operand TMA producer            warp 1   tensor memory, main MMAs (leader)
+//   warps 2-9   epilogue: two warps per tensor-memory lane quarter, 96 columns each
+//   warps 10-13 scale-factor movers             warp 14  scale-factor producer
+//   warp 15     L1'^T slice loader and t' MMA issuer (leader), per tile
+// Tensor memory (512 columns): two 192-column accumulators, two 48-column
+// scale-factor buffers, and the 32-column t' accumulator, so the down layer's
+// rank is at most 32.  Every wait is bounded; no load uses cluster multicast.
+#include <cuda_bf16.h>
+
+#include <cstring>
+
+#include "sm100.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+namespace {
+
+constexpr int BM = kGemmBM;   // 128 rows per CTA
+constexpr int BN = kNvfp4BN;  // 192
+constexpr int PB_ROWS = BN / 2;
+constexpr int STAGES = 5;
+constexpr int A_BYTES = BM * 128;
+constexpr int B_BYTES = PB_ROWS * 128;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SFA_BYTES = 4 * kSfAtomBytes;
+constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;
+constexpr int SF_SLOTS = 2;
+constexpr int SF_SLOT_BYTES = 2 * (SFA_BYTES + SFB_BYTES);
+constexpr int XT_BYTES = 3 * BM * 128;    // bf16 x^' tile: three 64-column halves, 128B-swizzled
+constexpr int L1_MAX_ROWS = 16;           // rank/2 rows of L1'^T per CTA (rank <= 32)
+constexpr int L1_BYTES = 3 * L1_MAX_ROWS * 128;
+constexpr int THREADS = 512;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL = 2 * BN;
+constexpr uint32_t SF_BUF_COLS = 48;
+constexpr uint32_t TP_COL = SF_COL + 2 * SF_BUF_COLS;  // 480
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + XT_BYTES + L1_BYTES;
+constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(2 * BM, BN);
+constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(2 * BM, BN);
+static_assert(STAGE_BYTES % 1024 == 0 && SF_SLOT_BYTES % 1024 == 0 && XT_BYTES % 1024 == 0, "alignment");
+static_assert(SMEM_BYTES + 1024 + 512 <= 227 * 1024, "shared memory budget");
+static_assert(TP_COL + 32 <= TMEM_COLS, "tensor memory budget");
+
+struct FusedMaps {
+  CUtensorMap a, b, t[3], l2[3], l1dn;
+};
+
+struct FParams {
+  int M, N, K, m_tiles, n_tiles, num_units, S, k_stages, katoms;
+  int n_lr;
+  int lr_off[4], lr_w[4];
+  int rank_dn, katoms_dn;
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* bias;        // up layer
+  float out_scale;          // g_x g_w of the up layer (static)
+  const float* gx_dev;      // up layer's dynamic g_x (else null)
+  float g_w;
+  const float* inv_lambda_dn;
+  float den_dn, inv_g_dn;   // 6 g_x' and 1/g_x' of the down layer (powers of two: exact)
+  uint8_t* codes_dn;        // [M, N/2]
+  uint8_t* scales_dn;       // atom layout, 128-row tiles, katoms_dn
+  uint16_t* t_dn;           // [M, rank_dn]
+  float* tpart;             // [S, M, rank_dn]
+  int* counters;            // per 32-row group (128-row block x lane quarter)
+  uint16_t* H;              // optional [M, N] bf16: bf16(GELU(h))
+  int* status;
+  unsigned long long limit;
+};
+
+__device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
+
+__device__ __forceinline__ uint32_t cvt_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+__device__ __forceinline__ float e4m3_value(uint32_t c) {  // c in [0, 0x7E]
+  const uint32_t e = (c >> 3) & 0xF, m = c & 7;
+  if (e == 0) return (float)m * (1.0f / 512.0f);
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return out;
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// bf16 round-to-nearest-even of a binary32 value, returned as the binary32 it denotes
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_gemm_gelu_quant(const __grid_constant__ FusedMaps maps, const __grid_constant__ FParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sfring = smem + STAGES * STAGE_BYTES;
+  uint8_t* xt = sfring + SF_SLOTS * SF_SLOT_BYTES;  // 1024-aligned
+  uint8_t* l1s = xt + XT_BYTES;                     // 1024-aligned
+  uint64_t* full = (uint64_t*)(l1s + L1_BYTES);     // leader
+  uint64_t* empty = full + STAGES;                  // both
+  uint64_t* acc_full = empty + STAGES;              // both [2]
+  uint64_t* acc_empty = acc_full + 2;               // leader [2]: 16 epilogue warps
+  uint64_t* mma_done = acc_empty + 2;               // leader
+  uint64_t* sf_ready = mma_done + 1;                // leader [2]: 8 movers
+  uint64_t* sf_free = sf_ready + 2;                 // both [2]
+  uint64_t* sfs_full = sf_free + 2;                 // local [SF_SLOTS]
+  uint64_t* sfs_empty = sfs_full + SF_SLOTS;        // local
+  uint64_t* l1_full = sfs_empty + SF_SLOTS;         // leader: both CTAs' L1' slices
+  uint64_t* xt_full = l1_full + 1;                  // leader: 16 epilogue warps
+  uint64_t* xt_free = xt_full + 1;                  // both: t' MMAs of the tile done (x^' tile and L1' slot free)
+  uint64_t* tp_full = xt_free + 1;                  // both: the unit's t' sum is complete
+  uint64_t* tp_empty = tp_full + 1;                 // leader: 8 reader warps (4 per CTA)
+  uint64_t* tdone = tp_empty + 1;                   // leader: t' issuer drain
+  uint32_t* tmem_slot = (uint32_t*)(tdone + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  volatile int* ticket = abort_flag + 1;            // [4] one per lane-quarter reader warp
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  WaitCtl wc{abort_flag, p.status, p.limit};
+  const unsigned long long drain_limit = p.limit > (1ull << 24) ? p.limit : (1ull << 24);
+  const int units = p.n_lr + p.k_stages;
+  const int rh = p.rank_dn / 2;  // L1'^T rows per CTA
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 16);
+      mbar_init(&sf_ready[b], 8);
+      mbar_init(&sf_free[b], 1);
+    }
+    mbar_init(mma_done, 1);
+    for (int b = 0; b < SF_SLOTS; ++b) {
+      mbar_init(&sfs_full[b], 1);
+      mbar_init(&sfs_empty[b], 4);
+    }
+    mbar_init(l1_full, 1);
+    mbar_init(xt_full, 16);
+    mbar_init(xt_free, 1);
+    mbar_init(tp_full, 1);
+    mbar_init(tp_empty, 8);
+    mbar_init(tdone, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ operand producer (both CTAs)
+    if (lane == 0) {
+      prefetch_tmap(&maps.a);
+      prefetch_tmap(&maps.b);
+      int it = 0;
+      bool ok = true;
+      for (int u = pair; u < p.num_units && ok; u += npairs) {
+        const int mt = u % p.m_tiles, sg = u / p.m_tiles;
+        const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+        for (int nt = nt0; nt < nt1 && ok; ++nt) {
+          const int arow = mt * 2 * BM + (int)rank * BM, brow = nt * BN + (int)rank * PB_ROWS;
+          for (int st = 0; st < units; ++st, ++it) {
+            const int s = it % STAGES;
+            if (!mbar_wait_cl(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
+              ok = false;
+              break;
+            }
+            uint8_t* dst = smem + s * STAGE_BYTES;
+            const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+            if (st < p.n_lr) {
+              const int w = p.lr_w[st], mi = lr_map_index(w);
+              if (leader) mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)(BM + PB_ROWS) * 2 * w);
+              tma_load_2d_pair(&maps.t[mi], fbar, dst, p.lr_off[st], arow);
+              tma_load_2d_pair(&maps.l2[mi], fbar, dst + A_BYTES, p.lr_off[st], brow);
+            } else {
+              const int ks = st - p.n_lr;
+              if (leader) mbar_arrive_expect_tx(&full[s], 2u * STAGE_BYTES);
+              tma_load_2d_pair(&maps.a, fbar, dst, ks * 128, arow);
+              tma_load_2d_pair(&maps.b, fbar, dst + A_BYTES, ks * 128, brow);
+            }
+          }
+        }
+      }
+      if (!ok && leader) {
+        for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+          mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, drain_limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ main MMA issuer (leader)
+    if (leader && lane == 0) {
+      int it = 0, local = 0, kst = 0;
+      bool ok = true;
+      for (int u = pair; u < p.num_units && ok; u += npairs) {
+        const int sg = u / p.m_tiles;
+        const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+        for (int nt = nt0; nt < nt1 && ok; ++nt, ++local) {
+          const int b = local & 1;
+          if (!mbar_wait_cl(&acc_empty[b], ((local >> 1) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(b * BN);
+          uint32_t accum = 0;
+          for (int st = 0; st < units; ++st, ++it) {
+            const int s = it % STAGES;
+            if (!mbar_wait_cl(&full[s], (it / STAGES) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t b_addr = a_addr + A_BYTES;
+            if (st < p.n_lr) {
+              const int w = p.lr_w[st];
+              const uint32_t layout = w == 64 ? LAYOUT_SW128 : (w == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
+              const uint32_t sbo = 8u * 2u * (uint32_t)w;
+              for (int kk = 0; kk < w / 16; ++kk) {
+                mma_bf16_pair(d, make_sdesc(a_addr + 32 * kk, 16, sbo, layout),
+                              make_sdesc(b_addr + 32 * kk, 16, sbo, layout), IDESC_BF16, accum);
+                accum = 1;
+              }
+            } else {
+              const int sb = kst & 1;
+              if (!mbar_wait_cl(&sf_ready[sb], (kst >> 1) & 1, wc)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sfa_t = tmem + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+              const uint32_t sfb_t = sfa_t + 16;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                mma_nvf4_pair(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
+                              make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), IDESC_NVF4, sfa_t + 4 * j,
+                              sfb_t + 8 * j, accum);
+                accum = 1;
+              }
+              umma_commit_pair(&sf_free[sb], 3);
+              ++kst;
+            }
+            umma_commit_pair(&empty[s], 3);
+          }
+          if (ok) umma_commit_pair(&acc_full[b], 3);
+        }
+      }
+      umma_commit_pair(mma_done, 1);
+      mbar_wait_drain(mma_done, 0, drain_limit);
+    }
+  } else if (warp == 14) {
+    // ------------------------------------------------------------ scale-factor producer (both CTAs)
+    if (lane == 0) {
+      int pit = 0;
+      bool ok = true;
+      const int pairs_k = (p.k_stages + 1) / 2;
+      for (int u = pair; u < p.num_units && ok; u += npairs) {
+        const int mt = u % p.m_tiles, sg = u / p.m_tiles;
+        const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+        const int at = 2 * mt + (int)rank;
+        for (int nt = nt0; nt < nt1 && ok; ++nt) {
+          for (int j = 0; j < pairs_k; ++j, ++pit) {
+            const int slot = pit % SF_SLOTS;
+            if (!mbar_wait(&sfs_empty[slot], ((pit / SF_SLOTS) & 1) ^ 1, wc)) {
+              ok = false;
+              break;
+            }
+            const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
+            uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
+            mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
+            bulk_load(dst, p.sfa + ((size_t)at * p.katoms + 8 * j) * kSfAtomBytes, ns * SFA_BYTES, &sfs_full[slot]);
+            bulk_load(dst + 2 * SFA_BYTES, p.sfb + ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes,
+                      ns * SFB_BYTES, &sfs_full[slot]);
+          }
+        }
+      }
+      if (!ok) {
+        for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
+          mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, drain_limit);
+      }
+    }
+  } else if (warp >= 10 && warp <= 13) {
+    // ------------------------------------------------------------ scale-factor movers (both CTAs)
+    const int q = warp & 3;
+    int kst = 0, pit = 0;
+    bool ok = true;
+    for (int u = pair; u < p.num_units && ok; u += npairs) {
+      const int sg = u / p.m_tiles;
+      const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+      for (int nt = nt0; nt < nt1 && ok; ++nt) {
+        for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
+          const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
+          const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
+          if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
+          ok = ok && mbar_wait_cl(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+          if (!ok) break;
+          const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
+          const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
+          uint32_t ra[16], rb[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
+            ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + hh) * kSfAtomBytes + lane * 16);
+              rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
+            }
+          }
+          const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+          tmem_st_32x32b_x16(tq, ra);
+          tmem_st_32x32b_x32(tq + 16, rb);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster(mapa_shared(smem_u32(&sf_ready[sb]), 0));
+            if (last_of_pair) mbar_arrive(&sfs_empty[slot]);
+          }
+          if (last_of_pair) ++pit;
+        }
+      }
+    }
+  } else if (warp == 15) {
+    // ------------------------------------------------------------ L1'^T slices and t' MMAs
+    // Per tile: this CTA's rank/2 rows of L1'^T for the tile's 192 columns (three
+    // 64-column boxes, 128-byte swizzle) into its slot; the leader then issues
+    // t' += bf16(x^'_tile) . L1'[tile] (M = 256, N = rank, K = 192) once both
+    // CTAs' epilogues have written their x^' tiles, and releases the x^' tiles
+    // and the L1' slots when those MMAs complete.
+    if (lane == 0 && p.rank_dn > 0) {
+      bool ok = true;
+      int tt = 0, ut = 0;  // tiles and units done
+      const uint32_t l1bar = mapa_shared(smem_u32(l1_full), 0);
+      const uint32_t idesc_t = idesc_bf16_f32(2 * BM, p.rank_dn);
+      for (int u = pair; u < p.num_units && ok; u += npairs, ++ut) {
+        const int sg = u / p.m_tiles;
+        const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+        for (int nt = nt0; nt < nt1 && ok; ++nt, ++tt) {
+          // the slot is free once the previous tile's t' MMAs completed
+          if (!mbar_wait_cl(xt_free, (tt & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(l1_full, 2u * 3u * (uint32_t)rh * 128u);
+          for (int hb = 0; hb < 3; ++hb)
+            tma_load_2d_pair(&maps.l1dn, l1bar, l1s + hb * L1_MAX_ROWS * 128, nt * BN + 64 * hb, (int)rank * rh);
+          if (leader) {
+            if (!mbar_wait_cl(l1_full, tt & 1, wc) || !mbar_wait_cl(xt_full, tt & 1, wc)) {
+              ok = false;
+              break;
+            }
+            if (nt == nt0 && !mbar_wait_cl(tp_empty, (ut & 1) ^ 1, wc)) {  // the unit's t' was read out
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(xt), b0 = smem_u32(l1s);
+            for (int kk = 0; kk < 12; ++kk) {
+              const uint32_t hb = kk >> 2, koff = (kk & 3) * 32;
+              mma_bf16_pair(tmem + TP_COL, make_sdesc(a0 + hb * (BM * 128) + koff, 16, 1024, LAYOUT_SW128),
+                            make_sdesc(b0 + hb * (L1_MAX_ROWS * 128) + koff, 16, 1024, LAYOUT_SW128), idesc_t,
+                            (nt > nt0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit_pair(xt_free, 3);
+            if (nt + 1 == nt1) umma_commit_pair(tp_full, 3);
+          }
+        }
+      }
+      if (leader) {
+        umma_commit_pair(tdone, 1);
+        mbar_wait_drain(tdone, 0, drain_limit);
+      } else if (!ok) {
+        // the peer's slice copies complete on the leader's barrier; give them time to land
+        const unsigned long long t0 = clock64();
+        while ((unsigned long long)clock64() - t0 < (1ull << 16)) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-9, both CTAs)
+    const int e = warp - 2;         // 0..7
+    const int q = warp & 3;         // tensor-memory lane quarter
+    const int half = e >> 2;        // columns 96*half .. 96*half + 95 of the tile
+    const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;
+    const uint32_t empty_cl0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    const uint32_t empty_cl1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    const uint32_t xtfull_cl = mapa_shared(smem_u32(xt_full), 0);
+    const uint32_t tpempty_cl = mapa_shared(smem_u32(tp_empty), 0);
+    const int row = 32 * q + lane;  // row of this CTA's 128-row tile
+    int local = 0, tt = 0, ut = 0;
+    bool ok = true;
+    for (int u = pair; u < p.num_units && ok; u += npairs, ++ut) {
+      const int mt = u % p.m_tiles, sg = u / p.m_tiles;
+      const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+      const int rb = 2 * mt + (int)rank;  // 128-row block
+      const int64_t m = (int64_t)rb * BM + row;
+      const bool live = m < p.M;
+      for (int nt = nt0; nt < nt1 && ok; ++nt, ++local, ++tt) {
+        const int b = local & 1;
+        if (!mbar_wait_cl(&acc_full[b], (local >> 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        // the x^' tile may be overwritten once the previous tile's t' MMAs completed
+        if (p.rank_dn > 0 && !mbar_wait_cl(xt_free, (tt & 1) ^ 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN) + 96 * half;
+        uint64_t swords = 0;  // the six block scales' of this warp's columns, one byte each
+#pragma unroll 1
+        for (int blk = 0; blk < 6; ++blk) {
+          const int n = nt * BN + 96 * half + 16 * blk;  // first column (= the down layer's K index)
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tbase + 16 * blk, r);
+          float bb[16], il[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float4 v = __ldg((const float4*)(p.bias + n) + j);
+            const float4 w = __ldg((const float4*)(p.inv_lambda_dn + n) + j);
+            bb[4 * j] = v.x; bb[4 * j + 1] = v.y; bb[4 * j + 2] = v.z; bb[4 * j + 3] = v.w;
+            il[4 * j] = w.x; il[4 * j + 1] = w.y; il[4 * j + 2] = w.z; il[4 * j + 3] = w.w;
+          }
+          tmem_ld_wait();
+          if (blk == 5) {  // this warp's 96 accumulator columns are in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(b ? empty_cl1 : empty_cl0);
+          }
+          float2 v[8];
+          uint32_t hbits[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            // the up layer's bf16 output, GELU in binary32, rounded to bf16 (the down layer's input)
+            const float h0 = bf16_round(fmaf(__uint_as_float(r[2 * j]), out_scale, bb[2 * j]));
+            const float h1 = bf16_round(fmaf(__uint_as_float(r[2 * j + 1]), out_scale, bb[2 * j + 1]));
+            const float g0 = 0.5f * h0 * (1.0f + erff(h0 * 0.70710678118654752f));
+            const float g1 = 0.5f * h1 * (1.0f + erff(h1 * 0.70710678118654752f));
+            const __nv_bfloat162 gh = __floats2bfloat162_rn(g0, g1);
+            hbits[j] = *(const uint32_t*)&gh;
+            v[j] = __fmul2_rn(__bfloat1622float2(gh), make_float2(il[2 * j], il[2 * j + 1]));
+          }
+          if (p.H != nullptr && live) {  // parity export of the down layer's input
+            *(uint4*)(p.H + (size_t)m * p.N + n) = make_uint4(hbits[0], hbits[1], hbits[2], hbits[3]);
+            *(uint4*)(p.H + (size_t)m * p.N + n + 8) = make_uint4(hbits[4], hbits[5], hbits[6], hbits[7]);
+          }
+          float mx[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) mx[j] = fmaxf(fabsf(v[j].x), fabsf(v[j].y));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) mx[j] = fmaxf(mx[j], mx[j + 4]);
+          const float amax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+          const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, p.den_dn));
+          // 1 / (e4m3(sb) g') = (1 / e4m3(sb)) (1 / g'), exact: g' is a power of two
+          const float inv = sb != 0 ? __frcp_rn(e4m3_value(sb)) * p.inv_g_dn : 0.f;
+          const float2 inv2 = make_float2(inv, inv);
+          float2 qv[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) qv[j] = __fmul2_rn(v[j], inv2);
+          uint32_t c0 = cvt_e2m1x8(qv[0], qv[1], qv[2], qv[3]), c1 = cvt_e2m1x8(qv[4], qv[5], qv[6], qv[7]);
+          if (sb == 0) c0 = c1 = 0u;  // a zero block scale: all codes +0
+          if (live) *(uint2*)(p.codes_dn + (size_t)m * (p.N / 2) + n / 2) = make_uint2(c0, c1);
+          swords |= (uint64_t)sb << (8 * blk);
+          if (p.rank_dn > 0) {  // bf16(x^') into the swizzled x^' tile
+            uint32_t xb[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const __nv_bfloat162 hx = __float22bfloat162_rn(v[j]);
+              xb[j] = *(const uint32_t*)&hx;
+            }
+            const int col = 96 * half + 16 * blk;          // tile column of the block
+            const int hb = col >> 6, ch = (col & 63) >> 3;  // 64-column half, 16-byte chunk in the row
+            uint8_t* rowp = xt + hb * (BM * 128) + row * 128;
+            *(uint4*)(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(xb[0], xb[1], xb[2], xb[3]);
+            *(uint4*)(rowp + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(xb[4], xb[5], xb[6], xb[7]);
+          }
+        }
+        if (p.rank_dn > 0) {
+          fence_proxy_async_smem();  // x^' tile -> tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(xtfull_cl);
+        }
+        if (live) {
+          // scale bytes of blocks blk0 .. blk0 + 5 (four consecutive blocks share an atom word)
+          const int blk0 = (nt * BN + 96 * half) / 16;
+          if (half == 0) {  // blocks 12t .. 12t+5: a whole word, then the first half of the next
+            *(uint32_t*)(p.scales_dn + sf_offset(m, blk0, p.katoms_dn, kSfAtomRows)) = (uint32_t)swords;
+            *(uint16_t*)(p.scales_dn + sf_offset(m, blk0 + 4, p.katoms_dn, kSfAtomRows)) = (uint16_t)(swords >> 32);
+          } else {  // blocks 12t+6 .. 12t+11: the second half of a word, then a whole word
+            *(uint16_t*)(p.scales_dn + sf_offset(m, blk0, p.katoms_dn, kSfAtomRows)) = (uint16_t)swords;
+            *(uint32_t*)(p.scales_dn + sf_offset(m, blk0 + 2, p.katoms_dn, kSfAtomRows)) = (uint32_t)(swords >> 16);
+          }
+        }
+      }
+      // ------------------------------------------------------------ the unit's t' partial
+      if (ok && p.rank_dn > 0 && half == 0) {
+        if (!mbar_wait_cl(tp_full, ut & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r0[16], r1[16];
+        const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + TP_COL;
+        tmem_ld_32x32b_x16(ta, r0);
+        if (p.rank_dn > 16) tmem_ld_32x32b_x16(ta + 16, r1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tpempty_cl);
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          acc[j] = __uint_as_float(r0[j]);
+          acc[16 + j] = __uint_as_float(r1[j]);
+        }
+        const int R = p.rank_dn;
+        if (live && p.S > 1) {
+          float* dst = p.tpart + ((size_t)sg * p.M + m) * R;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (j < R) *(float4*)(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        }
+        if (p.S == 1) {  // one group covers every column: the sum is complete
+          if (live) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              if (j < R) {
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
+                *(uint2*)(p.t_dn + (size_t)m * R + j) = make_uint2(*(const uint32_t*)&h0, *(const uint32_t*)&h1);
+              }
+            }
+          }
+          continue;
+        }
+        __threadfence();
+        __syncwarp();
+        // the last of the S units to finish these 32 rows adds the partials in group order
+        int* cnt = p.counters + 4 * rb + q;
+        if (lane == 0) ticket[q] = atomicAdd(cnt, 1);
+        __syncwarp();
+        if (ticket[q] == p.S - 1) {
+          __threadfence();
+          if (live) {
+            for (int j = 0; j < R; j += 4) {
+              float4 sum = __ldcg((const float4*)(p.tpart + (size_t)m * R + j));
+              for (int g = 1; g < p.S; ++g) {
+                const float4 v4 = __ldcg((const float4*)(p.tpart + ((size_t)g * p.M + m) * R + j));
+                sum.x += v4.x;
+                sum.y += v4.y;
+                sum.z += v4.z;
+                sum.w += v4.w;
+              }
+              const __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+              const __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+              *(uint2*)(p.t_dn + (size_t)m * R + j) = make_uint2(*(const uint32_t*)&h0, *(const uint32_t*)&h1);
+            }
+          }
+          if (lane == 0) *cnt = 0;  // every unit has arrived: ready for the next call
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+int pair_units_groups(int m_tiles, int n_tiles, int npairs, int max_groups) {
+  int S = (npairs + m_tiles - 1) / m_tiles;
+  if (S > max_groups) S = max_groups;
+  if (S > n_tiles) S = n_tiles;
+  return S < 1 ? 1 : S;
+}
+
+}  // namespace
+
+int fused_mlp_supported(const svdq_layer* up, const svdq_layer* dn) {
+  if (!up || !dn) return SVDQ_ERR_INVALID_ARG;
+  if (up->fmt != SVDQ_NVFP4_G16 || dn->fmt != SVDQ_NVFP4_G16) return SVDQ_ERR_INVALID_ARG;
+  if (up->N != dn->K || up->device != dn->device) return SVDQ_ERR_INVALID_ARG;
+  if (dn->dyn_gx || dn->rank > 32 || up->N % kNvfp4BN != 0) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
+int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, uint8_t* ws, const Workspace& w,
+                           uint8_t* wsd, const Workspace& wd, void* H, cudaStream_t stream) {
+  int st = fused_mlp_supported(L, D);
+  if (st != SVDQ_OK) return st;
+  const int K = (int)L->K, N = (int)L->N, r = L->rank;
+  FusedMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
+                      (uint64_t)K / 2, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SVDQ_OK) return st;
+  maps.b = L->map_w_half;
+  FParams p{};
+  const LowRankChunks ch = lowrank_chunks(r);
+  p.n_lr = ch.n;
+  for (int i = 0; i < ch.n; ++i) {
+    p.lr_off[i] = ch.off[i];
+    p.lr_w[i] = ch.width[i];
+  }
+  if (r > 0) {
+    const int widths[3] = {64, 32, 16};
+    const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_64B,
+                                       CU_TENSOR_MAP_SWIZZLE_32B};
+    for (int i = 0; i < 3; ++i) {
+      if (widths[i] > r) continue;
+      st = encode_tmap_2d(&maps.t[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.t, (uint64_t)r, (uint64_t)M,
+                          (uint64_t)r * 2, widths[i], BM, swz[i]);
+      if (st != SVDQ_OK) return st;
+      maps.l2[i] = L->map_l2_half[i];
+    }
+  }
+  const int rd = D->rank;
+  if (rd > 0) {  // L1'^T [rd, N] bf16: per CTA rd/2 rows, 64 columns per box
+    st = encode_tmap_2d(&maps.l1dn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D->L1t, (uint64_t)D->K, (uint64_t)rd,
+                        (uint64_t)D->K * 2, 64, (uint32_t)rd / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != SVDQ_OK) return st;
+  }
+  p.M = (int)M;
+  p.N = N;
+  p.K = K;
+  p.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
+  p.n_tiles = N / BN;
+  p.k_stages = K / kKStage;
+  p.katoms = K / 64;
+  p.sfa = ws + w.scales;
+  p.sfb = L->wscales;
+  p.bias = L->bias;
+  p.out_scale = L->g_x * L->g_w;
+  p.gx_dev = L->dyn_gx ? (const float*)(ws + w.status + 4) : nullptr;
+  p.g_w = L->g_w;
+  p.rank_dn = rd;
+  p.katoms_dn = (int)(D->K / 64);
+  p.inv_lambda_dn = D->inv_lambda;
+  p.den_dn = 6.0f * D->g_x;
+  p.inv_g_dn = 1.0f / D->g_x;  // exact: a power of two
+  p.codes_dn = wsd + wd.codes;
+  p.scales_dn = wsd + wd.scales;
+  p.t_dn = (uint16_t*)(wsd + wd.t);
+  p.tpart = (float*)(wsd + wd.tpart);
+  // one counter per 32-row group in the down workspace's first-pass slots (idle:
+  // the down layer has a static activation scale); zero between calls
+  if (4 * ((M + BM - 1) / BM) > kAmaxSlots) return SVDQ_ERR_INVALID_ARG;
+  p.counters = (int*)(wsd + wd.amax);
+  p.H = (uint16_t*)H;
+  p.status = (int*)(ws + w.status);
+  p.limit = wait_limit_cycles();
+
+  const size_t smem = 1024 + (size_t)SMEM_BYTES + 512;
+  static int attr_done[64] = {0};
+  const int dev = L->device;
+  if (dev < 0 || dev >= 64) return SVDQ_ERR_INVALID_ARG;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(k_gemm_gelu_quant, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  static int maxc_cache[64] = {0};
+  if (!maxc_cache[dev]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_gelu_quant, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return SVDQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    maxc_cache[dev] = n;
+  }
+  const int npairs_max = maxc_cache[dev];
+  // work units: (256-row M tile) x (one of S groups of N tiles); the t' partial
+  // sums of the groups land in the down layer's split-K area (wd.nslices of them)
+  const int S = pair_units_groups(p.m_tiles, p.n_tiles, npairs_max, rd > 0 ? wd.nslices : p.n_tiles);
+  if (rd > 0 && S > 1 && wd.tpart_bytes < (size_t)S * M * rd * 4) return SVDQ_ERR_INVALID_ARG;
+  p.S = S;
+  p.num_units = p.m_tiles * S;
+  const int npairs = p.num_units < npairs_max ? p.num_units : npairs_max;
+  k_gemm_gelu_quant<<<2 * npairs, THREADS, smem, stream>>>(maps, p);
+  return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+}  // namespace svdq

@@ -369,6 +369,332 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   }
 }
 
+// ------------------------------------------------------------------------------
+// CTA-pair variant: a cluster of two CTAs computes a 256 x 192 tile with
+// tcgen05.mma cta_group::2 (M = 256).  CTA r of the pair holds accumulator rows
+// 128r..128r+127 in its own tensor memory; its shared memory holds activation
+// rows 128r.. of the tile and weight rows 96r..96r+95 (each CTA loads its own
+// halves -- no multicast), and the pair MMA reads the B halves of both CTAs.
+// Per SM and per 256-deep K stage that is 16 KiB of activation codes and
+// 12 KiB of weight codes for the same tensor work as the single-CTA tile's
+// 16 + 24 KiB.  Each CTA keeps the E4M3 scale factors of its own 128 rows and
+// of all 192 weight rows in its tensor memory (the pair MMA reads both).
+// Only CTA 0 ("leader") issues MMAs; its operand barriers count the bytes of
+// both CTAs' loads, and it waits for both CTAs' scale-factor movers and
+// epilogues.  Its MMA completions are signalled to the same barrier in both
+// CTAs (multicast commit).
+constexpr int PB_ROWS = BN / 2;              // 96 weight rows per CTA
+constexpr int P_STAGES = 6;
+constexpr int P_B_BYTES = PB_ROWS * 128;     // 12 KiB
+constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + 4 * 2 * EPI_STAGE_BYTES;
+constexpr uint32_t P_IDESC_NVF4 = idesc_nvf4_ue4m3(2 * BM, BN);
+constexpr uint32_t P_IDESC_BF16 = idesc_bf16_f32(2 * BM, BN);
+static_assert(P_STAGE_BYTES % 1024 == 0 && P_B_BYTES % 1024 == 0, "pair stage alignment");
+static_assert(P_SMEM_BYTES + 1024 + 256 <= 227 * 1024, "pair shared memory budget");
+
+struct PairMaps {
+  CUtensorMap a, b, t[3], l2[3], y;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_gemm_nvfp4_pair(const __grid_constant__ PairMaps maps, const __grid_constant__ GParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sfring = smem + P_STAGES * P_STAGE_BYTES;
+  uint8_t* epi_stage = sfring + SF_SLOTS * SF_SLOT_BYTES;
+  uint64_t* full = (uint64_t*)(smem + P_SMEM_BYTES);  // leader: operand stages of both CTAs
+  uint64_t* empty = full + P_STAGES;                  // both: released by the leader's MMAs
+  uint64_t* acc_full = empty + P_STAGES;              // both [2]
+  uint64_t* acc_empty = acc_full + 2;                 // leader [2]: 8 epilogue warps
+  uint64_t* mma_done = acc_empty + 2;                 // leader
+  uint64_t* sf_ready = mma_done + 1;                  // leader [2]: 8 mover warps
+  uint64_t* sf_free = sf_ready + 2;                   // both [2]
+  uint64_t* sfs_full = sf_free + 2;                   // local [SF_SLOTS]
+  uint64_t* sfs_empty = sfs_full + SF_SLOTS;
+  uint32_t* tmem_slot = (uint32_t*)(sfs_empty + SF_SLOTS);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  WaitCtl wc{abort_flag, p.status, p.limit};
+  const unsigned long long drain_limit = p.limit > (1ull << 24) ? p.limit : (1ull << 24);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);
+      mbar_init(&sf_ready[b], 8);
+      mbar_init(&sf_free[b], 1);
+    }
+    mbar_init(mma_done, 1);
+    for (int b = 0; b < SF_SLOTS; ++b) {
+      mbar_init(&sfs_full[b], 1);
+      mbar_init(&sfs_empty[b], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int units = p.n_lr + p.k_stages;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      prefetch_tmap(&maps.a);
+      prefetch_tmap(&maps.b);
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        const int arow = mt * 2 * BM + (int)rank * BM, brow = nt * BN + (int)rank * PB_ROWS;
+        for (int u = 0; u < units; ++u, ++it) {
+          const int s = it % P_STAGES;
+          if (!mbar_wait_cl(&empty[s], ((it / P_STAGES) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * P_STAGE_BYTES;
+          const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+          if (u < p.n_lr) {
+            const int w = p.lr_w[u], mi = lr_map_index(w);
+            if (leader) mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)(BM + PB_ROWS) * 2 * w);
+            tma_load_2d_pair(&maps.t[mi], fbar, st, p.lr_off[u], arow);
+            tma_load_2d_pair(&maps.l2[mi], fbar, st + A_BYTES, p.lr_off[u], brow);
+          } else {
+            const int ks = u - p.n_lr;
+            if (leader) mbar_arrive_expect_tx(&full[s], 2u * P_STAGE_BYTES);
+            tma_load_2d_pair(&maps.a, fbar, st, ks * 128, arow);
+            tma_load_2d_pair(&maps.b, fbar, st + A_BYTES, ks * 128, brow);
+          }
+        }
+      }
+      if (!ok && leader) {  // drain the copies of both CTAs still in flight
+        for (int j = (it > P_STAGES ? it - P_STAGES : 0); j < it; ++j)
+          mbar_wait_drain(&full[j % P_STAGES], (j / P_STAGES) & 1, drain_limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      int it = 0, local = 0, kst = 0;
+      bool ok = true;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++local) {
+        const int b = local & 1;
+        if (!mbar_wait_cl(&acc_empty[b], ((local >> 1) & 1) ^ 1, wc)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(b * BN);
+        uint32_t accum = 0;
+        for (int u = 0; u < units; ++u, ++it) {
+          const int s = it % P_STAGES;
+          if (!mbar_wait_cl(&full[s], (it / P_STAGES) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * P_STAGE_BYTES);
+          const uint32_t b_addr = a_addr + A_BYTES;
+          if (u < p.n_lr) {
+            const int w = p.lr_w[u];
+            const uint32_t layout = w == 64 ? LAYOUT_SW128 : (w == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
+            const uint32_t sbo = 8u * 2u * (uint32_t)w;  // 8 rows of w bf16
+            for (int kk = 0; kk < w / 16; ++kk) {
+              mma_bf16_pair(d, make_sdesc(a_addr + 32 * kk, 16, sbo, layout),
+                            make_sdesc(b_addr + 32 * kk, 16, sbo, layout), P_IDESC_BF16, accum);
+              accum = 1;
+            }
+          } else {
+            const int sb = kst & 1;
+            if (!mbar_wait_cl(&sf_ready[sb], (kst >> 1) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sfa_t = tmem + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+            const uint32_t sfb_t = sfa_t + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              mma_nvf4_pair(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
+                            make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), P_IDESC_NVF4, sfa_t + 4 * j,
+                            sfb_t + 8 * j, accum);
+              accum = 1;
+            }
+            umma_commit_pair(&sf_free[sb], 3);
+            ++kst;
+          }
+          umma_commit_pair(&empty[s], 3);
+        }
+        if (ok) umma_commit_pair(&acc_full[b], 3);
+      }
+      umma_commit_pair(mma_done, 1);  // every pair MMA issued above has completed when this fires
+      mbar_wait_drain(mma_done, 0, drain_limit);
+    }
+  } else if (warp == SF_WARP) {
+    // ------------------------------------------------------------ scale-factor producer (both CTAs)
+    // This CTA's 128 activation rows (128-row atom tile 2*mt + rank) and all 192
+    // weight rows of the tile.
+    if (lane == 0) {
+      int pit = 0;
+      bool ok = true;
+      const int pairs_k = (p.k_stages + 1) / 2;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        const int at = 2 * mt + (int)rank;
+        for (int j = 0; j < pairs_k; ++j, ++pit) {
+          const int slot = pit % SF_SLOTS;
+          if (!mbar_wait(&sfs_empty[slot], ((pit / SF_SLOTS) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
+          uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
+          mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
+          bulk_load(dst, p.sfa + ((size_t)at * p.katoms + 8 * j) * kSfAtomBytes, ns * SFA_BYTES, &sfs_full[slot]);
+          bulk_load(dst + 2 * SFA_BYTES, p.sfb + ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes, ns * SFB_BYTES,
+                    &sfs_full[slot]);
+        }
+      }
+      if (!ok) {
+        for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
+          mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, drain_limit);
+      }
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ scale-factor movers (both CTAs)
+    // As in the single-CTA kernel; each warp's arrival goes to the leader's barrier.
+    const int q = warp & 3;
+    int kst = 0, pit = 0;
+    bool ok = true;
+    for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+      for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
+        const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
+        const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
+        if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
+        ok = ok && mbar_wait_cl(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+        if (!ok) break;
+        const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
+        const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
+          ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + hh) * kSfAtomBytes + lane * 16);
+            rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
+          }
+        }
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+        tmem_st_32x32b_x16(tq, ra);
+        tmem_st_32x32b_x32(tq + 16, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_cluster(mapa_shared(smem_u32(&sf_ready[sb]), 0));
+          if (last_of_pair) mbar_arrive(&sfs_empty[slot]);  // the slot's atoms are in tensor memory
+        }
+        if (last_of_pair) ++pit;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;  // exact: powers of two
+    const int q = warp & 3;  // tensor-memory lane quarter this warp may access
+    uint8_t* stg = epi_stage + (warp - 2) * 2 * EPI_STAGE_BYTES;
+    const uint32_t empty_cl0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    const uint32_t empty_cl1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    int local = 0, sbuf = 0;
+    for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
+      const int b = local & 1;
+      if (!mbar_wait_cl(&acc_full[b], (local >> 1) & 1, wc)) break;
+      tc_fence_after();
+      const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+      const int m0 = mt * 2 * BM + (int)rank * BM + 32 * q;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 64; ++c) {
+        const int n0 = nt * BN + 64 * c;
+        uint8_t* dst = stg + sbuf * EPI_STAGE_BYTES + lane * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float bb[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int n = n0 + 32 * h + 4 * j;
+            const float4 v = (n < p.N) ? __ldg((const float4*)(p.bias + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            bb[4 * j] = v.x;
+            bb[4 * j + 1] = v.y;
+            bb[4 * j + 2] = v.z;
+            bb[4 * j + 3] = v.w;
+          }
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + 64 * c + 32 * h, r);
+          tmem_ld_wait();
+          if (c == BN / 64 - 1 && h == 1) {  // the whole accumulator is in registers
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(b ? empty_cl1 : empty_cl0);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 16-byte chunk 4h+k of this row, swizzled
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 8 * k + 2 * e;
+              const float y0 = fmaf(__uint_as_float(r[j]), out_scale, bb[j]);
+              const float y1 = fmaf(__uint_as_float(r[j + 1]), out_scale, bb[j + 1]);
+              __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
+              o[e] = *(uint32_t*)&hv;
+            }
+            const int chunk = 4 * h + k;
+            *(uint4*)(dst + ((chunk ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (m0 < p.M && n0 < p.N) {  // boxes wholly past the edge are skipped
+            tma_store_2d(&maps.y, stg + sbuf * EPI_STAGE_BYTES, n0, m0);
+            bulk_commit();
+            bulk_wait_read<1>();  // the other staging buffer is free again
+          } else {
+            bulk_wait_read<0>();  // no store from this buffer: both buffers are free
+          }
+        }
+        __syncwarp();
+        sbuf ^= 1;
+      }
+    }
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  __syncwarp();
+  // Neither CTA leaves (or frees tensor memory) while the pair MMAs, the peer's
+  // remote arrivals or its loads completing on the leader's barriers may still
+  // touch it.
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 int sm_count(int dev) {
   static int cache[64] = {0};
   if (dev < 0 || dev >= 64) return 148;
@@ -380,16 +706,37 @@ int sm_count(int dev) {
   return cache[dev];
 }
 
+// Largest number of co-resident CTA pairs of the pair kernel on a device (0 if
+// the query fails), cached per device.
+int pair_clusters(int dev, size_t smem) {
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (!cache[dev]) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_nvfp4_pair, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = -1;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev] > 0 ? cache[dev] : 0;
+}
+
 }  // namespace
 
 int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w, cudaStream_t stream) {
-  GemmMaps maps;
-  std::memset(&maps, 0, sizeof(maps));
   const int K = (int)L->K, N = (int)L->N, r = L->rank;
-  int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
-                          (uint64_t)K / 2, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != SVDQ_OK) return st;
-  maps.b = L->map_w;
   GParams p{};
   const LowRankChunks ch = lowrank_chunks(r);
   p.n_lr = ch.n;
@@ -397,6 +744,71 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
     p.lr_off[i] = ch.off[i];
     p.lr_w[i] = ch.width[i];
   }
+  p.M = (int)M;
+  p.N = N;
+  p.K = K;
+  p.n_tiles = (N + BN - 1) / BN;
+  p.k_stages = K / kKStage;
+  p.katoms = K / 64;
+  p.sfa = ws + w.scales;
+  p.sfb = L->wscales;
+  p.bias = L->bias;
+  p.Y = (uint16_t*)Y;
+  p.out_scale = L->g_x * L->g_w;
+  p.g_w = L->g_w;
+  p.gx_dev = L->dyn_gx ? (const float*)(ws + w.status + 4) : nullptr;
+  p.status = (int*)(ws + w.status);
+  p.limit = wait_limit_cycles();
+
+  // Token counts above one 128-row tile use the CTA-pair kernel (256-row tiles)
+  // when the device can co-schedule its clusters.
+  const size_t psmem = 1024 + (size_t)P_SMEM_BYTES + 256;
+  if (M > BM) {
+    static int attr_done[64] = {0};
+    const int dev = L->device;
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+      if (cudaFuncSetAttribute(k_gemm_nvfp4_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem) !=
+          cudaSuccess)
+        return SVDQ_ERR_CUDA;
+      attr_done[dev] = 1;
+    }
+    const int maxc = pair_clusters(dev, psmem);
+    if (maxc > 0) {
+      PairMaps maps;
+      std::memset(&maps, 0, sizeof(maps));
+      int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
+                              (uint64_t)K / 2, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (st != SVDQ_OK) return st;
+      maps.b = L->map_w_half;
+      if (r > 0) {
+        const int widths[3] = {64, 32, 16};
+        const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_64B,
+                                           CU_TENSOR_MAP_SWIZZLE_32B};
+        for (int i = 0; i < 3; ++i) {
+          if (widths[i] > r) continue;
+          st = encode_tmap_2d(&maps.t[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.t, (uint64_t)r, (uint64_t)M,
+                              (uint64_t)r * 2, widths[i], BM, swz[i]);
+          if (st != SVDQ_OK) return st;
+          maps.l2[i] = L->map_l2_half[i];
+        }
+      }
+      st = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64,
+                          32, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (st != SVDQ_OK) return st;
+      p.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
+      p.num_tiles = p.m_tiles * p.n_tiles;
+      const int npairs = p.num_tiles < maxc ? p.num_tiles : maxc;
+      k_gemm_nvfp4_pair<<<2 * npairs, THREADS, psmem, stream>>>(maps, p);
+      return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+    }
+  }
+
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  int st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
+                          (uint64_t)K / 2, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != SVDQ_OK) return st;
+  maps.b = L->map_w;
   if (r > 0) {
     const int widths[3] = {64, 32, 16};
     const CUtensorMapSwizzle swz[3] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -409,23 +821,8 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
       maps.l2[i] = L->map_l2[i];
     }
   }
-  p.M = (int)M;
-  p.N = N;
-  p.K = K;
   p.m_tiles = (int)((M + BM - 1) / BM);
-  p.n_tiles = (N + BN - 1) / BN;
   p.num_tiles = p.m_tiles * p.n_tiles;
-  p.k_stages = K / kKStage;
-  p.katoms = K / 64;
-  p.sfa = ws + w.scales;
-  p.sfb = L->wscales;
-  p.bias = L->bias;
-  p.Y = (uint16_t*)Y;
-  p.out_scale = L->g_x * L->g_w;
-  p.g_w = L->g_w;
-  p.gx_dev = L->dyn_gx ? (const float*)(ws + w.status + 4) : nullptr;
-  p.status = (int*)(ws + w.status);
-  p.limit = wait_limit_cycles();
   st = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64, 32,
                       CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != SVDQ_OK) return st;

@@ -73,8 +73,8 @@ Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M) {
   w.codes_bytes = fmt == SVDQ_NVFP4_G16 ? (size_t)M * K / 2 : (size_t)M * K;
   o = align_up(o + w.codes_bytes, kAlign);
   w.scales = o;
-  if (fmt == SVDQ_NVFP4_G16)
-    w.scales_bytes = (size_t)((M + kSfAtomRows - 1) / kSfAtomRows) * (size_t)(K / 64) * kSfAtomBytes;
+  if (fmt == SVDQ_NVFP4_G16)  // whole 256-row tiles: the pair GEMM reads both halves' atoms
+    w.scales_bytes = (size_t)((M + kPairBM - 1) / kPairBM) * 2 * (size_t)(K / 64) * kSfAtomBytes;
   else
     w.scales_bytes = (size_t)(K / 64) * (size_t)int4_scale_ld(M) * 2;
   o = align_up(o + w.scales_bytes, kAlign);
@@ -297,10 +297,13 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   L->wcodes = L->blob + b.wcodes;
   L->wscales = L->blob + b.wscales;
   int e = SVDQ_OK;
-  if (fmt == SVDQ_NVFP4_G16)  // 256 codes (128 B) per row per stage, swizzled for the MMA
+  if (fmt == SVDQ_NVFP4_G16) {  // 256 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
                        (uint64_t)K / 2, 128, kNvfp4BN, CU_TENSOR_MAP_SWIZZLE_128B);
-  else  // 128 E4M3 codes (128 B) per row per stage, swizzled for the MMA
+    if (e == SVDQ_OK)
+      e = encode_tmap_2d(&L->map_w_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
+                         (uint64_t)K / 2, 128, kNvfp4BN / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else  // 128 E4M3 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K, (uint64_t)N, (uint64_t)K,
                        128, kInt4BN, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e == SVDQ_OK && rank > 0) {
@@ -314,6 +317,9 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
       if (widths[i] > rank) continue;
       e = encode_tmap_2d(&L->map_l2[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, (uint64_t)rank, (uint64_t)N,
                          (uint64_t)rank * 2, widths[i], bn, swz[i]);
+      if (e == SVDQ_OK && fmt == SVDQ_NVFP4_G16)
+        e = encode_tmap_2d(&L->map_l2_half[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, (uint64_t)rank,
+                           (uint64_t)N, (uint64_t)rank * 2, widths[i], kNvfp4BN / 2, swz[i]);
     }
   }
   if (e != SVDQ_OK) {
@@ -369,6 +375,7 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!X || ((uintptr_t)X & 15)) return SVDQ_ERR_INVALID_ARG;
+  NvtxRange range("svdq/quantize");
   if (L->dyn_gx) {  // first pass: the tensor's largest |x^|
     const int e = launch_act_amax(L, X, M, (uint8_t*)ws, w, (cudaStream_t)stream);
     if (e != SVDQ_OK) return (svdq_status)e;
@@ -382,6 +389,7 @@ svdq_status svdq_gemm(const svdq_layer* L, int64_t M, void* Y, void* ws, size_t 
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!Y || ((uintptr_t)Y & 15)) return SVDQ_ERR_INVALID_ARG;
+  NvtxRange range("svdq/gemm");
   if (L->fmt == SVDQ_NVFP4_G16) return (svdq_status)launch_gemm_nvfp4(L, M, Y, (uint8_t*)ws, w, (cudaStream_t)stream);
   return (svdq_status)launch_gemm_int4(L, M, Y, (uint8_t*)ws, w, nullptr, (cudaStream_t)stream);
 }
@@ -391,6 +399,37 @@ svdq_status svdq_forward(const svdq_layer* L, const void* X, int64_t M, void* Y,
   svdq_status st = svdq_quantize_act(L, X, M, ws, ws_bytes, stream);
   if (st != SVDQ_OK) return st;
   return svdq_gemm(L, M, Y, ws, ws_bytes, stream);
+}
+
+svdq_status svdq_mlp_fusable(const svdq_layer* up, const svdq_layer* down) {
+  return (svdq_status)fused_mlp_supported(up, down);
+}
+
+svdq_status svdq_gemm_gelu_quantize(const svdq_layer* up, const svdq_layer* down, int64_t M, void* ws_up,
+                                    size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* H, void* stream) {
+  Workspace wu, wd;
+  svdq_status st = check_ws(up, M, ws_up, ws_up_bytes, &wu);
+  if (st != SVDQ_OK) return st;
+  st = check_ws(down, M, ws_dn, ws_dn_bytes, &wd);
+  if (st != SVDQ_OK) return st;
+  st = (svdq_status)fused_mlp_supported(up, down);
+  if (st != SVDQ_OK) return st;
+  if (M == 0) return SVDQ_OK;
+  if (H && ((uintptr_t)H & 15)) return SVDQ_ERR_INVALID_ARG;
+  NvtxRange range("svdq/gemm_gelu_quantize");
+  return (svdq_status)launch_gemm_gelu_quant(up, down, M, (uint8_t*)ws_up, wu, (uint8_t*)ws_dn, wd, H,
+                                             (cudaStream_t)stream);
+}
+
+svdq_status svdq_mlp_forward(const svdq_layer* up, const svdq_layer* down, const void* X, int64_t M, void* Y,
+                             void* ws_up, size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* stream) {
+  svdq_status st = (svdq_status)fused_mlp_supported(up, down);
+  if (st != SVDQ_OK) return st;
+  st = svdq_quantize_act(up, X, M, ws_up, ws_up_bytes, stream);
+  if (st != SVDQ_OK) return st;
+  st = svdq_gemm_gelu_quantize(up, down, M, ws_up, ws_up_bytes, ws_dn, ws_dn_bytes, nullptr, stream);
+  if (st != SVDQ_OK) return st;
+  return svdq_gemm(down, M, Y, ws_dn, ws_dn_bytes, stream);
 }
 
 svdq_status svdq_int4_group_acc(const svdq_layer* L, int64_t M, void* ws, size_t ws_bytes, int32_t* acc,
@@ -404,6 +443,10 @@ svdq_status svdq_int4_group_acc(const svdq_layer* L, int64_t M, void* ws, size_t
 }
 
 svdq_status svdq_read_status(const svdq_layer* L, int64_t M, const void* ws, size_t ws_bytes, int* device_status) {
+  if (!ws && ws_bytes == 0) {  // the fixed scratch of svdq_forward_noalloc
+    if (!device_status) return SVDQ_ERR_INVALID_ARG;
+    return (svdq_status)read_status_noalloc(L, M, device_status);
+  }
   Workspace w;
   svdq_status st = check_ws(L, M, ws, ws_bytes, &w);
   if (st != SVDQ_OK) return st;

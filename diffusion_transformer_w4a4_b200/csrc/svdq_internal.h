@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstddef>
 #include <cstdint>
@@ -16,6 +17,7 @@ namespace svdq {
 constexpr int kKStage = 256;       // K elements per pipeline stage / per quantizer chunk
 constexpr int kGemmBM = 128;       // GEMM tile rows (tokens), = tcgen05 M
 constexpr int kNvfp4BN = 192;      // NVFP4 GEMM tile columns (output features)
+constexpr int kPairBM = 256;       // NVFP4 CTA-pair GEMM tile rows (128 per CTA)
 constexpr int kInt4BN = 128;       // INT4 GEMM tile columns
 constexpr int kSfAtomRows = 128;   // rows per tensor-core scale-factor atom
 constexpr int kSfAtomBytes = 512;  // 128 rows x 4 blocks of 16
@@ -27,6 +29,16 @@ constexpr size_t kAlign = 1024;
 constexpr int kAmaxSlots = 1024;  // per-CTA maxima of the dynamic activation-scale pass
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// NVTX range around the host-side enqueue of a kernel group ("svdq/quantize",
+// "svdq/gemm", ...), so a timeline tool can attribute the launches; without a
+// tool attached the calls do nothing.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Byte offset of the E4M3 scale of (row, block) in a scale-factor atom tiling
 // whose row tiles are `tile_rows` rows (128 for activations, 192 for weights)
@@ -101,6 +113,10 @@ struct svdq_layer {
   CUtensorMap map_w;         // weight codes
   CUtensorMap map_l1;        // L1^T, box {64, rank}, 128B swizzle (quantizer)
   CUtensorMap map_l2[3];     // L2^T chunks of width 64/32/16
+  // NVFP4, CTA-pair GEMM: each CTA of a pair loads half of a 192-row weight
+  // tile (96 rows) of the codes and of the L2^T chunks
+  CUtensorMap map_w_half;
+  CUtensorMap map_l2_half[3];
 };
 
 namespace svdq {
@@ -136,5 +152,12 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
                       cudaStream_t stream);
 int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w, int32_t* acc_dbg,
                      cudaStream_t stream);
+// MLP pair fusion: the up layer's GEMM whose epilogue writes the down layer's
+// quantized input (GELU between them) into the down layer's workspace
+int fused_mlp_supported(const svdq_layer* up, const svdq_layer* down);
+int launch_gemm_gelu_quant(const svdq_layer* up, const svdq_layer* down, int64_t M, uint8_t* ws_up,
+                           const Workspace& w_up, uint8_t* ws_dn, const Workspace& w_dn, void* H, cudaStream_t stream);
+// status word of the last svdq_forward_noalloc on the current device (M tokens)
+int read_status_noalloc(const svdq_layer* L, int64_t M, int* device_status);
 
 }  // namespace svdq

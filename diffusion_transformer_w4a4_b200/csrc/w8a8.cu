@@ -448,6 +448,7 @@ svdq_status svdq_w8a8_quantize_act(const svdq_w8a8_layer* L, const void* X, int6
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!X || ((uintptr_t)X & 15)) return SVDQ_ERR_INVALID_ARG;
+  NvtxRange range("svdq/w8a8_quantize");
   return (svdq_status)launch_w8_quantize(L, X, M, (uint8_t*)ws, (cudaStream_t)stream);
 }
 
@@ -456,6 +457,7 @@ svdq_status svdq_w8a8_gemm(const svdq_w8a8_layer* L, int64_t M, void* Y, void* w
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!Y || ((uintptr_t)Y & 15)) return SVDQ_ERR_INVALID_ARG;
+  NvtxRange range("svdq/w8a8_gemm");
   return (svdq_status)launch_w8_gemm(L, M, Y, (uint8_t*)ws, (cudaStream_t)stream);
 }
 

@@ -197,8 +197,42 @@ svdq_status svdq_gemm(const svdq_layer* layer, int64_t M, void* Y, void* ws, siz
 svdq_status svdq_int4_group_acc(const svdq_layer* layer, int64_t M, void* ws, size_t ws_bytes, int32_t* acc,
                                 void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* Cross-layer fusion of a transformer block's MLP pair: up -> GELU -> down. */
+/* ------------------------------------------------------------------------ */
+/* "Hugging Face встроила Nunchaku в Diffusers ..." (paragraph on Nunchaku
+ * Lite): the engine's speed comes from fused, model-specific kernels.  Here the
+ * up-projection's GEMM epilogue computes, per output element,
+ *     h = bf16(y_up),   x' = bf16(GELU(h)),   GELU(h) = h/2 (1 + erf(h/sqrt 2)) in binary32,
+ * and quantizes x' as the down-projection's input exactly as svdq_quantize_act
+ * would (x^' = f32(x') inv_lambda', E4M3 block scales and E2M1 codes under the
+ * down layer's static g_x', t' = bf16(bf16(x^') L1')), writing codes, scales and
+ * t' into the down layer's workspace; y_up itself is never written.
+ * Requirements (else SVDQ_ERR_INVALID_ARG): both layers NVFP4, up.N == down.K,
+ * up.N a multiple of 192, the down layer's activation scale static (g_x != 0)
+ * and its rank <= 32, both layers on the current device. */
+svdq_status svdq_mlp_fusable(const svdq_layer* up, const svdq_layer* down);
+
+/* After svdq_quantize_act(up, X, M, ws_up, ...): the fused up-projection GEMM.
+ * ws_up / ws_dn are the two layers' workspaces for M tokens (device, 256-byte
+ * aligned; ws_dn initialised once with svdq_workspace_init); H, if not NULL, is
+ * a device bf16 [M, up.N] array (16-byte aligned) that receives x' (a parity
+ * export; costs one extra write).  Then svdq_gemm(down, M, Y, ws_dn, ...) gives
+ * the block's MLP output.  Asynchronous on `stream`; device-side errors land in
+ * ws_up's status word. */
+svdq_status svdq_gemm_gelu_quantize(const svdq_layer* up, const svdq_layer* down, int64_t M, void* ws_up,
+                                    size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* H, void* stream);
+
+/* Y[M, down.N] = down(GELU(up(X))): svdq_quantize_act(up), svdq_gemm_gelu_quantize,
+ * svdq_gemm(down), all on `stream`. */
+svdq_status svdq_mlp_forward(const svdq_layer* up, const svdq_layer* down, const void* X, int64_t M, void* Y,
+                             void* ws_up, size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* stream);
+
 /* Synchronously read the workspace status word (0 = fine, else an svdq_status
- * recorded by a kernel). */
+ * recorded by a kernel).  With ws == NULL and ws_bytes == 0 it reads instead the
+ * status word of the last svdq_forward_noalloc call for M tokens on the current
+ * device (which must be the layer's); that word is zeroed by the next such
+ * call, so read it after the call's work has finished and before the next one. */
 svdq_status svdq_read_status(const svdq_layer* layer, int64_t M, const void* ws, size_t ws_bytes,
                              int* device_status);
 
@@ -218,7 +252,10 @@ svdq_status svdq_read_status(const svdq_layer* layer, int64_t M, const void* ws,
  * the array keeps the last call's contents otherwise.  All calls share the
  * array: calls whose GPU work can overlap (other streams, other threads) race
  * and must be serialized by the caller.  Allocates nothing (no cudaMalloc,
- * cudaFree or allocating library routine); asynchronous like svdq_forward. */
+ * cudaFree or allocating library routine); asynchronous like svdq_forward.
+ * Device-side failures (an in-kernel wait past its limit) are read with
+ * svdq_read_status(layer, M, NULL, 0, &status).  A failed address lookup is
+ * not cached: the next call tries again.  M > 2^30 returns INVALID_ARG. */
 svdq_status svdq_forward_noalloc(const svdq_layer* layer, const void* X, int64_t M, void* Y, void* stream);
 
 /* Upper bound, in SM clock cycles, on every in-kernel wait of later launches
