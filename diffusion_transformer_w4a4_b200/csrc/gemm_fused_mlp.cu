@@ -2,7 +2,7 @@
 // quantizer fused into its epilogue (cross-layer fusion of the MLP pair).
 //
 //   h  = bf16( g_x g_w [ sum_blocks (s_x s_w)(qx . qw) + t . L2/(g_x g_w) ] + b )   (the up layer's y)
-//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) in binary32
+//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) = h/2 erfc(-h / sqrt 2) in binary32
 //   x^' = f32(x') * inv_lambda'                                                     (the down layer's input)
 //   codes', E4M3 block scales'  of x^' (blocks of 16, static g_x'),  t' = bf16( bf16(x^') . L1' )
 //
@@ -20,14 +20,14 @@
 // quantizer does for its K slices.
 //
 // Same main loop as the CTA-pair NVFP4 GEMM (k_gemm_nvfp4_pair: 256 x 192 tile,
-// cta_group::2, no multicast loads).  Roles per CTA (512 threads):
+// cta_group::2, no multicast loads; scale factors copied into tensor memory by
+// the leader with tcgen05.cp.cta_group::2).  Roles per CTA (384 threads):
 //   warp 0      operand TMA producer            warp 1   tensor memory, main MMAs (leader)
 //   warps 2-9   epilogue: two warps per tensor-memory lane quarter, 96 columns each
-//   warps 10-13 scale-factor movers             warp 14  scale-factor producer
-//   warp 15     L1'^T slice loader and t' MMA issuer (leader), per tile
-// Tensor memory (512 columns): two 192-column accumulators, two 48-column
-// scale-factor buffers, and the 32-column t' accumulator, so the down layer's
-// rank is at most 32.  Every wait is bounded; no load uses cluster multicast.
+//   warp 10     scale-factor producer           warp 11  L1'^T slices and t' MMAs (leader)
+// Tensor memory: two 192-column accumulators, one 48-column scale-factor
+// buffer and the 32-column t' accumulator, so the down layer's rank is at most
+// 32.  Every wait is bounded; no load uses cluster multicast.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -52,11 +52,12 @@ constexpr int SF_SLOT_BYTES = 2 * (SFA_BYTES + SFB_BYTES);
 constexpr int XT_BYTES = 3 * BM * 128;    // bf16 x^' tile: three 64-column halves, 128B-swizzled
 constexpr int L1_MAX_ROWS = 16;           // rank/2 rows of L1'^T per CTA (rank <= 32)
 constexpr int L1_BYTES = 3 * L1_MAX_ROWS * 128;
-constexpr int THREADS = 512;
+constexpr int THREADS = 384;
+constexpr int SF_WARP = 10, T_WARP = 11;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 2 * BN;
 constexpr uint32_t SF_BUF_COLS = 48;
-constexpr uint32_t TP_COL = SF_COL + 2 * SF_BUF_COLS;  // 480
+constexpr uint32_t TP_COL = SF_COL + SF_BUF_COLS;  // 432
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + XT_BYTES + L1_BYTES;
 constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(2 * BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(2 * BM, BN);
@@ -65,8 +66,12 @@ static_assert(SMEM_BYTES + 1024 + 512 <= 227 * 1024, "shared memory budget");
 static_assert(TP_COL + 32 <= TMEM_COLS, "tensor memory budget");
 
 struct FusedMaps {
-  CUtensorMap a, b, t[3], l2[3], l1dn;
+  CUtensorMap a, b, t[3], l2[3], l1dn, sfa, sfb;
 };
+
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 
 struct FParams {
   int M, N, K, m_tiles, n_tiles, num_units, S, k_stages, katoms;
@@ -138,10 +143,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + STAGES;              // both [2]
   uint64_t* acc_empty = acc_full + 2;               // leader [2]: 16 epilogue warps
   uint64_t* mma_done = acc_empty + 2;               // leader
-  uint64_t* sf_ready = mma_done + 1;                // leader [2]: 8 movers
-  uint64_t* sf_free = sf_ready + 2;                 // both [2]
-  uint64_t* sfs_full = sf_free + 2;                 // local [SF_SLOTS]
-  uint64_t* sfs_empty = sfs_full + SF_SLOTS;        // local
+  uint64_t* sfs_full = mma_done + 1;                // leader [SF_SLOTS]: both CTAs' atoms
+  uint64_t* sfs_empty = sfs_full + SF_SLOTS;        // both: released by the leader's MMAs
   uint64_t* l1_full = sfs_empty + SF_SLOTS;         // leader: both CTAs' L1' slices
   uint64_t* xt_full = l1_full + 1;                  // leader: 16 epilogue warps
   uint64_t* xt_free = xt_full + 1;                  // both: t' MMAs of the tile done (x^' tile and L1' slot free)
@@ -169,13 +172,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 16);
-      mbar_init(&sf_ready[b], 8);
-      mbar_init(&sf_free[b], 1);
     }
     mbar_init(mma_done, 1);
     for (int b = 0; b < SF_SLOTS; ++b) {
       mbar_init(&sfs_full[b], 1);
-      mbar_init(&sfs_empty[b], 4);
+      mbar_init(&sfs_empty[b], 1);
     }
     mbar_init(l1_full, 1);
     mbar_init(xt_full, 16);
@@ -237,7 +238,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ main MMA issuer (leader)
     if (leader && lane == 0) {
-      int it = 0, local = 0, kst = 0;
+      int it = 0, local = 0, pit = 0;
       bool ok = true;
       for (int u = pair; u < p.num_units && ok; u += npairs) {
         const int sg = u / p.m_tiles;
@@ -253,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           uint32_t accum = 0;
           for (int st = 0; st < units; ++st, ++it) {
             const int s = it % STAGES;
-            if (!mbar_wait_cl(&full[s], (it / STAGES) & 1, wc)) {
+            if (!mbar_wait(&full[s], (it / STAGES) & 1, wc)) {
               ok = false;
               break;
             }
@@ -270,14 +271,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 accum = 1;
               }
             } else {
-              const int sb = kst & 1;
-              if (!mbar_wait_cl(&sf_ready[sb], (kst >> 1) & 1, wc)) {
+              // the stage's scale-factor atoms into tensor memory ahead of the MMAs
+              // that read them (the pipe keeps this thread's copies and MMAs in order)
+              const int ks = st - p.n_lr, h = ks & 1, slot = pit % SF_SLOTS;
+              const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
+              if (h == 0 && !mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              const uint32_t sfa_t = tmem + SF_COL + (uint32_t)sb * SF_BUF_COLS;
-              const uint32_t sfb_t = sfa_t + 16;
+              const uint32_t sfa_s = smem_u32(sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES);
+              const uint32_t sfb_s = smem_u32(sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES);
+              const uint32_t sfa_t = tmem + SF_COL, sfb_t = sfa_t + 16;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                tmem_cp_32x128b_x4_pair(sfa_t + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+                tmem_cp_32x128b_x4_pair(sfb_t + 8 * j, make_sdesc(sfb_s + 2 * j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+                tmem_cp_32x128b_x4_pair(sfb_t + 8 * j + 4,
+                                        make_sdesc(sfb_s + (2 * j + 1) * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              }
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 mma_nvf4_pair(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
@@ -285,8 +297,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                               sfb_t + 8 * j, accum);
                 accum = 1;
               }
-              umma_commit_pair(&sf_free[sb], 3);
-              ++kst;
+              if (last_of_pair) {
+                umma_commit_pair(&sfs_empty[slot], 3);
+                ++pit;
+              }
             }
             umma_commit_pair(&empty[s], 3);
           }
@@ -296,9 +310,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       umma_commit_pair(mma_done, 1);
       mbar_wait_drain(mma_done, 0, drain_limit);
     }
-  } else if (warp == 14) {
+  } else if (warp == SF_WARP) {
     // ------------------------------------------------------------ scale-factor producer (both CTAs)
+    // Two K stages per slot: this CTA's 128 activation rows (atom tile 2 mt +
+    // rank) and all 192 weight rows; both CTAs' copies complete on the leader's barrier.
     if (lane == 0) {
+      prefetch_tmap(&maps.sfa);
+      prefetch_tmap(&maps.sfb);
       int pit = 0;
       bool ok = true;
       const int pairs_k = (p.k_stages + 1) / 2;
@@ -315,61 +333,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
             uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
-            mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
-            bulk_load(dst, p.sfa + ((size_t)at * p.katoms + 8 * j) * kSfAtomBytes, ns * SFA_BYTES, &sfs_full[slot]);
-            bulk_load(dst + 2 * SFA_BYTES, p.sfb + ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes,
-                      ns * SFB_BYTES, &sfs_full[slot]);
+            const uint32_t fbar = mapa_shared(smem_u32(&sfs_full[slot]), 0);
+            if (leader) mbar_arrive_expect_tx(&sfs_full[slot], 2u * (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
+            for (int h = 0; h < ns; ++h) {
+              tma_load_2d_pair(&maps.sfa, fbar, dst + h * SFA_BYTES, 0, at * p.katoms + 8 * j + 4 * h);
+              tma_load_2d_pair(&maps.sfb, fbar, dst + 2 * SFA_BYTES + h * SFB_BYTES, 0,
+                               (nt * p.katoms + 8 * j + 4 * h) * 2);
+            }
           }
         }
       }
-      if (!ok) {
+      if (!ok && leader) {
         for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
           mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, drain_limit);
       }
     }
-  } else if (warp >= 10 && warp <= 13) {
-    // ------------------------------------------------------------ scale-factor movers (both CTAs)
-    const int q = warp & 3;
-    int kst = 0, pit = 0;
-    bool ok = true;
-    for (int u = pair; u < p.num_units && ok; u += npairs) {
-      const int sg = u / p.m_tiles;
-      const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
-      for (int nt = nt0; nt < nt1 && ok; ++nt) {
-        for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
-          const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
-          const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
-          if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
-          ok = ok && mbar_wait_cl(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
-          if (!ok) break;
-          const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
-          const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
-          uint32_t ra[16], rb[32];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
-            ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + hh) * kSfAtomBytes + lane * 16);
-              rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
-            }
-          }
-          const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
-          tmem_st_32x32b_x16(tq, ra);
-          tmem_st_32x32b_x32(tq + 16, rb);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_cluster(mapa_shared(smem_u32(&sf_ready[sb]), 0));
-            if (last_of_pair) mbar_arrive(&sfs_empty[slot]);
-          }
-          if (last_of_pair) ++pit;
-        }
-      }
-    }
-  } else if (warp == 15) {
+  } else if (warp == T_WARP) {
     // ------------------------------------------------------------ L1'^T slices and t' MMAs
     // Per tile: this CTA's rank/2 rows of L1'^T for the tile's 192 columns (three
     // 64-column boxes, 128-byte swizzle) into its slot; the leader then issues
@@ -484,8 +463,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // the up layer's bf16 output, GELU in binary32, rounded to bf16 (the down layer's input)
             const float h0 = bf16_round(fmaf(__uint_as_float(r[2 * j]), out_scale, bb[2 * j]));
             const float h1 = bf16_round(fmaf(__uint_as_float(r[2 * j + 1]), out_scale, bb[2 * j + 1]));
-            const float g0 = 0.5f * h0 * (1.0f + erff(h0 * 0.70710678118654752f));
-            const float g1 = 0.5f * h1 * (1.0f + erff(h1 * 0.70710678118654752f));
+            // 1 + erf(h / sqrt 2) = erfc(-h / sqrt 2): no cancellation for negative h
+            const float g0 = 0.5f * h0 * erfcf(-h0 * 0.70710678118654752f);
+            const float g1 = 0.5f * h1 * erfcf(-h1 * 0.70710678118654752f);
             const __nv_bfloat162 gh = __floats2bfloat162_rn(g0, g1);
             hbits[j] = *(const uint32_t*)&gh;
             v[j] = __fmul2_rn(__bfloat1622float2(gh), make_float2(il[2 * j], il[2 * j + 1]));
@@ -674,6 +654,14 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
                         (uint64_t)D->K * 2, 64, (uint32_t)rd / 2, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SVDQ_OK) return st;
   }
+  // scale-factor atoms (512 B each) as rows of 128 u32 (see k_gemm_nvfp4_pair)
+  st = encode_tmap_2d(&maps.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, ws + w.scales, 128,
+                      (uint64_t)((M + 2 * BM - 1) / (2 * BM)) * 2 * (K / 64), kSfAtomBytes, 128, 4,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != SVDQ_OK) return st;
+  st = encode_tmap_2d(&maps.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, L->wscales, 128,
+                      (uint64_t)((N + BN - 1) / BN) * (K / 64) * 2, kSfAtomBytes, 128, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != SVDQ_OK) return st;
   p.M = (int)M;
   p.N = N;
   p.K = K;

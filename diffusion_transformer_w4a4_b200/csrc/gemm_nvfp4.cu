@@ -377,16 +377,20 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
 // halves -- no multicast), and the pair MMA reads the B halves of both CTAs.
 // Per SM and per 256-deep K stage that is 16 KiB of activation codes and
 // 12 KiB of weight codes for the same tensor work as the single-CTA tile's
-// 16 + 24 KiB.  Each CTA keeps the E4M3 scale factors of its own 128 rows and
-// of all 192 weight rows in its tensor memory (the pair MMA reads both).
-// Only CTA 0 ("leader") issues MMAs; its operand barriers count the bytes of
-// both CTAs' loads, and it waits for both CTAs' scale-factor movers and
-// epilogues.  Its MMA completions are signalled to the same barrier in both
-// CTAs (multicast commit).
+// 16 + 24 KiB.  Each CTA stages the E4M3 scale-factor atoms of its own 128
+// rows and of all 192 weight rows; the leader copies them into both CTAs'
+// tensor memory with tcgen05.cp.cta_group::2 in the tensor pipe, in order with
+// the MMAs that read them, so the scale factors need no cross-CTA handshake of
+// their own.  Only CTA 0 ("leader") issues tensor-core work; its barriers count
+// the bytes of both CTAs' loads and the arrivals of both CTAs' epilogues, and
+// its completions are signalled to the same barrier in both CTAs.
 constexpr int PB_ROWS = BN / 2;              // 96 weight rows per CTA
 constexpr int P_STAGES = 6;
 constexpr int P_B_BYTES = PB_ROWS * 128;     // 12 KiB
 constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES;
+constexpr int P_THREADS = 224;               // warps: 0 operands, 1 MMA, 2-5 epilogue, 6 scale factors
+constexpr int P_SF_WARP = 6;
+constexpr uint32_t P_SF_COL = 2 * BN;        // one 48-column scale-factor buffer
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + 4 * 2 * EPI_STAGE_BYTES;
 constexpr uint32_t P_IDESC_NVF4 = idesc_nvf4_ue4m3(2 * BM, BN);
 constexpr uint32_t P_IDESC_BF16 = idesc_bf16_f32(2 * BM, BN);
@@ -394,10 +398,14 @@ static_assert(P_STAGE_BYTES % 1024 == 0 && P_B_BYTES % 1024 == 0, "pair stage al
 static_assert(P_SMEM_BYTES + 1024 + 256 <= 227 * 1024, "pair shared memory budget");
 
 struct PairMaps {
-  CUtensorMap a, b, t[3], l2[3], y;
+  CUtensorMap a, b, t[3], l2[3], y, sfa, sfb;  // sfa/sfb: scale-factor atoms as rows of 128 u32
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     k_gemm_nvfp4_pair(const __grid_constant__ PairMaps maps, const __grid_constant__ GParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -408,10 +416,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + P_STAGES;              // both [2]
   uint64_t* acc_empty = acc_full + 2;                 // leader [2]: 8 epilogue warps
   uint64_t* mma_done = acc_empty + 2;                 // leader
-  uint64_t* sf_ready = mma_done + 1;                  // leader [2]: 8 mover warps
-  uint64_t* sf_free = sf_ready + 2;                   // both [2]
-  uint64_t* sfs_full = sf_free + 2;                   // local [SF_SLOTS]
-  uint64_t* sfs_empty = sfs_full + SF_SLOTS;
+  uint64_t* sfs_full = mma_done + 1;                  // leader [SF_SLOTS]: both CTAs' atoms
+  uint64_t* sfs_empty = sfs_full + SF_SLOTS;          // both: released by the leader's MMAs
   uint32_t* tmem_slot = (uint32_t*)(sfs_empty + SF_SLOTS);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -430,13 +436,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 8);
-      mbar_init(&sf_ready[b], 8);
-      mbar_init(&sf_free[b], 1);
     }
     mbar_init(mma_done, 1);
     for (int b = 0; b < SF_SLOTS; ++b) {
       mbar_init(&sfs_full[b], 1);
-      mbar_init(&sfs_empty[b], 4);
+      mbar_init(&sfs_empty[b], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -463,7 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int arow = mt * 2 * BM + (int)rank * BM, brow = nt * BN + (int)rank * PB_ROWS;
         for (int u = 0; u < units; ++u, ++it) {
           const int s = it % P_STAGES;
-          if (!mbar_wait_cl(&empty[s], ((it / P_STAGES) & 1) ^ 1, wc)) {
+          if (!mbar_wait(&empty[s], ((it / P_STAGES) & 1) ^ 1, wc)) {
             ok = false;
             break;
           }
@@ -490,7 +494,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (leader && lane == 0) {
-      int it = 0, local = 0, kst = 0;
+      int it = 0, local = 0, pit = 0;
       bool ok = true;
       for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++local) {
         const int b = local & 1;
@@ -500,7 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint32_t accum = 0;
         for (int u = 0; u < units; ++u, ++it) {
           const int s = it % P_STAGES;
-          if (!mbar_wait_cl(&full[s], (it / P_STAGES) & 1, wc)) {
+          if (!mbar_wait(&full[s], (it / P_STAGES) & 1, wc)) {
             ok = false;
             break;
           }
@@ -517,14 +521,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               accum = 1;
             }
           } else {
-            const int sb = kst & 1;
-            if (!mbar_wait_cl(&sf_ready[sb], (kst >> 1) & 1, wc)) {
+            // this stage's scale-factor atoms into tensor memory, in the tensor
+            // pipe ahead of the MMAs that read them (one buffer: the pipe keeps
+            // this thread's copies and MMAs in order)
+            const int ks = u - p.n_lr, h = ks & 1, slot = pit % SF_SLOTS;
+            const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
+            if (h == 0 && !mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t sfa_t = tmem + SF_COL + (uint32_t)sb * SF_BUF_COLS;
-            const uint32_t sfb_t = sfa_t + 16;
+            const uint32_t sfa_s = smem_u32(sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES);
+            const uint32_t sfb_s = smem_u32(sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES);
+            const uint32_t sfa_t = tmem + P_SF_COL, sfb_t = sfa_t + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tmem_cp_32x128b_x4_pair(sfa_t + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4_pair(sfb_t + 8 * j, make_sdesc(sfb_s + 2 * j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+              tmem_cp_32x128b_x4_pair(sfb_t + 8 * j + 4,
+                                      make_sdesc(sfb_s + (2 * j + 1) * kSfAtomBytes, 0, 128, LAYOUT_NONE));
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               mma_nvf4_pair(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
@@ -532,8 +548,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                             sfb_t + 8 * j, accum);
               accum = 1;
             }
-            umma_commit_pair(&sf_free[sb], 3);
-            ++kst;
+            if (last_of_pair) {  // the slot's atoms are read once these MMAs complete
+              umma_commit_pair(&sfs_empty[slot], 3);
+              ++pit;
+            }
           }
           umma_commit_pair(&empty[s], 3);
         }
@@ -542,11 +560,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       umma_commit_pair(mma_done, 1);  // every pair MMA issued above has completed when this fires
       mbar_wait_drain(mma_done, 0, drain_limit);
     }
-  } else if (warp == SF_WARP) {
+  } else if (warp == P_SF_WARP) {
     // ------------------------------------------------------------ scale-factor producer (both CTAs)
-    // This CTA's 128 activation rows (128-row atom tile 2*mt + rank) and all 192
-    // weight rows of the tile.
+    // Two K stages per slot: [SFA 2j | SFA 2j+1 | SFB 2j | SFB 2j+1], this CTA's
+    // 128 activation rows (atom tile 2 mt + rank) and all 192 weight rows; the
+    // copies of both CTAs complete on the leader's barrier.
     if (lane == 0) {
+      prefetch_tmap(&maps.sfa);
+      prefetch_tmap(&maps.sfb);
       int pit = 0;
       bool ok = true;
       const int pairs_k = (p.k_stages + 1) / 2;
@@ -561,54 +582,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
           uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
-          mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
-          bulk_load(dst, p.sfa + ((size_t)at * p.katoms + 8 * j) * kSfAtomBytes, ns * SFA_BYTES, &sfs_full[slot]);
-          bulk_load(dst + 2 * SFA_BYTES, p.sfb + ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes, ns * SFB_BYTES,
-                    &sfs_full[slot]);
-        }
-      }
-      if (!ok) {
-        for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
-          mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, drain_limit);
-      }
-    }
-  } else if (warp >= 6) {
-    // ------------------------------------------------------------ scale-factor movers (both CTAs)
-    // As in the single-CTA kernel; each warp's arrival goes to the leader's barrier.
-    const int q = warp & 3;
-    int kst = 0, pit = 0;
-    bool ok = true;
-    for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
-      for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
-        const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
-        const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
-        if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
-        ok = ok && mbar_wait_cl(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
-        if (!ok) break;
-        const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
-        const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
-        uint32_t ra[16], rb[32];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
-          ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + hh) * kSfAtomBytes + lane * 16);
-            rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
+          const uint32_t fbar = mapa_shared(smem_u32(&sfs_full[slot]), 0);
+          if (leader) mbar_arrive_expect_tx(&sfs_full[slot], 2u * (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
+          for (int h = 0; h < ns; ++h) {
+            tma_load_2d_pair(&maps.sfa, fbar, dst + h * SFA_BYTES, 0, at * p.katoms + 8 * j + 4 * h);
+            tma_load_2d_pair(&maps.sfb, fbar, dst + 2 * SFA_BYTES + h * SFB_BYTES, 0,
+                             (nt * p.katoms + 8 * j + 4 * h) * 2);
           }
         }
-        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
-        tmem_st_32x32b_x16(tq, ra);
-        tmem_st_32x32b_x32(tq + 16, rb);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_cluster(mapa_shared(smem_u32(&sf_ready[sb]), 0));
-          if (last_of_pair) mbar_arrive(&sfs_empty[slot]);  // the slot's atoms are in tensor memory
-        }
-        if (last_of_pair) ++pit;
+      }
+      if (!ok && leader) {
+        for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
+          mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, drain_limit);
       }
     }
   } else {
@@ -621,7 +606,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     int local = 0, sbuf = 0;
     for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
       const int b = local & 1;
-      if (!mbar_wait_cl(&acc_full[b], (local >> 1) & 1, wc)) break;
+      if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) break;
       tc_fence_after();
       const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
       const int m0 = mt * 2 * BM + (int)rank * BM + 32 * q;
@@ -719,7 +704,7 @@ int pair_clusters(int dev, size_t smem) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * 74, 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.blockDim = dim3(P_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -795,10 +780,20 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
       st = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2, 64,
                           32, CU_TENSOR_MAP_SWIZZLE_128B);
       if (st != SVDQ_OK) return st;
+      // scale-factor atoms (512 B each) as rows of 128 u32: 4 k-atoms (one K
+      // stage) per activation load, 8 per weight load (two atoms per k-atom)
+      const uint64_t sfa_rows = (uint64_t)((M + 2 * BM - 1) / (2 * BM)) * 2 * (K / 64);
+      const uint64_t sfb_rows = (uint64_t)((N + BN - 1) / BN) * (K / 64) * 2;
+      st = encode_tmap_2d(&maps.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, ws + w.scales, 128, sfa_rows, kSfAtomBytes, 128, 4,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != SVDQ_OK) return st;
+      st = encode_tmap_2d(&maps.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, L->wscales, 128, sfb_rows, kSfAtomBytes, 128, 8,
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != SVDQ_OK) return st;
       p.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
       p.num_tiles = p.m_tiles * p.n_tiles;
       const int npairs = p.num_tiles < maxc ? p.num_tiles : maxc;
-      k_gemm_nvfp4_pair<<<2 * npairs, THREADS, psmem, stream>>>(maps, p);
+      k_gemm_nvfp4_pair<<<2 * npairs, P_THREADS, psmem, stream>>>(maps, p);
       return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
     }
   }

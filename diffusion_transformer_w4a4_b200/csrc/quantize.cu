@@ -8,21 +8,24 @@
 // t = bf16( bf16(x^) L1 ) with fp32 accumulation.
 //
 // Work split: a CTA owns 128 token rows and one slice of K (the K range is cut
-// into enough slices that about one CTA per SM is in flight).  Per 128-column
+// into enough slices that about one CTA per SM is in flight).  Per 256-column
 // chunk, with C quantizing warps (16, or 8 for ranks above 80):
-//   warp C      TMA: the X tile [128 x 128], and a bulk copy of the chunk's
-//               128 entries of 1/lambda, into a ring that the quantizing warps
-//               release as soon as they have read it;
-//   warp C+2    TMA: the matching L1^T slice [rank x 128] (two 64-column boxes,
-//               128-byte swizzle) into a small ring released by the MMAs;
-//   warps 0..C-1 quantize 128/C rows each (a lane holds 16 consecutive
-//               elements: one NVFP4 block, or a quarter of a 64-element INT4
-//               group whose maximum takes two warp shuffles; products in packed
-//               f32x2), store codes and scales, and write bf16(x^) into a
-//               128-byte-swizzled K-major tile;
-//   warp C+1    issues tcgen05.mma kind::f16 (M = 128 tokens, N = rank, K = 16)
+//   warps 0..C-1 load their rows of the chunk straight from global memory into
+//               registers (16 lanes cover a row's 512-byte run, so a load
+//               instruction reads two whole runs; the 1/lambda entries come from
+//               the L2-resident weight blob), then quantize them: a lane holds
+//               16 consecutive elements (one NVFP4 block, or a quarter of a
+//               64-element INT4 group whose maximum takes two warp shuffles;
+//               products in packed f32x2), stores codes and scales, and writes
+//               bf16(x^) into a 128-byte-swizzled K-major tile;
+//   warp C+1    TMA: the matching L1^T slice [rank x 256] (four 64-column
+//               boxes, 128-byte swizzle) into a small ring released by the MMAs;
+//   warp C      issues tcgen05.mma kind::f16 (M = 128 tokens, N = rank, K = 16)
 //               on that tile and the L1^T slice, accumulating the slice's part of
 //               t in tensor memory.
+// Loading through registers rather than a TMA ring keeps one independent stream
+// per warp in flight (measured on the FLUX MLP shapes: 16 warp streams of
+// 512-byte runs read X at about 4.1 TB/s, one TMA ring per SM at about 3.6 TB/s).
 // At the end the slice's fp32 partial of t leaves tensor memory; the last CTA of
 // a row block to finish (arrival counter) adds the slices in a fixed order and
 // writes bf16 t, so the result does not depend on scheduling.  HBM traffic is
@@ -37,31 +40,26 @@ namespace svdq {
 namespace {
 
 constexpr int kRows = kQRows;    // 128
-constexpr int kChunk = kQChunk;  // 128
+constexpr int kChunk = kQChunk;  // 256
 // Quantizing warps per CTA: 16 (8 rows each) where the registers allow it, 8
 // (16 rows each) for ranks above 80, whose fp32 partial of t takes a register per
-// rank column; the three role warps follow them.
+// rank column; the two role warps follow them.
 template <int RANK>
 struct Roles {
   static constexpr int kConsumerWarps = RANK <= 80 ? 16 : 8;
   static constexpr int kRowsPerWarp = 128 / kConsumerWarps;
-  static constexpr int kTmaWarp = kConsumerWarps;
-  static constexpr int kMmaWarp = kConsumerWarps + 1;
-  static constexpr int kL1Warp = kConsumerWarps + 2;
-  static constexpr int kThreads = (kConsumerWarps + 3) * 32;
+  static constexpr int kMmaWarp = kConsumerWarps;
+  static constexpr int kL1Warp = kConsumerWarps + 1;
+  static constexpr int kThreads = (kConsumerWarps + 2) * 32;
 };
-constexpr int kXTileBytes = kRows * kChunk * 2;  // 32 KiB
-constexpr int kIlBytes = kChunk * 4;              // the chunk's 1/lambda slice
-constexpr int kXStageBytes = kXTileBytes + kIlBytes;
-// the X ring, padded so the 128-byte-swizzled tiles after it stay 1024-aligned
-__host__ __device__ constexpr int xring_bytes(int xs) { return (xs * kXStageBytes + 1023) & ~1023; }
-constexpr int kAHalfBytes = kRows * 128;         // 64 bf16 columns, 128B-swizzled
-constexpr int kATileBytes = 2 * kAHalfBytes;     // 32 KiB
+constexpr int kABlockBytes = kRows * 128;       // 64 bf16 columns, 128B-swizzled
+constexpr int kATileBytes = (kChunk / 64) * kABlockBytes;  // 64 KiB
 constexpr int kSmemBudget = 220 * 1024;
 
 struct QParams {
-  int M, K, xstages, lstages, nslices, nch, katoms;
+  int M, K, lstages, nslices, nch, katoms;
   int64_t sld;  // INT4: row stride of the fp16 [K/64, sld] scales
+  const uint16_t* x;  // [M, K] bf16
   const float* inv_lambda;
   float g, inv_g, den;  // NVFP4 per-tensor scale, its exact inverse, 6*g
   // dynamic per-tensor scale: the first pass's per-CTA maxima of |x^| (else null),
@@ -78,7 +76,9 @@ struct QParams {
   unsigned long long limit;
 };
 
-__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+// eight floats (as four pairs, element order a.x a.y b.x b.y ...) -> eight E2M1
+// codes, element 2i in the low nibble of byte i
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
   uint32_t out;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -87,7 +87,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
       "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(out)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
   return out;
 }
 
@@ -144,24 +144,21 @@ __device__ __forceinline__ float nvfp4_tensor_scale_dev(float amax) {
 
 template <int FMT, int RANK>
 __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
-    k_quantize(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_l1, QParams p) {
+    k_quantize(const __grid_constant__ CUtensorMap map_l1, QParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int kConsumerWarps = Roles<RANK>::kConsumerWarps, kTmaWarp = Roles<RANK>::kTmaWarp;
+  constexpr int kConsumerWarps = Roles<RANK>::kConsumerWarps;
   constexpr int kMmaWarp = Roles<RANK>::kMmaWarp, kL1Warp = Roles<RANK>::kL1Warp, kThreads = Roles<RANK>::kThreads;
   constexpr int kRowsPerWarp = Roles<RANK>::kRowsPerWarp;
-  const int XS = p.xstages, LS = p.lstages;
-  constexpr int kL1Bytes = RANK * kChunk * 2;  // two boxes of RANK rows x 128 B
-  uint8_t* xring = smem;                          // [XS][X tile | 1/lambda slice]
-  uint8_t* atile = xring + xring_bytes(XS);       // [2][kATileBytes] when RANK > 0 (1024-aligned)
+  const int LS = p.lstages;
+  constexpr int kL1Bytes = RANK * kChunk * 2;  // kChunk/64 boxes of RANK rows x 128 B
+  uint8_t* atile = smem;                                      // [2][kATileBytes] when RANK > 0
   uint8_t* lring = atile + (RANK > 0 ? 2 * kATileBytes : 0);  // [LS][kL1Bytes]
-  float* rtab = (float*)(lring + LS * kL1Bytes);  // [128] 1/e4m3
-  uint64_t* full_x = (uint64_t*)(rtab + 128);
-  uint64_t* empty_x = full_x + XS;
-  uint64_t* full_l = empty_x + XS;
-  uint64_t* empty_l = full_l + LS;
-  uint64_t* xready = empty_l + LS;  // [2]
-  uint64_t* xfree = xready + 2;     // [2]
+  float* rtab = (float*)(lring + LS * kL1Bytes);              // [128] 1/e4m3
+  uint64_t* full_l = (uint64_t*)(rtab + 128);
+  uint64_t* empty_l = full_l + 2;
+  uint64_t* xready = empty_l + 2;  // [2]
+  uint64_t* xfree = xready + 2;    // [2]
   uint64_t* tdone = xfree + 2;
   uint32_t* tmem_slot = (uint32_t*)(tdone + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
@@ -177,10 +174,6 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
   WaitCtl wc{abort_flag, p.status, p.limit};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < XS; ++s) {
-      mbar_init(&full_x[s], 1);
-      mbar_init(&empty_x[s], kConsumerWarps);
-    }
     for (int s = 0; s < LS; ++s) {
       mbar_init(&full_l[s], 1);
       mbar_init(&empty_l[s], 1);
@@ -208,7 +201,7 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
   // NVFP4 per-tensor scale: the prepared static one, or the dynamic one from the
   // first pass's maxima (then t is stored as t / g_x, an exact power-of-two
   // scaling, because the packed L2 carries only 1/g_w)
-  float gs = p.g, inv_gs = p.inv_g, dens = p.den, tsc = 1.f;
+  float inv_gs = p.inv_g, dens = p.den, tsc = 1.f;
   if (FMT == SVDQ_NVFP4_G16 && p.amax_slots != nullptr) {
     __shared__ float dred[kThreads / 32];
     float m = 0.f;
@@ -220,33 +213,14 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
     m = dred[0];
 #pragma unroll
     for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, dred[i]);
-    gs = nvfp4_tensor_scale_dev(m);
+    const float gs = nvfp4_tensor_scale_dev(m);
     inv_gs = 1.0f / gs;  // exact: a power of two
     dens = 6.0f * gs;
     tsc = inv_gs;
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.g_out = gs;
   }
 
-  if (warp == kTmaWarp) {
-    // ------------------------------------------------------------ X producer
-    if (lane == 0) {
-      prefetch_tmap(&map_x);
-      int issued = 0;
-      for (int i = 0; i < nchunks; ++i) {
-        const int s = i % XS;
-        if (!mbar_wait(&empty_x[s], ((i / XS) & 1) ^ 1, wc)) break;
-        uint8_t* dst = xring + s * kXStageBytes;
-        mbar_arrive_expect_tx(&full_x[s], kXStageBytes);
-        tma_load_2d(&map_x, &full_x[s], dst, (c_begin + i) * kChunk, m0);
-        bulk_load(dst + kXTileBytes, p.inv_lambda + (size_t)(c_begin + i) * kChunk, kIlBytes, &full_x[s]);
-        issued = i + 1;
-      }
-      if (*abort_flag) {  // drain copies that are still in flight before leaving
-        for (int i = (issued > XS ? issued - XS : 0); i < issued; ++i)
-          mbar_wait_drain(&full_x[i % XS], (i / XS) & 1, p.limit);
-      }
-    }
-  } else if (warp == kL1Warp) {
+  if (warp == kL1Warp) {
     // ------------------------------------------------------------ L1^T producer
     if constexpr (RANK > 0) {
       if (lane == 0) {
@@ -258,8 +232,8 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
           const int k0 = (c_begin + i) * kChunk;
           uint8_t* dst = lring + s * kL1Bytes;
           mbar_arrive_expect_tx(&full_l[s], kL1Bytes);
-          tma_load_2d(&map_l1, &full_l[s], dst, k0, 0);
-          tma_load_2d(&map_l1, &full_l[s], dst + RANK * 128, k0 + 64, 0);
+#pragma unroll
+          for (int h = 0; h < kChunk / 64; ++h) tma_load_2d(&map_l1, &full_l[s], dst + h * RANK * 128, k0 + 64 * h, 0);
           issued = i + 1;
         }
         if (*abort_flag) {
@@ -284,7 +258,7 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kChunk / 16; ++kk) {
             const uint32_t h = kk >> 2, koff = (kk & 3) * 32;
-            mma_bf16(tmem, make_sdesc(a_addr + h * kAHalfBytes + koff, 16, 1024, LAYOUT_SW128),
+            mma_bf16(tmem, make_sdesc(a_addr + h * kABlockBytes + koff, 16, 1024, LAYOUT_SW128),
                      make_sdesc(b_addr + h * RANK * 128 + koff, 16, 1024, LAYOUT_SW128), idesc,
                      (i > 0 || kk > 0) ? 1u : 0u);
           }
@@ -297,114 +271,129 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ quantizing warps
-    const int rsub = lane >> 3;  // row within the warp's 4-row step
-    const int j = lane & 7;      // 16-column group within the chunk
-    const int K2 = p.K / 2;
+    // A lane owns 16 consecutive columns (one NVFP4 block, a quarter of an INT4
+    // group) of two rows... of the warp's rows: 16 lanes cover a row's 256-column
+    // chunk, so a warp reads two rows (two 512-byte runs) per load instruction.
+    // Each warp loads its rows of a chunk straight from global memory into
+    // registers (no staging), then quantizes them.
+    const int rsub = lane >> 4;  // row within the warp's 2-row step
+    const int j = lane & 15;     // 16-column block within the chunk
+    constexpr int ITS = kRowsPerWarp / 2;
+    // Row step `it` handles row rbase + 2 it.  Its code, scale and x^-tile
+    // offsets are affine in `it` (a warp's rows stay inside one 32-row group of
+    // the scale-factor atom), so only the step-0 values are kept.
+    const int rbase = warp * kRowsPerWarp + rsub;
+    const int64_t mbase = m0 + rbase;
+    const int kk0 = c_begin * kChunk + 16 * j;
+    const size_t code_row = FMT == SVDQ_NVFP4_G16 ? (size_t)p.K / 2 : (size_t)p.K;
+    const size_t coff0 = (size_t)mbase * code_row + (FMT == SVDQ_NVFP4_G16 ? kk0 / 2 : kk0);
+    const size_t soff0 = FMT == SVDQ_NVFP4_G16 ? sf_offset(mbase, kk0 / 16, p.katoms, kSfAtomRows)
+                                               : ((size_t)(kk0 / 64) * p.sld + mbase) * 2;
+    constexpr int kScaleRowStep = FMT == SVDQ_NVFP4_G16 ? 2 * 16 : 2 * 2;  // bytes per 2 rows
+    const int c0 = 2 * (j & 3);
+    const int ablk = (j >> 2) * kABlockBytes;
+    const float* ilp = p.inv_lambda + kk0;
+    constexpr size_t kCodeStep = FMT == SVDQ_NVFP4_G16 ? kChunk / 2 : kChunk;
+    const size_t scale_step = FMT == SVDQ_NVFP4_G16 ? (kChunk / 64) * kSfAtomBytes : (kChunk / 32) * (size_t)p.sld;
     for (int i = 0; i < nchunks; ++i) {
-      const int s = i % XS, buf = i & 1;
-      bool ok = mbar_wait(&full_x[s], (i / XS) & 1, wc);
-      if constexpr (RANK > 0) ok = ok && mbar_wait(&xfree[buf], ((i >> 1) & 1) ^ 1, wc);
+      const int buf = i & 1;
+      // this chunk's rows and 1/lambda, straight into registers (rows past M read row 0)
+      uint4 xr[ITS][2];
+#pragma unroll
+      for (int it = 0; it < ITS; ++it) {
+        const int64_t m = mbase + 2 * it;
+        const int64_t mr = m < p.M ? m : 0;  // rows past M read row 0 (never stored)
+        const uint4* src = (const uint4*)(p.x + (size_t)mr * p.K + kk0 + (size_t)i * kChunk);
+        xr[it][0] = __ldcs(src);
+        xr[it][1] = __ldcs(src + 1);
+      }
+      float2 il[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 t4 = __ldg((const float4*)(ilp + (size_t)i * kChunk) + q);
+        il[2 * q] = make_float2(t4.x, t4.y);
+        il[2 * q + 1] = make_float2(t4.z, t4.w);
+      }
+      bool ok = true;
+      if constexpr (RANK > 0) ok = mbar_wait(&xfree[buf], ((i >> 1) & 1) ^ 1, wc);
       if (ok) {
-        const uint8_t* st = xring + s * kXStageBytes;
-        const int k0 = (c_begin + i) * kChunk;
-        const int kk0 = k0 + 16 * j;
-        float il[16];
-        const float4* ils = (const float4*)(st + kXTileBytes) + 4 * j;  // staged with the X tile
+        uint8_t* at = atile + buf * kATileBytes;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 t4 = ils[q];
-          il[4 * q] = t4.x;
-          il[4 * q + 1] = t4.y;
-          il[4 * q + 2] = t4.z;
-          il[4 * q + 3] = t4.w;
-        }
-        uint8_t* at = atile + buf * kATileBytes + (j >> 2) * kAHalfBytes;
-#pragma unroll 2
-        for (int it = 0; it < kRowsPerWarp / 4; ++it) {
-          const int row = warp * kRowsPerWarp + 4 * it + rsub;
-          const int m = m0 + row;
-          const uint4 r0 = *(const uint4*)(st + row * (kChunk * 2) + 32 * j);
-          const uint4 r1 = *(const uint4*)(st + row * (kChunk * 2) + 32 * j + 16);
-          const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-          float v[16];
+        for (int it = 0; it < ITS; ++it) {
+          const uint32_t w[8] = {xr[it][0].x, xr[it][0].y, xr[it][0].z, xr[it][0].w,
+                                 xr[it][1].x, xr[it][1].y, xr[it][1].z, xr[it][1].w};
+          float2 v[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            v[2 * e] = __uint_as_float(w[e] << 16);
-            v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-            mul2(v[2 * e], v[2 * e + 1], il[2 * e], il[2 * e + 1]);
-          }
-          float amax = 0.f;
+          for (int e = 0; e < 8; ++e)
+            v[e] = __fmul2_rn(make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)), il[e]);
+          float mx[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(v[e]));
-          uint2 packed = make_uint2(0u, 0u);
+          for (int e = 0; e < 8; ++e) mx[e] = fmaxf(fabsf(v[e].x), fabsf(v[e].y));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mx[e] = fmaxf(mx[e], mx[e + 4]);
+          float amax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+          const bool live = mbase + 2 * it < p.M;
+          const size_t cbyte = coff0 + 2 * it * code_row + (size_t)i * kCodeStep;
+          const size_t sbyte = soff0 + it * kScaleRowStep + (size_t)i * scale_step;
           if (FMT == SVDQ_NVFP4_G16) {
             const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, dens));
-            if (sb != 0) {
-              // 1 / (e4m3(sb) * g) exactly: g is a power of two
-              const float inv = rtab[sb] * inv_gs;
-              float q0[8], q1[8];
+            // 1 / (e4m3(sb) * g) exactly (g is a power of two); 0 for sb = 0
+            const float inv = rtab[sb] * inv_gs;
+            const float2 inv2 = make_float2(inv, inv);
+            float2 q[8];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                q0[2 * e] = v[2 * e];
-                q0[2 * e + 1] = v[2 * e + 1];
-                q1[2 * e] = v[8 + 2 * e];
-                q1[2 * e + 1] = v[9 + 2 * e];
-                mul2(q0[2 * e], q0[2 * e + 1], inv, inv);
-                mul2(q1[2 * e], q1[2 * e + 1], inv, inv);
-              }
-              packed = make_uint2(cvt_e2m1x8(q0), cvt_e2m1x8(q1));
-            }
+            for (int e = 0; e < 8; ++e) q[e] = __fmul2_rn(v[e], inv2);
+            uint2 packed = make_uint2(cvt_e2m1x8(q[0], q[1], q[2], q[3]), cvt_e2m1x8(q[4], q[5], q[6], q[7]));
+            if (sb == 0) packed = make_uint2(0u, 0u);  // a zero block scale: all codes +0
             const int base = lane & ~3;  // 4 lanes = 64 columns = one scale-factor atom word
             const uint32_t s1 = __shfl_sync(0xffffffffu, sb, base + 1);
             const uint32_t s2 = __shfl_sync(0xffffffffu, sb, base + 2);
             const uint32_t s3 = __shfl_sync(0xffffffffu, sb, base + 3);
-            if ((lane & 3) == 0 && m < p.M)
-              *(uint32_t*)(p.scales + sf_offset(m, kk0 / 16, p.katoms, kSfAtomRows)) =
-                  sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            if ((lane & 3) == 0 && live) *(uint32_t*)(p.scales + sbyte) = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            if (live) *(uint2*)(p.codes + cbyte) = packed;
           } else {
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             const __half s16 = __float2half_rn(__fdiv_rn(amax, 7.0f));
             const float S16 = __half2float(s16);
-            uint32_t qb[4] = {0u, 0u, 0u, 0u};
-            if (S16 != 0.f) {
-              const float inv = __frcp_rn(S16);
+            // a zero scale gives inv = 0: every product is +-0 and rounds to the code +0
+            const float inv = S16 != 0.f ? __frcp_rn(S16) : 0.f;
+            const float2 inv2 = make_float2(inv, inv);
+            const float2 magic = make_float2(12582912.0f, 12582912.0f), nmagic = make_float2(-12582912.0f, -12582912.0f);
+            uint32_t qb[4];
 #pragma unroll
-              for (int e = 0; e < 16; e += 2) {
-                float y0 = v[e], y1 = v[e + 1];
-                mul2(y0, y1, inv, inv);
-                // clamp, then round half to even: (y + 1.5 * 2^23) - 1.5 * 2^23
-                // is the nearest integer (a +0 for codes of zero), and E4M3
-                // holds every integer of [-8, 7] exactly
-                y0 = fminf(fmaxf(y0, -8.0f), 7.0f);
-                y1 = fminf(fmaxf(y1, -8.0f), 7.0f);
-                y0 = __fsub_rn(__fadd_rn(y0, 12582912.0f), 12582912.0f);
-                y1 = __fsub_rn(__fadd_rn(y1, 12582912.0f), 12582912.0f);
-                qb[e >> 2] |= cvt_e4m3x2(y0, y1) << (8 * (e & 2));
-              }
+            for (int e = 0; e < 8; e += 2) {
+              float2 y0 = __fmul2_rn(v[e], inv2), y1 = __fmul2_rn(v[e + 1], inv2);
+              // clamp, then round half to even: (y + 1.5 * 2^23) - 1.5 * 2^23
+              // is the nearest integer (a +0 for codes of zero), and E4M3
+              // holds every integer of [-8, 7] exactly
+              y0 = make_float2(fminf(fmaxf(y0.x, -8.0f), 7.0f), fminf(fmaxf(y0.y, -8.0f), 7.0f));
+              y1 = make_float2(fminf(fmaxf(y1.x, -8.0f), 7.0f), fminf(fmaxf(y1.y, -8.0f), 7.0f));
+              y0 = __fadd2_rn(__fadd2_rn(y0, magic), nmagic);
+              y1 = __fadd2_rn(__fadd2_rn(y1, magic), nmagic);
+              qb[e >> 1] = cvt_e4m3x2(y0.x, y0.y) | (cvt_e4m3x2(y1.x, y1.y) << 16);
             }
-            if ((lane & 3) == 0 && m < p.M) ((__half*)p.scales)[(size_t)(kk0 / 64) * p.sld + m] = s16;
-            if (m < p.M) *(uint4*)(p.codes + (size_t)m * p.K + kk0) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
+            if ((lane & 3) == 0 && live) *(__half*)(p.scales + sbyte) = s16;
+            if (live) *(uint4*)(p.codes + cbyte) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
           }
-          if (FMT == SVDQ_NVFP4_G16 && m < p.M) *(uint2*)(p.codes + (size_t)m * K2 + kk0 / 2) = packed;
           if constexpr (RANK > 0) {
             uint32_t b[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+              __nv_bfloat162 h = __float22bfloat162_rn(v[e]);
               b[e] = *(uint32_t*)&h;
             }
-            const int c0 = 2 * (j & 3);
-            *(uint4*)(at + row * 128 + ((c0 ^ (row & 7)) << 4)) = make_uint4(b[0], b[1], b[2], b[3]);
-            *(uint4*)(at + row * 128 + (((c0 + 1) ^ (row & 7)) << 4)) = make_uint4(b[4], b[5], b[6], b[7]);
+            const int row = rbase + 2 * it;
+            uint8_t* arow = at + ablk + row * 128;
+            *(uint4*)(arow + ((c0 ^ (row & 7)) << 4)) = make_uint4(b[0], b[1], b[2], b[3]);
+            *(uint4*)(arow + (((c0 + 1) ^ (row & 7)) << 4)) = make_uint4(b[4], b[5], b[6], b[7]);
           }
         }
       }
-      if constexpr (RANK > 0) fence_proxy_async_smem();  // x^ tile -> tensor core
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&empty_x[s]);  // the X tile has been read
-        if constexpr (RANK > 0) mbar_arrive(&xready[buf]);
+      if constexpr (RANK > 0) {
+        fence_proxy_async_smem();  // x^ tile -> tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xready[buf]);
       }
     }
 
@@ -486,36 +475,31 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
 }
 
 template <int FMT, int RANK>
-int launch_rank(const CUtensorMap& mx, const CUtensorMap& ml1, const QParams& p, int64_t M, cudaStream_t stream) {
+int launch_rank(const CUtensorMap& ml1, const QParams& p, int64_t M, cudaStream_t stream) {
   constexpr int kL1Bytes = RANK * kChunk * 2;
-  constexpr int kFixed = (RANK > 0 ? 2 * kATileBytes : 0) + 512 + 512;
   QParams q = p;
-  q.lstages = RANK > 0 ? (RANK <= 64 ? 3 : 2) : 0;
-  int XS = 5;
-  while (XS > 2 && xring_bytes(XS) + kFixed + q.lstages * kL1Bytes > kSmemBudget) --XS;
-  q.xstages = XS;
-  const size_t smem = 1024 + (size_t)xring_bytes(XS) + (size_t)q.lstages * kL1Bytes + kFixed;
+  q.lstages = RANK == 0 ? 0 : (2 * kATileBytes + 2 * kL1Bytes + 2048 <= kSmemBudget ? 2 : 1);
+  const size_t smem = 1024 + (RANK > 0 ? 2 * (size_t)kATileBytes : 0) + (size_t)q.lstages * kL1Bytes + 512 + 256;
   auto kern = k_quantize<FMT, RANK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   const dim3 grid((unsigned)((M + kRows - 1) / kRows), (unsigned)p.nslices);
-  kern<<<grid, Roles<RANK>::kThreads, smem, stream>>>(mx, ml1, q);
+  kern<<<grid, Roles<RANK>::kThreads, smem, stream>>>(ml1, q);
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
 template <int FMT>
-int launch_fmt(const CUtensorMap& mx, const CUtensorMap& ml1, const QParams& p, int64_t M, int rank,
-               cudaStream_t stream) {
+int launch_fmt(const CUtensorMap& ml1, const QParams& p, int64_t M, int rank, cudaStream_t stream) {
   switch (rank) {
-    case 0: return launch_rank<FMT, 0>(mx, ml1, p, M, stream);
-    case 16: return launch_rank<FMT, 16>(mx, ml1, p, M, stream);
-    case 32: return launch_rank<FMT, 32>(mx, ml1, p, M, stream);
-    case 48: return launch_rank<FMT, 48>(mx, ml1, p, M, stream);
-    case 64: return launch_rank<FMT, 64>(mx, ml1, p, M, stream);
-    case 80: return launch_rank<FMT, 80>(mx, ml1, p, M, stream);
-    case 96: return launch_rank<FMT, 96>(mx, ml1, p, M, stream);
-    case 112: return launch_rank<FMT, 112>(mx, ml1, p, M, stream);
-    case 128: return launch_rank<FMT, 128>(mx, ml1, p, M, stream);
+    case 0: return launch_rank<FMT, 0>(ml1, p, M, stream);
+    case 16: return launch_rank<FMT, 16>(ml1, p, M, stream);
+    case 32: return launch_rank<FMT, 32>(ml1, p, M, stream);
+    case 48: return launch_rank<FMT, 48>(ml1, p, M, stream);
+    case 64: return launch_rank<FMT, 64>(ml1, p, M, stream);
+    case 80: return launch_rank<FMT, 80>(ml1, p, M, stream);
+    case 96: return launch_rank<FMT, 96>(ml1, p, M, stream);
+    case 112: return launch_rank<FMT, 112>(ml1, p, M, stream);
+    case 128: return launch_rank<FMT, 128>(ml1, p, M, stream);
     default: return SVDQ_ERR_INVALID_ARG;
   }
 }
@@ -524,10 +508,6 @@ int launch_fmt(const CUtensorMap& mx, const CUtensorMap& ml1, const QParams& p, 
 
 int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, const Workspace& w,
                     cudaStream_t stream) {
-  CUtensorMap mx;
-  int st = encode_tmap_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)L->K, (uint64_t)M,
-                          (uint64_t)L->K * 2, kChunk, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (st != SVDQ_OK) return st;
   QParams p{};
   p.M = (int)M;
   p.K = (int)L->K;
@@ -535,6 +515,7 @@ int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, 
   p.nslices = w.nslices;
   p.katoms = (int)(L->K / 64);
   p.sld = int4_scale_ld(M);
+  p.x = (const uint16_t*)X;
   p.inv_lambda = L->inv_lambda;
   p.g = L->g_x;
   p.inv_g = 1.0f / L->g_x;  // exact: g_x is a power of two
@@ -554,8 +535,8 @@ int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, 
   p.status = (int*)(ws + w.status);
   p.counters = (int*)(ws + w.status + 16);
   p.limit = wait_limit_cycles();
-  if (L->fmt == SVDQ_NVFP4_G16) return launch_fmt<SVDQ_NVFP4_G16>(mx, L->map_l1, p, M, L->rank, stream);
-  return launch_fmt<SVDQ_INT4_G64>(mx, L->map_l1, p, M, L->rank, stream);
+  if (L->fmt == SVDQ_NVFP4_G16) return launch_fmt<SVDQ_NVFP4_G16>(L->map_l1, p, M, L->rank, stream);
+  return launch_fmt<SVDQ_INT4_G64>(L->map_l1, p, M, L->rank, stream);
 }
 
 }  // namespace svdq

@@ -23,7 +23,7 @@ constexpr int kSfAtomRows = 128;   // rows per tensor-core scale-factor atom
 constexpr int kSfAtomBytes = 512;  // 128 rows x 4 blocks of 16
 constexpr int kMaxRank = 128;
 constexpr int kQRows = 128;   // activation quantizer: token rows per CTA (= tcgen05 M)
-constexpr int kQChunk = 128;  // activation quantizer: K columns per pipeline chunk
+constexpr int kQChunk = 256;  // activation quantizer: K columns per chunk
 constexpr int kQSmCount = 148;  // SM count the quantizer's K-split is sized for (fixed, so sizes are device-free)
 constexpr size_t kAlign = 1024;
 constexpr int kAmaxSlots = 1024;  // per-CTA maxima of the dynamic activation-scale pass

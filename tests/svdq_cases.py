@@ -100,6 +100,34 @@ def assert_y_close(y_gpu_bits, y_orc_bits, act=None, prep=None):
     return s
 
 
+def check_layer_output(gl, X, prep, y, rows=None):
+    """Parity of one svdq_w4a4 forward whose workspace still holds its quantized
+    activations: codes and scales bit-exact on every row; the GPU's t within its
+    summation bound (assert_t_close); Y on `rows` (all by default) within the
+    stated gate given the GPU's own t (the low-rank input teacher-forced: a t
+    one bf16 ulp away from the oracle's, which its own gate allows, moves y by
+    that ulp times L2, more than 2e-2 where |t| is large); and the fully
+    independent oracle output (its own t) within rel-L2 1e-3, its statistics
+    reported."""
+    M = X.shape[0]
+    got = gl.read_act(M)
+    ref = oracle.quantize_act(X, prep)
+    if "g_x" in got and prep["fmt"] == oracle.NVFP4:
+        assert got["g_x"] == ref["g_x"], (got["g_x"], ref["g_x"])
+    np.testing.assert_array_equal(got["codes"], ref["codes"])
+    np.testing.assert_array_equal(got["scales"], ref["scales"])
+    st = assert_t_close(got["t"], ref["t"], ref, prep) if prep["rank"] else {}
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
+    taught = dict(sub, t=got["t"][rows])
+    s = assert_y_close(y[rows], oracle.forward_from_act(taught, prep), taught, prep)
+    ind = y_stats(y[rows], oracle.forward_from_act(sub, prep))
+    assert ind["rel_l2"] <= REL_L2, ind
+    s.update(indep_rel_l2=ind["rel_l2"], indep_max_abs=ind["max_abs"], indep_n_over_abs_ulp=ind["n_over_abs_ulp"])
+    s.update(st)
+    return s
+
+
 def tile_rows(M, seed, spread=40, tile=128):
     """Sampled output rows: one seeded row inside every 128-row M tile (the ragged
     last tile included), the first/last rows of the first two tiles and of the

@@ -12,9 +12,10 @@ are calibrated on the inputs of the dense bf16 chain from the same x0.  Token
 rows never mix in this chain, so the oracle's free-running chain can be run on
 the sampled rows alone; its drift from the GPU chain is reported, not gated.
 
-Bar per layer: activation codes and scales bit-exact on all rows, t within its
-derived bound, bf16 Y on sampled rows within rel-L2 1e-3 and the elementwise
-bound of svdq_cases."""
+Bar per layer (svdq_cases.check_layer_output): activation codes and scales
+bit-exact on all rows, t within its derived bound, bf16 Y on sampled rows (one
+in every 128-row tile) within rel-L2 1e-3 and |dy| <= 2e-2 + 1 bf16 ulp given
+the GPU's t, and the fully independent oracle output within rel-L2 1e-3."""
 import functools
 
 import numpy as np
@@ -22,7 +23,7 @@ import pytest
 
 import oracle
 import workloads as wl
-from svdq_cases import GpuLayer, assert_t_close, assert_y_close, tile_rows
+from svdq_cases import GpuLayer, check_layer_output, tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -54,14 +55,7 @@ def _check_layer(gl, X, prep, rows):
     M = X.shape[0]
     y = gl.forward(X)
     assert gl.status(M) == 0
-    got = gl.read_act(M)
-    ref = oracle.quantize_act(X, prep)
-    np.testing.assert_array_equal(got["codes"], ref["codes"])
-    np.testing.assert_array_equal(got["scales"], ref["scales"])
-    st = assert_t_close(got["t"], ref["t"], ref, prep)
-    sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
-    sy = assert_y_close(y[rows], oracle.forward_from_act(sub, prep), sub, prep)
-    return y, dict(sy, **st)
+    return y, check_layer_output(gl, X, prep, y, rows)
 
 
 @functools.lru_cache(maxsize=1)

@@ -9,7 +9,7 @@ import pytest
 
 import oracle
 import workloads as wl
-from svdq_cases import GpuLayer, assert_t_close, assert_y_close, oracle_layer, tile_rows, y_stats
+from svdq_cases import GpuLayer, assert_t_close, check_layer_output, oracle_layer, tile_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -55,8 +55,7 @@ def test_forward_nvfp4(M, K, N, rank):
     gl = GpuLayer(prep)
     y = gl.forward(X)
     assert gl.status(M) == 0
-    act = oracle.quantize_act(X, prep)
-    assert_y_close(y, oracle.forward_from_act(act, prep), act, prep)
+    print(M, K, N, rank, check_layer_output(gl, X, prep, y))
 
 
 def test_forward_empty_and_reuse():
@@ -82,18 +81,8 @@ def test_flux_workloads_nvfp4(name):
     M = layer.M
     y = gl.forward(X)
     assert gl.status(M) == 0
-    # every quantized activation, bit-exact (t within one ulp)
-    got = gl.read_act(M)
-    ref = oracle.quantize_act(X, prep)
-    np.testing.assert_array_equal(got["codes"], ref["codes"])
-    np.testing.assert_array_equal(got["scales"], ref["scales"])
-    st = assert_t_close(got["t"], ref["t"], ref, prep)
-    # sampled output rows: first/last tile rows and a seeded spread
-    rows = tile_rows(M, 1)
-    sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
-    y_ref = oracle.forward_from_act(sub, prep)
-    s = assert_y_close(y[rows], y_ref, sub, prep)
-    print(name, s, st)
+    # every quantized activation bit-exact, t within its bound, sampled output rows
+    print(name, check_layer_output(gl, X, prep, y, tile_rows(M, 1)))
 
 
 def test_wait_timeout_reports_status():
@@ -117,8 +106,7 @@ def test_wait_timeout_reports_status():
     svdq.svdq_workspace_init(gl.lin.handle, 512, gl.lin.workspace(512))
     y = gl.forward(X)
     assert gl.status(512) == 0
-    act = oracle.quantize_act(X, prep)
-    assert_y_close(y, oracle.forward_from_act(act, prep), act, prep)
+    check_layer_output(gl, X, prep, y)
 
 
 @pytest.mark.parametrize("M,K,N,rank", [(128, 256, 128, 0), (128, 256, 128, 16), (300, 1024, 576, 32),
@@ -129,8 +117,7 @@ def test_forward_int4(M, K, N, rank):
     gl = GpuLayer(prep)
     y = gl.forward(X)
     assert gl.status(M) == 0
-    act = oracle.quantize_act(X, prep)
-    assert_y_close(y, oracle.forward_from_act(act, prep), act, prep)
+    print(M, K, N, rank, check_layer_output(gl, X, prep, y))
 
 
 @pytest.mark.parametrize("M,K,N", [(128, 256, 128), (300, 512, 400), (64, 1024, 256)])
@@ -162,12 +149,4 @@ def test_flux_workloads_int4(name):
     M = layer.M
     y = gl.forward(X)
     assert gl.status(M) == 0
-    got = gl.read_act(M)
-    ref = oracle.quantize_act(X, prep)
-    np.testing.assert_array_equal(got["codes"], ref["codes"])
-    np.testing.assert_array_equal(got["scales"], ref["scales"])
-    st = assert_t_close(got["t"], ref["t"], ref, prep)
-    rows = tile_rows(M, 2)
-    sub = {k: (v[rows] if np.ndim(v) else v) for k, v in ref.items()}
-    s = assert_y_close(y[rows], oracle.forward_from_act(sub, prep), sub, prep)
-    print(name, s, st)
+    print(name, check_layer_output(gl, X, prep, y, tile_rows(M, 2)))
