@@ -17,7 +17,9 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+# SVDQ_LIBRARY=debug selects the bounds-checked debug variant (libsvdq_debug.so,
+# built by build.build(debug=True)); the default is the release library.
+LIB_PATH = os.path.join(_HERE, "libsvdq_debug.so" if os.environ.get("SVDQ_LIBRARY") == "debug" else "libsvdq.so")
 
 SVDQ_OK = 0
 SVDQ_ERR_INVALID_ARG = 1
@@ -26,6 +28,7 @@ SVDQ_ERR_OOM = 3
 SVDQ_ERR_CUDA = 4
 SVDQ_ERR_NUMERIC = 5
 SVDQ_ERR_TIMEOUT = 6
+SVDQ_ERR_BOUNDS = 7
 SVDQ_INT4_G64 = 1
 SVDQ_NVFP4_G16 = 2
 FORMATS = {"int4": SVDQ_INT4_G64, "nvfp4": SVDQ_NVFP4_G16, SVDQ_INT4_G64: SVDQ_INT4_G64,
@@ -62,6 +65,7 @@ _EXPORTS = {
     # name: (restype, argtypes)
     "svdq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "svdq_abi_version": (ctypes.c_int, []),
+    "svdq_debug_build": (ctypes.c_int, []),
     "svdq_canonical_sizes": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                             ctypes.POINTER(ctypes.c_size_t)]),
     "svdq_prepare": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
@@ -135,7 +139,7 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"libsvdq.so not found at {LIB_PATH}: build it with "
+            raise RuntimeError(f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}: build it with "
                                "`python -m diffusion_transformer_w4a4_b200.build` (there is no CPU fallback)")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in _EXPORTS.items():
@@ -171,6 +175,11 @@ def _stream(stream) -> int | None:
 # ----------------------------------------------------------------------------- C names
 def svdq_status_string(status: int) -> str:
     return lib().svdq_status_string(int(status)).decode()
+
+
+def svdq_debug_build() -> int:
+    """1 when the loaded library is the bounds-checked debug variant."""
+    return int(lib().svdq_debug_build())
 
 
 def svdq_abi_version() -> int:

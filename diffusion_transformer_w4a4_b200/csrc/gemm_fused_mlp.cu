@@ -94,6 +94,8 @@ struct FParams {
   uint16_t* H;              // optional [M, N] bf16: bf16(GELU(h))
   int* status;
   unsigned long long limit;
+  // extents in bytes (debug bounds checks)
+  size_t codes_dn_bytes, scales_dn_bytes, t_dn_bytes, tpart_bytes, cnt_bytes, H_bytes;
 };
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
@@ -194,6 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
+  if (threadIdx.x == 0) pdl_launch_dependents();  // the next kernel may start its prologue
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -201,6 +204,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&maps.a);
       prefetch_tmap(&maps.b);
+      pdl_wait();  // the quantized activations come from the previous kernel
       int it = 0;
       bool ok = true;
       for (int u = pair; u < p.num_units && ok; u += npairs) {
@@ -317,6 +321,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&maps.sfa);
       prefetch_tmap(&maps.sfb);
+      pdl_wait();
       int pit = 0;
       bool ok = true;
       const int pairs_k = (p.k_stages + 1) / 2;
@@ -406,6 +411,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9, both CTAs)
+    pdl_wait();  // g_x and the down layer's workspace belong to the stream's order
     const int e = warp - 2;         // 0..7
     const int q = warp & 3;         // tensor-memory lane quarter
     const int half = e >> 2;        // columns 96*half .. 96*half + 95 of the tile
@@ -470,7 +476,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             hbits[j] = *(const uint32_t*)&gh;
             v[j] = __fmul2_rn(__bfloat1622float2(gh), make_float2(il[2 * j], il[2 * j + 1]));
           }
-          if (p.H != nullptr && live) {  // parity export of the down layer's input
+          if (p.H != nullptr && live && SVDQ_INB(p.status, ((size_t)m * p.N + n) * 2, 32, p.H_bytes)) {
+            // parity export of the down layer's input
             *(uint4*)(p.H + (size_t)m * p.N + n) = make_uint4(hbits[0], hbits[1], hbits[2], hbits[3]);
             *(uint4*)(p.H + (size_t)m * p.N + n + 8) = make_uint4(hbits[4], hbits[5], hbits[6], hbits[7]);
           }
@@ -489,7 +496,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           for (int j = 0; j < 8; ++j) qv[j] = __fmul2_rn(v[j], inv2);
           uint32_t c0 = cvt_e2m1x8(qv[0], qv[1], qv[2], qv[3]), c1 = cvt_e2m1x8(qv[4], qv[5], qv[6], qv[7]);
           if (sb == 0) c0 = c1 = 0u;  // a zero block scale: all codes +0
-          if (live) *(uint2*)(p.codes_dn + (size_t)m * (p.N / 2) + n / 2) = make_uint2(c0, c1);
+          if (live && SVDQ_INB(p.status, (size_t)m * (p.N / 2) + n / 2, 8, p.codes_dn_bytes))
+            *(uint2*)(p.codes_dn + (size_t)m * (p.N / 2) + n / 2) = make_uint2(c0, c1);
           swords |= (uint64_t)sb << (8 * blk);
           if (p.rank_dn > 0) {  // bf16(x^') into the swizzled x^' tile
             uint32_t xb[8];
@@ -513,12 +521,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (live) {
           // scale bytes of blocks blk0 .. blk0 + 5 (four consecutive blocks share an atom word)
           const int blk0 = (nt * BN + 96 * half) / 16;
+          const size_t s0 = sf_offset(m, blk0, p.katoms_dn, kSfAtomRows);
+          const size_t s1 = sf_offset(m, blk0 + (half == 0 ? 4 : 2), p.katoms_dn, kSfAtomRows);
           if (half == 0) {  // blocks 12t .. 12t+5: a whole word, then the first half of the next
-            *(uint32_t*)(p.scales_dn + sf_offset(m, blk0, p.katoms_dn, kSfAtomRows)) = (uint32_t)swords;
-            *(uint16_t*)(p.scales_dn + sf_offset(m, blk0 + 4, p.katoms_dn, kSfAtomRows)) = (uint16_t)(swords >> 32);
+            if (SVDQ_INB(p.status, s0, 4, p.scales_dn_bytes)) *(uint32_t*)(p.scales_dn + s0) = (uint32_t)swords;
+            if (SVDQ_INB(p.status, s1, 2, p.scales_dn_bytes)) *(uint16_t*)(p.scales_dn + s1) = (uint16_t)(swords >> 32);
           } else {  // blocks 12t+6 .. 12t+11: the second half of a word, then a whole word
-            *(uint16_t*)(p.scales_dn + sf_offset(m, blk0, p.katoms_dn, kSfAtomRows)) = (uint16_t)swords;
-            *(uint32_t*)(p.scales_dn + sf_offset(m, blk0 + 2, p.katoms_dn, kSfAtomRows)) = (uint32_t)(swords >> 16);
+            if (SVDQ_INB(p.status, s0, 2, p.scales_dn_bytes)) *(uint16_t*)(p.scales_dn + s0) = (uint16_t)swords;
+            if (SVDQ_INB(p.status, s1, 4, p.scales_dn_bytes)) *(uint32_t*)(p.scales_dn + s1) = (uint32_t)(swords >> 16);
           }
         }
       }
@@ -548,13 +558,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           float* dst = p.tpart + ((size_t)sg * p.M + m) * R;
 #pragma unroll
           for (int j = 0; j < 32; j += 4)
-            if (j < R) *(float4*)(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+            if (j < R && SVDQ_INB(p.status, (((size_t)sg * p.M + m) * R + j) * 4, 16, p.tpart_bytes))
+              *(float4*)(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
         }
         if (p.S == 1) {  // one group covers every column: the sum is complete
           if (live) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-              if (j < R) {
+              if (j < R && SVDQ_INB(p.status, ((size_t)m * R + j) * 2, 8, p.t_dn_bytes)) {
                 const __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[j], acc[j + 1]);
                 const __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[j + 2], acc[j + 3]);
                 *(uint2*)(p.t_dn + (size_t)m * R + j) = make_uint2(*(const uint32_t*)&h0, *(const uint32_t*)&h1);
@@ -567,14 +578,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __syncwarp();
         // the last of the S units to finish these 32 rows adds the partials in group order
         int* cnt = p.counters + 4 * rb + q;
-        if (lane == 0) ticket[q] = atomicAdd(cnt, 1);
+        if (lane == 0)
+          ticket[q] = SVDQ_INB(p.status, (size_t)(4 * rb + q) * 4, 4, p.cnt_bytes) ? atomicAdd(cnt, 1) : -1;
         __syncwarp();
         if (ticket[q] == p.S - 1) {
           __threadfence();
           if (live) {
             for (int j = 0; j < R; j += 4) {
-              float4 sum = __ldcg((const float4*)(p.tpart + (size_t)m * R + j));
+              float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (SVDQ_INB(p.status, ((size_t)m * R + j) * 4, 16, p.tpart_bytes))
+                sum = __ldcg((const float4*)(p.tpart + (size_t)m * R + j));
               for (int g = 1; g < p.S; ++g) {
+                if (!SVDQ_INB(p.status, (((size_t)g * p.M + m) * R + j) * 4, 16, p.tpart_bytes)) continue;
                 const float4 v4 = __ldcg((const float4*)(p.tpart + ((size_t)g * p.M + m) * R + j));
                 sum.x += v4.x;
                 sum.y += v4.y;
@@ -583,7 +598,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               }
               const __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
               const __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
-              *(uint2*)(p.t_dn + (size_t)m * R + j) = make_uint2(*(const uint32_t*)&h0, *(const uint32_t*)&h1);
+              if (SVDQ_INB(p.status, ((size_t)m * R + j) * 2, 8, p.t_dn_bytes))
+                *(uint2*)(p.t_dn + (size_t)m * R + j) = make_uint2(*(const uint32_t*)&h0, *(const uint32_t*)&h1);
             }
           }
           if (lane == 0) *cnt = 0;  // every unit has arrived: ready for the next call
@@ -691,6 +707,12 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.H = (uint16_t*)H;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
+  p.codes_dn_bytes = wd.codes_bytes;
+  p.scales_dn_bytes = wd.scales_bytes;
+  p.t_dn_bytes = wd.t_bytes;
+  p.tpart_bytes = wd.tpart_bytes;
+  p.cnt_bytes = 4 * (size_t)kAmaxSlots;
+  p.H_bytes = (size_t)M * N * 2;
 
   const size_t smem = 1024 + (size_t)SMEM_BYTES + 512;
   static int attr_done[64] = {0};
@@ -723,7 +745,8 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.S = S;
   p.num_units = p.m_tiles * S;
   const int npairs = p.num_units < npairs_max ? p.num_units : npairs_max;
-  k_gemm_gelu_quant<<<2 * npairs, THREADS, smem, stream>>>(maps, p);
+  if (launch_pdl(k_gemm_gelu_quant, dim3(2 * npairs), dim3(THREADS), smem, stream, maps, p) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 

@@ -81,6 +81,7 @@ struct GParams {
   float g_w;
   int* status;
   unsigned long long limit;
+  size_t sfa_bytes, sfb_bytes;  // extents of the scale-factor arrays (debug bounds checks)
 };
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
@@ -133,6 +134,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) pdl_launch_dependents();  // the next kernel may start its prologue
   const uint32_t tmem = *tmem_slot;
   const int units = p.n_lr + p.k_stages;
 
@@ -141,6 +143,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     if (lane == 0) {
       prefetch_tmap(&maps.a);
       prefetch_tmap(&maps.b);
+      pdl_wait();  // the quantized activations come from the previous kernel
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     // Pair j of a tile carries the atoms of K stages 2j and 2j+1 (one stage for
     // an odd tail): [SFA stage 2j | SFA 2j+1 | SFB stage 2j | SFB 2j+1].
     if (lane == 0) {
+      pdl_wait();  // the activation scales come from the previous kernel
       int pit = 0;
       bool ok = true;
       const int pairs = (p.k_stages + 1) / 2;
@@ -244,9 +248,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
           const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
           uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
           mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
-          bulk_load(dst, p.sfa + ((size_t)mt * p.katoms + 8 * j) * kSfAtomBytes, ns * SFA_BYTES, &sfs_full[slot]);
-          bulk_load(dst + 2 * SFA_BYTES, p.sfb + ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes, ns * SFB_BYTES,
-                    &sfs_full[slot]);
+          const size_t oa = ((size_t)mt * p.katoms + 8 * j) * kSfAtomBytes;
+          const size_t ob = ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes;
+          // (debug variant: a copy that would leave its array is not issued; the
+          // stage's wait then expires, after the bounds error was recorded)
+          if (SVDQ_INB(p.status, oa, ns * SFA_BYTES, p.sfa_bytes))
+            bulk_load(dst, p.sfa + oa, ns * SFA_BYTES, &sfs_full[slot]);
+          if (SVDQ_INB(p.status, ob, ns * SFB_BYTES, p.sfb_bytes))
+            bulk_load(dst + 2 * SFA_BYTES, p.sfb + ob, ns * SFB_BYTES, &sfs_full[slot]);
         }
       }
       if (!ok) {  // drain the copies still in flight
@@ -298,6 +307,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();  // g_x and Y belong to the stream's order
     const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;  // exact: powers of two
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     uint8_t* stg = epi_stage + (warp - 2) * 2 * EPI_STAGE_BYTES;
@@ -452,6 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
+  if (threadIdx.x == 0) pdl_launch_dependents();  // the next kernel may start its prologue
   const uint32_t tmem = *tmem_slot;
   const int units = p.n_lr + p.k_stages;
 
@@ -460,6 +471,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&maps.a);
       prefetch_tmap(&maps.b);
+      pdl_wait();  // the quantized activations come from the previous kernel
       int it = 0;
       bool ok = true;
       for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
@@ -568,6 +580,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     if (lane == 0) {
       prefetch_tmap(&maps.sfa);
       prefetch_tmap(&maps.sfb);
+      pdl_wait();
       int pit = 0;
       bool ok = true;
       const int pairs_k = (p.k_stages + 1) / 2;
@@ -598,6 +611,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    pdl_wait();  // g_x and Y belong to the stream's order
     const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;  // exact: powers of two
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
     uint8_t* stg = epi_stage + (warp - 2) * 2 * EPI_STAGE_BYTES;
@@ -744,6 +758,8 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
   p.gx_dev = L->dyn_gx ? (const float*)(ws + w.status + 4) : nullptr;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
+  p.sfa_bytes = w.scales_bytes;
+  p.sfb_bytes = L->off.total - L->off.wscales;
 
   // Token counts above one 128-row tile use the CTA-pair kernel (256-row tiles)
   // when the device can co-schedule its clusters.
@@ -793,7 +809,8 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
       p.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
       p.num_tiles = p.m_tiles * p.n_tiles;
       const int npairs = p.num_tiles < maxc ? p.num_tiles : maxc;
-      k_gemm_nvfp4_pair<<<2 * npairs, P_THREADS, psmem, stream>>>(maps, p);
+      if (launch_pdl(k_gemm_nvfp4_pair, dim3(2 * npairs), dim3(P_THREADS), psmem, stream, maps, p) != cudaSuccess)
+        return SVDQ_ERR_CUDA;
       return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
     }
   }
@@ -825,7 +842,7 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
   if (cudaFuncSetAttribute(k_gemm_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   const int grid = p.num_tiles < sm_count(L->device) ? p.num_tiles : sm_count(L->device);
-  k_gemm_nvfp4<<<grid, THREADS, smem, stream>>>(maps, p);
+  if (launch_pdl(k_gemm_nvfp4, dim3(grid), dim3(THREADS), smem, stream, maps, p) != cudaSuccess) return SVDQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 

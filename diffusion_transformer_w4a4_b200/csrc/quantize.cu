@@ -74,6 +74,8 @@ struct QParams {
   int* counters;
   int* status;
   unsigned long long limit;
+  // buffer extents in bytes, for the debug variant's bounds checks
+  size_t x_bytes, il_bytes, codes_bytes, scales_bytes, t_bytes, tpart_bytes, cnt_bytes;
 };
 
 // eight floats (as four pairs, element order a.x a.y b.x b.y ...) -> eight E2M1
@@ -197,12 +199,14 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) pdl_launch_dependents();  // the GEMM's prologue may start as SMs free up
 
   // NVFP4 per-tensor scale: the prepared static one, or the dynamic one from the
   // first pass's maxima (then t is stored as t / g_x, an exact power-of-two
   // scaling, because the packed L2 carries only 1/g_w)
   float inv_gs = p.inv_g, dens = p.den, tsc = 1.f;
   if (FMT == SVDQ_NVFP4_G16 && p.amax_slots != nullptr) {
+    pdl_wait();  // the first pass's maxima
     __shared__ float dred[kThreads / 32];
     float m = 0.f;
     for (int i = threadIdx.x; i < p.nslots; i += kThreads) m = fmaxf(m, p.amax_slots[i]);
@@ -276,6 +280,7 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
     // chunk, so a warp reads two rows (two 512-byte runs) per load instruction.
     // Each warp loads its rows of a chunk straight from global memory into
     // registers (no staging), then quantizes them.
+    pdl_wait();  // X and the workspace belong to the stream's order
     const int rsub = lane >> 4;  // row within the warp's 2-row step
     const int j = lane & 15;     // 16-column block within the chunk
     constexpr int ITS = kRowsPerWarp / 2;
@@ -303,14 +308,21 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
       for (int it = 0; it < ITS; ++it) {
         const int64_t m = mbase + 2 * it;
         const int64_t mr = m < p.M ? m : 0;  // rows past M read row 0 (never stored)
-        const uint4* src = (const uint4*)(p.x + (size_t)mr * p.K + kk0 + (size_t)i * kChunk);
-        xr[it][0] = __ldcs(src);
-        xr[it][1] = __ldcs(src + 1);
+        const size_t xe = (size_t)mr * p.K + kk0 + (size_t)i * kChunk;
+        const uint4* src = (const uint4*)(p.x + xe);
+        if (SVDQ_INB(p.status, 2 * xe, 32, p.x_bytes)) {
+          xr[it][0] = __ldcs(src);
+          xr[it][1] = __ldcs(src + 1);
+        } else {
+          xr[it][0] = xr[it][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       float2 il[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float4 t4 = __ldg((const float4*)(ilp + (size_t)i * kChunk) + q);
+        const size_t ioff = ((size_t)(kk0 + i * kChunk) + 4 * q) * 4;
+        const float4 t4 = SVDQ_INB(p.status, ioff, 16, p.il_bytes) ? __ldg((const float4*)(ilp + (size_t)i * kChunk) + q)
+                                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
         il[2 * q] = make_float2(t4.x, t4.y);
         il[2 * q + 1] = make_float2(t4.z, t4.w);
       }
@@ -349,8 +361,9 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
             const uint32_t s1 = __shfl_sync(0xffffffffu, sb, base + 1);
             const uint32_t s2 = __shfl_sync(0xffffffffu, sb, base + 2);
             const uint32_t s3 = __shfl_sync(0xffffffffu, sb, base + 3);
-            if ((lane & 3) == 0 && live) *(uint32_t*)(p.scales + sbyte) = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
-            if (live) *(uint2*)(p.codes + cbyte) = packed;
+            if ((lane & 3) == 0 && live && SVDQ_INB(p.status, sbyte, 4, p.scales_bytes))
+              *(uint32_t*)(p.scales + sbyte) = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            if (live && SVDQ_INB(p.status, cbyte, 8, p.codes_bytes)) *(uint2*)(p.codes + cbyte) = packed;
           } else {
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -373,8 +386,10 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
               y1 = __fadd2_rn(__fadd2_rn(y1, magic), nmagic);
               qb[e >> 1] = cvt_e4m3x2(y0.x, y0.y) | (cvt_e4m3x2(y1.x, y1.y) << 16);
             }
-            if ((lane & 3) == 0 && live) *(__half*)(p.scales + sbyte) = s16;
-            if (live) *(uint4*)(p.codes + cbyte) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
+            if ((lane & 3) == 0 && live && SVDQ_INB(p.status, sbyte, 2, p.scales_bytes))
+              *(__half*)(p.scales + sbyte) = s16;
+            if (live && SVDQ_INB(p.status, cbyte, 16, p.codes_bytes))
+              *(uint4*)(p.codes + cbyte) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
           }
           if constexpr (RANK > 0) {
             uint32_t b[8];
@@ -424,7 +439,8 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
 #pragma unroll
               for (int j = 0; j < RANK; j += 2) {
                 __nv_bfloat162 h = scale_t(__floats2bfloat162_rn(acc[j], acc[j + 1]), tsc);
-                *(uint32_t*)(p.t + (size_t)m * RANK + j) = *(uint32_t*)&h;
+                if (SVDQ_INB(p.status, ((size_t)m * RANK + j) * 2, 4, p.t_bytes))
+                  *(uint32_t*)(p.t + (size_t)m * RANK + j) = *(uint32_t*)&h;
               }
             }
           } else {
@@ -432,19 +448,24 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
               float* dst = p.tpart + ((size_t)slice * p.M + m) * RANK;
 #pragma unroll
               for (int j = 0; j < RANK; j += 4)
-                *(float4*)(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                if (SVDQ_INB(p.status, (((size_t)slice * p.M + m) * RANK + j) * 4, 16, p.tpart_bytes))
+                  *(float4*)(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
             }
             __threadfence();
             named_bar_sync(2, 128);
-            if (threadIdx.x == 0) *ticket = atomicAdd(p.counters + rowblock, 1);
+            if (threadIdx.x == 0)
+              *ticket = SVDQ_INB(p.status, (size_t)rowblock * 4, 4, p.cnt_bytes) ? atomicAdd(p.counters + rowblock, 1) : -1;
             named_bar_sync(2, 128);
             if (*ticket == p.nslices - 1) {  // last slice of this row block: fixed-order sum
               __threadfence();
               if (m < p.M) {
 #pragma unroll
                 for (int j = 0; j < RANK; j += 4) {
-                  float4 sum = __ldcg((const float4*)(p.tpart + (size_t)m * RANK + j));
+                  float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                  if (SVDQ_INB(p.status, ((size_t)m * RANK + j) * 4, 16, p.tpart_bytes))
+                    sum = __ldcg((const float4*)(p.tpart + (size_t)m * RANK + j));
                   for (int sl = 1; sl < p.nslices; ++sl) {
+                    if (!SVDQ_INB(p.status, (((size_t)sl * p.M + m) * RANK + j) * 4, 16, p.tpart_bytes)) continue;
                     const float4 v = __ldcg((const float4*)(p.tpart + ((size_t)sl * p.M + m) * RANK + j));
                     sum.x += v.x;
                     sum.y += v.y;
@@ -453,10 +474,12 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
                   }
                   __nv_bfloat162 h0 = scale_t(__floats2bfloat162_rn(sum.x, sum.y), tsc);
                   __nv_bfloat162 h1 = scale_t(__floats2bfloat162_rn(sum.z, sum.w), tsc);
-                  *(uint2*)(p.t + (size_t)m * RANK + j) = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+                  if (SVDQ_INB(p.status, ((size_t)m * RANK + j) * 2, 8, p.t_bytes))
+                    *(uint2*)(p.t + (size_t)m * RANK + j) = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
                 }
               }
-              if (threadIdx.x == 0) p.counters[rowblock] = 0;  // ready for the next call
+              if (threadIdx.x == 0 && SVDQ_INB(p.status, (size_t)rowblock * 4, 4, p.cnt_bytes))
+                p.counters[rowblock] = 0;  // ready for the next call
             }
           }
         }
@@ -484,7 +507,7 @@ int launch_rank(const CUtensorMap& ml1, const QParams& p, int64_t M, cudaStream_
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   const dim3 grid((unsigned)((M + kRows - 1) / kRows), (unsigned)p.nslices);
-  kern<<<grid, Roles<RANK>::kThreads, smem, stream>>>(ml1, q);
+  if (launch_pdl(kern, grid, dim3(Roles<RANK>::kThreads), smem, stream, ml1, q) != cudaSuccess) return SVDQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
@@ -535,6 +558,13 @@ int launch_quantize(const svdq_layer* L, const void* X, int64_t M, uint8_t* ws, 
   p.status = (int*)(ws + w.status);
   p.counters = (int*)(ws + w.status + 16);
   p.limit = wait_limit_cycles();
+  p.x_bytes = (size_t)M * L->K * 2;
+  p.il_bytes = (size_t)L->K * 4;
+  p.codes_bytes = w.codes_bytes;
+  p.scales_bytes = w.scales_bytes;
+  p.t_bytes = w.t_bytes;
+  p.tpart_bytes = w.tpart_bytes;
+  p.cnt_bytes = w.amax - (w.status + 16);
   if (L->fmt == SVDQ_NVFP4_G16) return launch_fmt<SVDQ_NVFP4_G16>(L->map_l1, p, M, L->rank, stream);
   return launch_fmt<SVDQ_INT4_G64>(L->map_l1, p, M, L->rank, stream);
 }

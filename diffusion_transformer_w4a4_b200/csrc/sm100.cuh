@@ -76,6 +76,25 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
+// ---------------------------------------------------------------- debug bounds checks
+// In the library's debug variant (built with -DSVDQ_DEBUG_BOUNDS) every global
+// access that a kernel addresses itself (not through a tensor map, whose boxes
+// the hardware clips) is first checked against the extent of its buffer: an
+// access that would leave the buffer records SVDQ_ERR_BOUNDS (7) in the status
+// word and is skipped.  Nothing traps.  In the release build the check is the
+// constant `true` and compiles away.
+#ifdef SVDQ_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(int* status, size_t off, size_t bytes, size_t extent) {
+  if (off <= extent && bytes <= extent - off) return true;
+  if (status) atomicCAS(status, 0, 7);
+  return false;
+}
+#define SVDQ_INB(status, off, bytes, extent) \
+  ::svdq::in_bounds((status), (size_t)(off), (size_t)(bytes), (size_t)(extent))
+#else
+#define SVDQ_INB(status, off, bytes, extent) (static_cast<void>(off), true)
+#endif
+
 // ---------------------------------------------------------------- packed f32x2
 // (a0, a1) *= (b0, b1) with one packed instruction; each product is an ordinary
 // binary32 round-to-nearest multiply.

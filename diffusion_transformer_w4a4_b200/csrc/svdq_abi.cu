@@ -141,11 +141,20 @@ const char* svdq_status_string(int status) {
     case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA: a CUDA call failed";
     case SVDQ_ERR_NUMERIC: return "SVDQ_ERR_NUMERIC: non-finite input";
     case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT: an in-kernel wait ran past its limit";
+    case SVDQ_ERR_BOUNDS: return "SVDQ_ERR_BOUNDS: a kernel addressed memory outside its buffer (debug build)";
     default: return "SVDQ_ERR_UNKNOWN";
   }
 }
 
 int svdq_abi_version(void) { return SVDQ_ABI_VERSION; }
+
+int svdq_debug_build(void) {
+#ifdef SVDQ_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 svdq_status svdq_canonical_sizes(int64_t N, int64_t K, int rank, int fmt, size_t sizes[7]) {
   if (!sizes || !shape_ok(N, K, rank, fmt)) return SVDQ_ERR_INVALID_ARG;

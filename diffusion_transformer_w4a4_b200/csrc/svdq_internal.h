@@ -30,6 +30,27 @@ constexpr int kAmaxSlots = 1024;  // per-CTA maxima of the dynamic activation-sc
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch with programmatic dependent launch allowed: the kernel lets the next
+// one on the stream be scheduled early (griddepcontrol.launch_dependents) and
+// waits (griddepcontrol.wait) before it touches what earlier work on the stream
+// produced or still reads, so its prologue (barriers, tensor memory, tensor-map
+// fetches) overlaps the tail of the kernel before it.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // NVTX range around the host-side enqueue of a kernel group ("svdq/quantize",
 // "svdq/gemm", ...), so a timeline tool can attribute the launches; without a
 // tool attached the calls do nothing.

@@ -58,13 +58,22 @@ typedef enum svdq_status {
   SVDQ_ERR_OOM = 3,                /* a host allocation failed (svdq_prepare/pack) */
   SVDQ_ERR_CUDA = 4,               /* a CUDA runtime/driver call failed */
   SVDQ_ERR_NUMERIC = 5,            /* non-finite input to svdq_prepare */
-  SVDQ_ERR_TIMEOUT = 6             /* an in-kernel wait ran past its limit */
+  SVDQ_ERR_TIMEOUT = 6,            /* an in-kernel wait ran past its limit */
+  SVDQ_ERR_BOUNDS = 7              /* debug build only: a kernel computed a global address outside its
+                                      buffer; the access was skipped (see svdq_debug_build) */
 } svdq_status;
 
 typedef enum svdq_format { SVDQ_INT4_G64 = 1, SVDQ_NVFP4_G16 = 2 } svdq_format;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* svdq_status_string(int status);
+
+/* 1 in the library's bounds-checked debug variant (libsvdq_debug.so, built with
+ * -DSVDQ_DEBUG_BOUNDS), 0 in the release library.  In the debug variant every
+ * global access that a kernel addresses itself is checked against its buffer;
+ * one that would leave it records SVDQ_ERR_BOUNDS in the status word and is
+ * skipped (nothing traps).  Same entry points and results otherwise, slower. */
+int svdq_debug_build(void);
 
 /* ABI version of this header (increments on incompatible change).
  * 2: the svdq workspace control block holds the per-call g_x and the first
