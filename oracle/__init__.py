@@ -119,12 +119,14 @@ def bf16_to_f32(h):
 
 # ----------------------------------------------------------------------------- GELU
 def gelu_f64(h: np.ndarray) -> np.ndarray:
-    """GELU in its erf form, h/2 (1 + erf(h / sqrt 2)), in binary64 (the
-    activation between a diffusion transformer block's MLP linears)."""
-    from scipy.special import erf
+    """GELU in its erf form, h Phi(h) = h/2 (1 + erf(h / sqrt 2)), in binary64 (the
+    activation between a diffusion transformer block's MLP linears).  Evaluated
+    as h/2 erfc(-h / sqrt 2), the same value: 1 + erf(x) cancels to 0 in binary64
+    once x < -5.9 or so, erfc keeps the tail."""
+    from scipy.special import erfc
 
     h = np.asarray(h, np.float64)
-    return 0.5 * h * (1.0 + erf(h / math.sqrt(2.0)))
+    return 0.5 * h * erfc(-h / math.sqrt(2.0))
 
 
 def gelu_bf16(h_bits: np.ndarray) -> np.ndarray:

@@ -77,8 +77,14 @@ def _run(M, K, N, N2, r_up, r_dn, lid, rows=None):
     # x' against the binary64 GELU of the unfused GPU path's up output
     y_up = g_up.forward(X)
     ref_h = oracle.gelu_bf16(y_up)
-    dh = np.abs(oracle.bf16_to_f32(Hb).astype(np.float64) - oracle.bf16_to_f32(ref_h).astype(np.float64))
-    assert np.all(dh <= bf16_ulp(oracle.bf16_to_f32(ref_h))), int(np.sum(dh > bf16_ulp(oracle.bf16_to_f32(ref_h))))
+    hg, hr = oracle.bf16_to_f32(Hb).astype(np.float64), oracle.bf16_to_f32(ref_h).astype(np.float64)
+    # one ulp of the larger of the two (a rounding boundary may sit on a binade edge)
+    lim = np.maximum(bf16_ulp(hg), bf16_ulp(hr))
+    bad = np.abs(hg - hr) > lim
+    if bad.any():
+        i = np.argwhere(bad)[:5]
+        ex = [(float(oracle.bf16_to_f32(y_up[a, b])), float(hg[a, b]), float(hr[a, b])) for a, b in i]
+        raise AssertionError(f"{int(bad.sum())} x' elements beyond one ulp; (h, gpu, ref): {ex}")
     n_h_flip = int(np.sum(Hb != ref_h))
 
     # the down layer, teacher-forced on the GPU's x'

@@ -17,6 +17,14 @@ def test_normal_cdf_points():
     assert oracle.gelu_f64(np.array([0.0]))[0] == 0.0
 
 
+def test_negative_tail():
+    # Phi(-10) = 7.6198530241604696e-24, Phi(-8) = 6.2209605742717841e-16 (normal CDF tables)
+    np.testing.assert_allclose(oracle.gelu_f64(np.array([-10.0, -8.0])),
+                               [-10 * 7.6198530241604696e-24, -8 * 6.2209605742717841e-16], rtol=1e-13)
+    # the tail is kept through the bf16 rounding: bf16 has binary32's exponent range
+    assert oracle.bf16_to_f32(oracle.gelu_bf16(oracle.f32_to_bf16(np.array([-9.25], np.float32))))[0] < 0
+
+
 def test_odd_part_identity_and_asymptotes():
     h = np.linspace(-9.0, 9.0, 1801)
     g = oracle.gelu_f64(h)
