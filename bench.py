@@ -446,7 +446,7 @@ def fused_mlp_measure(dev, lins, xs, steps=20):
     flops = sum(_layer_flops(l) for l in LAYERS)
     return {"step_us": step, "quantize_up_us": med(0, 1), "fused_gemm_gelu_quantize_us": med(1, 2),
             "gemm_down_us": med(2, 3), "tops": flops / (step * 1e-6) / 1e12,
-            "kernels": ["k_quantize", "k_gemm_gelu_quant", "k_gemm_nvfp4_pair"], "gpu_launches": 3 * steps,
+            "kernels": ["k_quantize", "k_gemm_gelu_quant", "k_gemm_nvfp4"], "gpu_launches": 3 * steps,
             "note": "compare step_us with ms_per_step of the main line (unfused: two quantizers, two GEMMs)"}
 
 

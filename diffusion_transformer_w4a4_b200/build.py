@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
                "--fmad=false" if src.endswith("host_prepare.cpp") else "--fmad=true",
                "-I", os.path.join(HERE, "..", "include"), "-c", src, "-o", obj, *(extra or [])]
         if src.endswith(".cpp"):
-            cmd = [nvcc, "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-ffp-contract=off,-pthread",
+            cmd = [nvcc, *ARCH, "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-ffp-contract=off,-pthread",
                    "-I", os.path.join(HERE, "..", "include"), "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)

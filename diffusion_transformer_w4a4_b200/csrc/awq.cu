@@ -327,17 +327,6 @@ __global__ void __launch_bounds__(kAwqMaxThreads) k_awq_gemv(const __grid_consta
   }
 }
 
-int awq_sm_count(int dev) {
-  static int cache[64] = {0};
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cache[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
-  }
-  return cache[dev];
-}
-
 // Launch shape for a K: row groups, ring depth and dynamic shared memory.
 struct AwqShape {
   int T, G, stages, xs_off;
@@ -398,7 +387,7 @@ int launch_awq(AwqParams p, int dev, cudaStream_t stream) {
   if (per_sm < 1) return SVDQ_ERR_CUDA;
   const int R = a.G * kAwqRpt;
   const int nbatch = (p.N + R - 1) / R;
-  int grid = awq_sm_count(dev) * per_sm;
+  int grid = device_sm_count(dev) * per_sm;
   if (grid > nbatch) grid = nbatch;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

@@ -13,21 +13,23 @@
 // layer's quantizer need no cross-thread step, and the up layer's N columns
 // are the down layer's K columns.  The low-rank sum t' runs over all N columns
 // of a row; each tile contributes bf16(x^'_tile) . L1'[tile columns] with a
-// pair MMA into a 32-column tensor-memory accumulator that persists across the
-// tiles of a work unit (one 256-row M tile times one of S contiguous groups of
-// N tiles), and the S partial sums of a row are added in a fixed order by the
-// unit that finishes last (counter per 128-row block), as the standalone
-// quantizer does for its K slices.
+// tensor-core MMA into a 32-column tensor-memory accumulator that persists
+// across the tiles of a work unit (one 128-row M tile times one of S contiguous
+// groups of N tiles), and the S partial sums of a row are added in a fixed
+// order by the unit that finishes last (counter per 32-row group), as the
+// standalone quantizer does for its K slices.
 //
-// Same main loop as the CTA-pair NVFP4 GEMM (k_gemm_nvfp4_pair: 256 x 192 tile,
-// cta_group::2, no multicast loads; scale factors copied into tensor memory by
-// the leader with tcgen05.cp.cta_group::2).  Roles per CTA (384 threads):
-//   warp 0      operand TMA producer            warp 1   tensor memory, main MMAs (leader)
+// Same main loop as the single-CTA NVFP4 GEMM (k_gemm_nvfp4: 128 x 192 tile,
+// block-scaled kind::mxf4nvf4, scale factors moved into tensor memory by four
+// mover warps), with a 3-stage operand ring to make room for the x^' tile and
+// the L1' slice.  Roles per CTA (512 threads):
+//   warp 0      operand TMA producer            warp 1   tensor memory, main MMAs
 //   warps 2-9   epilogue: two warps per tensor-memory lane quarter, 96 columns each
-//   warp 10     scale-factor producer           warp 11  L1'^T slices and t' MMAs (leader)
-// Tensor memory: two 192-column accumulators, one 48-column scale-factor
-// buffer and the 32-column t' accumulator, so the down layer's rank is at most
-// 32.  Every wait is bounded; no load uses cluster multicast.
+//   warps 10-13 scale-factor movers             warp 14  scale-factor producer
+//   warp 15     L1'^T slice loader and t' MMA issuer, per tile
+// Tensor memory (512 columns): two 192-column accumulators, two 48-column
+// scale-factor buffers and the 32-column t' accumulator, so the down layer's
+// rank is at most 32.  Every wait is bounded; no load uses cluster multicast.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -38,40 +40,35 @@
 namespace svdq {
 namespace {
 
-constexpr int BM = kGemmBM;   // 128 rows per CTA
+constexpr int BM = kGemmBM;   // 128
 constexpr int BN = kNvfp4BN;  // 192
-constexpr int PB_ROWS = BN / 2;
-constexpr int STAGES = 5;
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * 128;
-constexpr int B_BYTES = PB_ROWS * 128;
+constexpr int B_BYTES = BN * 128;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SFA_BYTES = 4 * kSfAtomBytes;
 constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;
 constexpr int SF_SLOTS = 2;
 constexpr int SF_SLOT_BYTES = 2 * (SFA_BYTES + SFB_BYTES);
-constexpr int XT_BYTES = 3 * BM * 128;    // bf16 x^' tile: three 64-column halves, 128B-swizzled
-constexpr int L1_MAX_ROWS = 16;           // rank/2 rows of L1'^T per CTA (rank <= 32)
+constexpr int XT_BYTES = 3 * BM * 128;  // bf16 x^' tile: three 64-column blocks, 128B-swizzled
+constexpr int L1_MAX_ROWS = 32;         // rank rows of L1'^T (rank <= 32)
 constexpr int L1_BYTES = 3 * L1_MAX_ROWS * 128;
-constexpr int THREADS = 384;
-constexpr int SF_WARP = 10, T_WARP = 11;
+constexpr int THREADS = 512;
+constexpr int SF_WARP = 14, T_WARP = 15;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL = 2 * BN;
+constexpr uint32_t SF_COL = 2 * BN;     // 384: two buffers of [SFA 16 | SFB 32] columns
 constexpr uint32_t SF_BUF_COLS = 48;
-constexpr uint32_t TP_COL = SF_COL + SF_BUF_COLS;  // 432
+constexpr uint32_t TP_COL = SF_COL + 2 * SF_BUF_COLS;  // 480
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + XT_BYTES + L1_BYTES;
-constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(2 * BM, BN);
-constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(2 * BM, BN);
+constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(BM, BN);
+constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
 static_assert(STAGE_BYTES % 1024 == 0 && SF_SLOT_BYTES % 1024 == 0 && XT_BYTES % 1024 == 0, "alignment");
 static_assert(SMEM_BYTES + 1024 + 512 <= 227 * 1024, "shared memory budget");
 static_assert(TP_COL + 32 <= TMEM_COLS, "tensor memory budget");
 
 struct FusedMaps {
-  CUtensorMap a, b, t[3], l2[3], l1dn, sfa, sfb;
+  CUtensorMap a, b, t[3], l2[3], l1dn;
 };
-
-__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 
 struct FParams {
   int M, N, K, m_tiles, n_tiles, num_units, S, k_stages, katoms;
@@ -95,7 +92,7 @@ struct FParams {
   int* status;
   unsigned long long limit;
   // extents in bytes (debug bounds checks)
-  size_t codes_dn_bytes, scales_dn_bytes, t_dn_bytes, tpart_bytes, cnt_bytes, H_bytes;
+  size_t sfa_bytes, sfb_bytes, codes_dn_bytes, scales_dn_bytes, t_dn_bytes, tpart_bytes, cnt_bytes, H_bytes;
 };
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
@@ -133,38 +130,36 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 // bf16 round-to-nearest-even of a binary32 value, returned as the binary32 it denotes
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     k_gemm_gelu_quant(const __grid_constant__ FusedMaps maps, const __grid_constant__ FParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sfring = smem + STAGES * STAGE_BYTES;
   uint8_t* xt = sfring + SF_SLOTS * SF_SLOT_BYTES;  // 1024-aligned
   uint8_t* l1s = xt + XT_BYTES;                     // 1024-aligned
-  uint64_t* full = (uint64_t*)(l1s + L1_BYTES);     // leader
-  uint64_t* empty = full + STAGES;                  // both
-  uint64_t* acc_full = empty + STAGES;              // both [2]
-  uint64_t* acc_empty = acc_full + 2;               // leader [2]: 16 epilogue warps
-  uint64_t* mma_done = acc_empty + 2;               // leader
-  uint64_t* sfs_full = mma_done + 1;                // leader [SF_SLOTS]: both CTAs' atoms
-  uint64_t* sfs_empty = sfs_full + SF_SLOTS;        // both: released by the leader's MMAs
-  uint64_t* l1_full = sfs_empty + SF_SLOTS;         // leader: both CTAs' L1' slices
-  uint64_t* xt_full = l1_full + 1;                  // leader: 16 epilogue warps
-  uint64_t* xt_free = xt_full + 1;                  // both: t' MMAs of the tile done (x^' tile and L1' slot free)
-  uint64_t* tp_full = xt_free + 1;                  // both: the unit's t' sum is complete
-  uint64_t* tp_empty = tp_full + 1;                 // leader: 8 reader warps (4 per CTA)
-  uint64_t* tdone = tp_empty + 1;                   // leader: t' issuer drain
+  uint64_t* full = (uint64_t*)(l1s + L1_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;    // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2]: 8 epilogue warps
+  uint64_t* mma_done = acc_empty + 2;
+  uint64_t* sf_ready = mma_done + 1;      // [2]: 4 movers
+  uint64_t* sf_free = sf_ready + 2;       // [2]
+  uint64_t* sfs_full = sf_free + 2;       // [SF_SLOTS]
+  uint64_t* sfs_empty = sfs_full + SF_SLOTS;
+  uint64_t* l1_full = sfs_empty + SF_SLOTS;
+  uint64_t* xt_full = l1_full + 1;        // 8 epilogue warps
+  uint64_t* xt_free = xt_full + 1;        // t' MMAs of the tile done (x^' tile and L1' slot free)
+  uint64_t* tp_full = xt_free + 1;        // the unit's t' sum is complete
+  uint64_t* tp_empty = tp_full + 1;       // 4 reader warps
+  uint64_t* tdone = tp_empty + 1;
   uint32_t* tmem_slot = (uint32_t*)(tdone + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  volatile int* ticket = abort_flag + 1;            // [4] one per lane-quarter reader warp
+  volatile int* ticket = abort_flag + 1;  // [4] one per lane-quarter reader warp
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   WaitCtl wc{abort_flag, p.status, p.limit};
   const unsigned long long drain_limit = p.limit > (1ull << 24) ? p.limit : (1ull << 24);
   const int units = p.n_lr + p.k_stages;
-  const int rh = p.rank_dn / 2;  // L1'^T rows per CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -173,83 +168,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 16);
+      mbar_init(&acc_empty[b], 8);
+      mbar_init(&sf_ready[b], 4);
+      mbar_init(&sf_free[b], 1);
     }
     mbar_init(mma_done, 1);
     for (int b = 0; b < SF_SLOTS; ++b) {
       mbar_init(&sfs_full[b], 1);
-      mbar_init(&sfs_empty[b], 1);
+      mbar_init(&sfs_empty[b], 4);
     }
     mbar_init(l1_full, 1);
-    mbar_init(xt_full, 16);
+    mbar_init(xt_full, 8);
     mbar_init(xt_free, 1);
     mbar_init(tp_full, 1);
-    mbar_init(tp_empty, 8);
+    mbar_init(tp_empty, 4);
     mbar_init(tdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, TMEM_COLS);
-    tmem_relinquish_pair();
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
-  cluster_sync();
+  __syncthreads();
   tc_fence_after();
   if (threadIdx.x == 0) pdl_launch_dependents();  // the next kernel may start its prologue
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ operand producer (both CTAs)
+    // ------------------------------------------------------------ operand producer
     if (lane == 0) {
       prefetch_tmap(&maps.a);
       prefetch_tmap(&maps.b);
       pdl_wait();  // the quantized activations come from the previous kernel
       int it = 0;
       bool ok = true;
-      for (int u = pair; u < p.num_units && ok; u += npairs) {
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const int mt = u % p.m_tiles, sg = u / p.m_tiles;
         const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
         for (int nt = nt0; nt < nt1 && ok; ++nt) {
-          const int arow = mt * 2 * BM + (int)rank * BM, brow = nt * BN + (int)rank * PB_ROWS;
           for (int st = 0; st < units; ++st, ++it) {
             const int s = it % STAGES;
-            if (!mbar_wait_cl(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
+            if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
               ok = false;
               break;
             }
             uint8_t* dst = smem + s * STAGE_BYTES;
-            const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
             if (st < p.n_lr) {
               const int w = p.lr_w[st], mi = lr_map_index(w);
-              if (leader) mbar_arrive_expect_tx(&full[s], 2u * (uint32_t)(BM + PB_ROWS) * 2 * w);
-              tma_load_2d_pair(&maps.t[mi], fbar, dst, p.lr_off[st], arow);
-              tma_load_2d_pair(&maps.l2[mi], fbar, dst + A_BYTES, p.lr_off[st], brow);
+              mbar_arrive_expect_tx(&full[s], (uint32_t)(BM + BN) * 2 * w);
+              tma_load_2d(&maps.t[mi], &full[s], dst, p.lr_off[st], mt * BM);
+              tma_load_2d(&maps.l2[mi], &full[s], dst + A_BYTES, p.lr_off[st], nt * BN);
             } else {
               const int ks = st - p.n_lr;
-              if (leader) mbar_arrive_expect_tx(&full[s], 2u * STAGE_BYTES);
-              tma_load_2d_pair(&maps.a, fbar, dst, ks * 128, arow);
-              tma_load_2d_pair(&maps.b, fbar, dst + A_BYTES, ks * 128, brow);
+              mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+              tma_load_2d(&maps.a, &full[s], dst, ks * 128, mt * BM);
+              tma_load_2d(&maps.b, &full[s], dst + A_BYTES, ks * 128, nt * BN);
             }
           }
         }
       }
-      if (!ok && leader) {
+      if (!ok) {
         for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
           mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, drain_limit);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ main MMA issuer (leader)
-    if (leader && lane == 0) {
-      int it = 0, local = 0, pit = 0;
+    // ------------------------------------------------------------ main MMA issuer
+    if (lane == 0) {
+      int it = 0, local = 0, kst = 0;
       bool ok = true;
-      for (int u = pair; u < p.num_units && ok; u += npairs) {
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const int sg = u / p.m_tiles;
         const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
         for (int nt = nt0; nt < nt1 && ok; ++nt, ++local) {
           const int b = local & 1;
-          if (!mbar_wait_cl(&acc_empty[b], ((local >> 1) & 1) ^ 1, wc)) {
+          if (!mbar_wait(&acc_empty[b], ((local >> 1) & 1) ^ 1, wc)) {
             ok = false;
             break;
           }
@@ -270,65 +265,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               const uint32_t layout = w == 64 ? LAYOUT_SW128 : (w == 32 ? LAYOUT_SW64 : LAYOUT_SW32);
               const uint32_t sbo = 8u * 2u * (uint32_t)w;
               for (int kk = 0; kk < w / 16; ++kk) {
-                mma_bf16_pair(d, make_sdesc(a_addr + 32 * kk, 16, sbo, layout),
-                              make_sdesc(b_addr + 32 * kk, 16, sbo, layout), IDESC_BF16, accum);
+                mma_bf16(d, make_sdesc(a_addr + 32 * kk, 16, sbo, layout), make_sdesc(b_addr + 32 * kk, 16, sbo, layout),
+                         IDESC_BF16, accum);
                 accum = 1;
               }
             } else {
-              // the stage's scale-factor atoms into tensor memory ahead of the MMAs
-              // that read them (the pipe keeps this thread's copies and MMAs in order)
-              const int ks = st - p.n_lr, h = ks & 1, slot = pit % SF_SLOTS;
-              const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
-              if (h == 0 && !mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc)) {
+              const int sb = kst & 1;
+              if (!mbar_wait(&sf_ready[sb], (kst >> 1) & 1, wc)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              const uint32_t sfa_s = smem_u32(sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES);
-              const uint32_t sfb_s = smem_u32(sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES);
-              const uint32_t sfa_t = tmem + SF_COL, sfb_t = sfa_t + 16;
+              const uint32_t sfa_t = tmem + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+              const uint32_t sfb_t = sfa_t + 16;
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                tmem_cp_32x128b_x4_pair(sfa_t + 4 * j, make_sdesc(sfa_s + j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-                tmem_cp_32x128b_x4_pair(sfb_t + 8 * j, make_sdesc(sfb_s + 2 * j * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-                tmem_cp_32x128b_x4_pair(sfb_t + 8 * j + 4,
-                                        make_sdesc(sfb_s + (2 * j + 1) * kSfAtomBytes, 0, 128, LAYOUT_NONE));
-              }
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                mma_nvf4_pair(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
-                              make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), IDESC_NVF4, sfa_t + 4 * j,
-                              sfb_t + 8 * j, accum);
+                mma_nvf4(d, make_sdesc(a_addr + 32 * j, 16, 1024, LAYOUT_SW128),
+                         make_sdesc(b_addr + 32 * j, 16, 1024, LAYOUT_SW128), IDESC_NVF4, sfa_t + 4 * j, sfb_t + 8 * j,
+                         accum);
                 accum = 1;
               }
-              if (last_of_pair) {
-                umma_commit_pair(&sfs_empty[slot], 3);
-                ++pit;
-              }
+              umma_commit(&sf_free[sb]);
+              ++kst;
             }
-            umma_commit_pair(&empty[s], 3);
+            umma_commit(&empty[s]);
           }
-          if (ok) umma_commit_pair(&acc_full[b], 3);
+          if (ok) umma_commit(&acc_full[b]);
         }
       }
-      umma_commit_pair(mma_done, 1);
+      umma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, drain_limit);
     }
   } else if (warp == SF_WARP) {
-    // ------------------------------------------------------------ scale-factor producer (both CTAs)
-    // Two K stages per slot: this CTA's 128 activation rows (atom tile 2 mt +
-    // rank) and all 192 weight rows; both CTAs' copies complete on the leader's barrier.
+    // ------------------------------------------------------------ scale-factor producer
     if (lane == 0) {
-      prefetch_tmap(&maps.sfa);
-      prefetch_tmap(&maps.sfb);
-      pdl_wait();
+      pdl_wait();  // the activation scales come from the previous kernel
       int pit = 0;
       bool ok = true;
       const int pairs_k = (p.k_stages + 1) / 2;
-      for (int u = pair; u < p.num_units && ok; u += npairs) {
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const int mt = u % p.m_tiles, sg = u / p.m_tiles;
         const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
-        const int at = 2 * mt + (int)rank;
         for (int nt = nt0; nt < nt1 && ok; ++nt) {
           for (int j = 0; j < pairs_k; ++j, ++pit) {
             const int slot = pit % SF_SLOTS;
@@ -338,105 +315,135 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
             uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
-            const uint32_t fbar = mapa_shared(smem_u32(&sfs_full[slot]), 0);
-            if (leader) mbar_arrive_expect_tx(&sfs_full[slot], 2u * (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
-            for (int h = 0; h < ns; ++h) {
-              tma_load_2d_pair(&maps.sfa, fbar, dst + h * SFA_BYTES, 0, at * p.katoms + 8 * j + 4 * h);
-              tma_load_2d_pair(&maps.sfb, fbar, dst + 2 * SFA_BYTES + h * SFB_BYTES, 0,
-                               (nt * p.katoms + 8 * j + 4 * h) * 2);
-            }
+            mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
+            const size_t oa = ((size_t)mt * p.katoms + 8 * j) * kSfAtomBytes;
+            const size_t ob = ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes;
+            if (SVDQ_INB(p.status, oa, ns * SFA_BYTES, p.sfa_bytes))
+              bulk_load(dst, p.sfa + oa, ns * SFA_BYTES, &sfs_full[slot]);
+            if (SVDQ_INB(p.status, ob, ns * SFB_BYTES, p.sfb_bytes))
+              bulk_load(dst + 2 * SFA_BYTES, p.sfb + ob, ns * SFB_BYTES, &sfs_full[slot]);
           }
         }
       }
-      if (!ok && leader) {
+      if (!ok) {
         for (int j = (pit > SF_SLOTS ? pit - SF_SLOTS : 0); j < pit; ++j)
           mbar_wait_drain(&sfs_full[j % SF_SLOTS], (j / SF_SLOTS) & 1, drain_limit);
       }
     }
-  } else if (warp == T_WARP) {
-    // ------------------------------------------------------------ L1'^T slices and t' MMAs
-    // Per tile: this CTA's rank/2 rows of L1'^T for the tile's 192 columns (three
-    // 64-column boxes, 128-byte swizzle) into its slot; the leader then issues
-    // t' += bf16(x^'_tile) . L1'[tile] (M = 256, N = rank, K = 192) once both
-    // CTAs' epilogues have written their x^' tiles, and releases the x^' tiles
-    // and the L1' slots when those MMAs complete.
-    if (lane == 0 && p.rank_dn > 0) {
-      bool ok = true;
-      int tt = 0, ut = 0;  // tiles and units done
-      const uint32_t l1bar = mapa_shared(smem_u32(l1_full), 0);
-      const uint32_t idesc_t = idesc_bf16_f32(2 * BM, p.rank_dn);
-      for (int u = pair; u < p.num_units && ok; u += npairs, ++ut) {
-        const int sg = u / p.m_tiles;
-        const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
-        for (int nt = nt0; nt < nt1 && ok; ++nt, ++tt) {
-          // the slot is free once the previous tile's t' MMAs completed
-          if (!mbar_wait_cl(xt_free, (tt & 1) ^ 1, wc)) {
-            ok = false;
-            break;
+  } else if (warp >= 10 && warp <= 13) {
+    // ------------------------------------------------------------ scale-factor movers
+    // Warp q owns tensor-memory lanes 32q..32q+31; lane l writes, for every
+    // 128-row atom of the stage, the atom's 16-byte row l into 4 consecutive
+    // columns (the replicated layout the block-scaled MMA reads).
+    const int q = warp & 3;
+    int kst = 0, pit = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+      const int sg = u / p.m_tiles;
+      const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+      for (int nt = nt0; nt < nt1 && ok; ++nt) {
+        for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
+          const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
+          const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
+          if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
+          ok = ok && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+          if (!ok) break;
+          const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
+          const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
+          uint32_t ra[16], rb[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 a = *(const uint4*)(sfa_s + j * kSfAtomBytes + lane * 16);
+            ra[4 * j] = a.x; ra[4 * j + 1] = a.y; ra[4 * j + 2] = a.z; ra[4 * j + 3] = a.w;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint4 b4 = *(const uint4*)(sfb_s + (2 * j + hh) * kSfAtomBytes + lane * 16);
+              rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
+            }
           }
-          if (leader) mbar_arrive_expect_tx(l1_full, 2u * 3u * (uint32_t)rh * 128u);
-          for (int hb = 0; hb < 3; ++hb)
-            tma_load_2d_pair(&maps.l1dn, l1bar, l1s + hb * L1_MAX_ROWS * 128, nt * BN + 64 * hb, (int)rank * rh);
-          if (leader) {
-            if (!mbar_wait_cl(l1_full, tt & 1, wc) || !mbar_wait_cl(xt_full, tt & 1, wc)) {
-              ok = false;
-              break;
-            }
-            if (nt == nt0 && !mbar_wait_cl(tp_empty, (ut & 1) ^ 1, wc)) {  // the unit's t' was read out
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(xt), b0 = smem_u32(l1s);
-            for (int kk = 0; kk < 12; ++kk) {
-              const uint32_t hb = kk >> 2, koff = (kk & 3) * 32;
-              mma_bf16_pair(tmem + TP_COL, make_sdesc(a0 + hb * (BM * 128) + koff, 16, 1024, LAYOUT_SW128),
-                            make_sdesc(b0 + hb * (L1_MAX_ROWS * 128) + koff, 16, 1024, LAYOUT_SW128), idesc_t,
-                            (nt > nt0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit_pair(xt_free, 3);
-            if (nt + 1 == nt1) umma_commit_pair(tp_full, 3);
+          const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
+          tmem_st_32x32b_x16(tq, ra);
+          tmem_st_32x32b_x32(tq + 16, rb);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sf_ready[sb]);
+            if (last_of_pair) mbar_arrive(&sfs_empty[slot]);
           }
-        }
-      }
-      if (leader) {
-        umma_commit_pair(tdone, 1);
-        mbar_wait_drain(tdone, 0, drain_limit);
-      } else if (!ok) {
-        // the peer's slice copies complete on the leader's barrier; give them time to land
-        const unsigned long long t0 = clock64();
-        while ((unsigned long long)clock64() - t0 < (1ull << 16)) {
+          if (last_of_pair) ++pit;
         }
       }
     }
+  } else if (warp == T_WARP) {
+    // ------------------------------------------------------------ L1'^T slices and t' MMAs
+    // Per tile: the rank rows of L1'^T for the tile's 192 columns (three
+    // 64-column boxes, 128-byte swizzle) into the slot; once the epilogue has
+    // written the tile's x^', t' += bf16(x^'_tile) . L1'[tile] (M = 128,
+    // N = rank, K = 192); the x^' tile and the slot are free when those MMAs
+    // complete.
+    if (lane == 0 && p.rank_dn > 0) {
+      prefetch_tmap(&maps.l1dn);
+      bool ok = true;
+      int tt = 0, ut = 0;
+      const uint32_t idesc_t = idesc_bf16_f32(BM, p.rank_dn);
+      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++ut) {
+        const int sg = u / p.m_tiles;
+        const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
+        for (int nt = nt0; nt < nt1 && ok; ++nt, ++tt) {
+          if (!mbar_wait(xt_free, (tt & 1) ^ 1, wc)) {  // the previous tile's t' MMAs completed
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(l1_full, 3u * (uint32_t)p.rank_dn * 128u);
+          for (int hb = 0; hb < 3; ++hb)
+            tma_load_2d(&maps.l1dn, l1_full, l1s + hb * L1_MAX_ROWS * 128, nt * BN + 64 * hb, 0);
+          if (!mbar_wait(l1_full, tt & 1, wc) || !mbar_wait(xt_full, tt & 1, wc)) {
+            ok = false;
+            break;
+          }
+          if (nt == nt0 && !mbar_wait(tp_empty, (ut & 1) ^ 1, wc)) {  // the unit's t' was read out
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(xt), b0 = smem_u32(l1s);
+          for (int kk = 0; kk < 12; ++kk) {
+            const uint32_t hb = kk >> 2, koff = (kk & 3) * 32;
+            mma_bf16(tmem + TP_COL, make_sdesc(a0 + hb * (BM * 128) + koff, 16, 1024, LAYOUT_SW128),
+                     make_sdesc(b0 + hb * (L1_MAX_ROWS * 128) + koff, 16, 1024, LAYOUT_SW128), idesc_t,
+                     (nt > nt0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(xt_free);
+          if (nt + 1 == nt1) umma_commit(tp_full);
+        }
+      }
+      umma_commit(tdone);
+      mbar_wait_drain(tdone, 0, drain_limit);
+    }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9, both CTAs)
+    // ------------------------------------------------------------ epilogue (warps 2-9)
     pdl_wait();  // g_x and the down layer's workspace belong to the stream's order
     const int e = warp - 2;         // 0..7
     const int q = warp & 3;         // tensor-memory lane quarter
     const int half = e >> 2;        // columns 96*half .. 96*half + 95 of the tile
     const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;
-    const uint32_t empty_cl0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-    const uint32_t empty_cl1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-    const uint32_t xtfull_cl = mapa_shared(smem_u32(xt_full), 0);
-    const uint32_t tpempty_cl = mapa_shared(smem_u32(tp_empty), 0);
-    const int row = 32 * q + lane;  // row of this CTA's 128-row tile
+    const int row = 32 * q + lane;  // row of the 128-row tile
     int local = 0, tt = 0, ut = 0;
     bool ok = true;
-    for (int u = pair; u < p.num_units && ok; u += npairs, ++ut) {
+    for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++ut) {
       const int mt = u % p.m_tiles, sg = u / p.m_tiles;
       const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
-      const int rb = 2 * mt + (int)rank;  // 128-row block
-      const int64_t m = (int64_t)rb * BM + row;
+      const int64_t m = (int64_t)mt * BM + row;
       const bool live = m < p.M;
       for (int nt = nt0; nt < nt1 && ok; ++nt, ++local, ++tt) {
         const int b = local & 1;
-        if (!mbar_wait_cl(&acc_full[b], (local >> 1) & 1, wc)) {
+        if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) {
           ok = false;
           break;
         }
         // the x^' tile may be overwritten once the previous tile's t' MMAs completed
-        if (p.rank_dn > 0 && !mbar_wait_cl(xt_free, (tt & 1) ^ 1, wc)) {
+        if (p.rank_dn > 0 && !mbar_wait(xt_free, (tt & 1) ^ 1, wc)) {
           ok = false;
           break;
         }
@@ -460,7 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           if (blk == 5) {  // this warp's 96 accumulator columns are in registers
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(b ? empty_cl1 : empty_cl0);
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
           }
           float2 v[8];
           uint32_t hbits[8];
@@ -507,7 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               xb[j] = *(const uint32_t*)&hx;
             }
             const int col = 96 * half + 16 * blk;          // tile column of the block
-            const int hb = col >> 6, ch = (col & 63) >> 3;  // 64-column half, 16-byte chunk in the row
+            const int hb = col >> 6, ch = (col & 63) >> 3;  // 64-column block, 16-byte chunk in the row
             uint8_t* rowp = xt + hb * (BM * 128) + row * 128;
             *(uint4*)(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(xb[0], xb[1], xb[2], xb[3]);
             *(uint4*)(rowp + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(xb[4], xb[5], xb[6], xb[7]);
@@ -516,7 +523,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (p.rank_dn > 0) {
           fence_proxy_async_smem();  // x^' tile -> tensor core
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(xtfull_cl);
+          if (lane == 0) mbar_arrive(xt_full);
         }
         if (live) {
           // scale bytes of blocks blk0 .. blk0 + 5 (four consecutive blocks share an atom word)
@@ -534,7 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       // ------------------------------------------------------------ the unit's t' partial
       if (ok && p.rank_dn > 0 && half == 0) {
-        if (!mbar_wait_cl(tp_full, ut & 1, wc)) {
+        if (!mbar_wait(tp_full, ut & 1, wc)) {
           ok = false;
           break;
         }
@@ -546,12 +553,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tpempty_cl);
+        if (lane == 0) mbar_arrive(tp_empty);
         float acc[32];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           acc[j] = __uint_as_float(r0[j]);
-          acc[16 + j] = __uint_as_float(r1[j]);
+          acc[16 + j] = p.rank_dn > 16 ? __uint_as_float(r1[j]) : 0.f;
         }
         const int R = p.rank_dn;
         if (live && p.S > 1) {
@@ -577,9 +584,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         __threadfence();
         __syncwarp();
         // the last of the S units to finish these 32 rows adds the partials in group order
-        int* cnt = p.counters + 4 * rb + q;
+        int* cnt = p.counters + 4 * mt + q;
         if (lane == 0)
-          ticket[q] = SVDQ_INB(p.status, (size_t)(4 * rb + q) * 4, 4, p.cnt_bytes) ? atomicAdd(cnt, 1) : -1;
+          ticket[q] = SVDQ_INB(p.status, (size_t)(4 * mt + q) * 4, 4, p.cnt_bytes) ? atomicAdd(cnt, 1) : -1;
         __syncwarp();
         if (ticket[q] == p.S - 1) {
           __threadfence();
@@ -610,18 +617,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   __syncwarp();
   tc_fence_before();
-  cluster_sync();
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
-}
-
-int pair_units_groups(int m_tiles, int n_tiles, int npairs, int max_groups) {
-  int S = (npairs + m_tiles - 1) / m_tiles;
-  if (S > max_groups) S = max_groups;
-  if (S > n_tiles) S = n_tiles;
-  return S < 1 ? 1 : S;
 }
 
 }  // namespace
@@ -644,7 +644,7 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   st = encode_tmap_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.codes, (uint64_t)K / 2, (uint64_t)M,
                       (uint64_t)K / 2, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != SVDQ_OK) return st;
-  maps.b = L->map_w_half;
+  maps.b = L->map_w;
   FParams p{};
   const LowRankChunks ch = lowrank_chunks(r);
   p.n_lr = ch.n;
@@ -661,27 +661,19 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
       st = encode_tmap_2d(&maps.t[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.t, (uint64_t)r, (uint64_t)M,
                           (uint64_t)r * 2, widths[i], BM, swz[i]);
       if (st != SVDQ_OK) return st;
-      maps.l2[i] = L->map_l2_half[i];
+      maps.l2[i] = L->map_l2[i];
     }
   }
   const int rd = D->rank;
-  if (rd > 0) {  // L1'^T [rd, N] bf16: per CTA rd/2 rows, 64 columns per box
+  if (rd > 0) {  // L1'^T [rd, N] bf16, 64 columns per box
     st = encode_tmap_2d(&maps.l1dn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D->L1t, (uint64_t)D->K, (uint64_t)rd,
-                        (uint64_t)D->K * 2, 64, (uint32_t)rd / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+                        (uint64_t)D->K * 2, 64, (uint32_t)rd, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != SVDQ_OK) return st;
   }
-  // scale-factor atoms (512 B each) as rows of 128 u32 (see k_gemm_nvfp4_pair)
-  st = encode_tmap_2d(&maps.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, ws + w.scales, 128,
-                      (uint64_t)((M + 2 * BM - 1) / (2 * BM)) * 2 * (K / 64), kSfAtomBytes, 128, 4,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (st != SVDQ_OK) return st;
-  st = encode_tmap_2d(&maps.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, L->wscales, 128,
-                      (uint64_t)((N + BN - 1) / BN) * (K / 64) * 2, kSfAtomBytes, 128, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (st != SVDQ_OK) return st;
   p.M = (int)M;
   p.N = N;
   p.K = K;
-  p.m_tiles = (int)((M + 2 * BM - 1) / (2 * BM));
+  p.m_tiles = (int)((M + BM - 1) / BM);
   p.n_tiles = N / BN;
   p.k_stages = K / kKStage;
   p.katoms = K / 64;
@@ -702,11 +694,13 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.tpart = (float*)(wsd + wd.tpart);
   // one counter per 32-row group in the down workspace's first-pass slots (idle:
   // the down layer has a static activation scale); zero between calls
-  if (4 * ((M + BM - 1) / BM) > kAmaxSlots) return SVDQ_ERR_INVALID_ARG;
+  if (4 * (int64_t)p.m_tiles > kAmaxSlots) return SVDQ_ERR_INVALID_ARG;
   p.counters = (int*)(wsd + wd.amax);
   p.H = (uint16_t*)H;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
+  p.sfa_bytes = w.scales_bytes;
+  p.sfb_bytes = L->off.total - L->off.wscales;
   p.codes_dn_bytes = wd.codes_bytes;
   p.scales_dn_bytes = wd.scales_bytes;
   p.t_dn_bytes = wd.t_bytes;
@@ -715,37 +709,22 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.H_bytes = (size_t)M * N * 2;
 
   const size_t smem = 1024 + (size_t)SMEM_BYTES + 512;
-  static int attr_done[64] = {0};
-  const int dev = L->device;
-  if (dev < 0 || dev >= 64) return SVDQ_ERR_INVALID_ARG;
-  if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(k_gemm_gelu_quant, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return SVDQ_ERR_CUDA;
-    attr_done[dev] = 1;
-  }
-  static int maxc_cache[64] = {0};
-  if (!maxc_cache[dev]) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 74, 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_gelu_quant, &cfg) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      return SVDQ_ERR_UNSUPPORTED_DEVICE;
-    }
-    maxc_cache[dev] = n;
-  }
-  const int npairs_max = maxc_cache[dev];
-  // work units: (256-row M tile) x (one of S groups of N tiles); the t' partial
-  // sums of the groups land in the down layer's split-K area (wd.nslices of them)
-  const int S = pair_units_groups(p.m_tiles, p.n_tiles, npairs_max, rd > 0 ? wd.nslices : p.n_tiles);
+  if (cudaFuncSetAttribute(k_gemm_gelu_quant, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  const int sms = device_sm_count(L->device);
+  // work units: (128-row M tile) x (one of S contiguous groups of N tiles); the
+  // t' partial sums of the groups land in the down layer's split-K area
+  // (wd.nslices of them)
+  int S = (sms + p.m_tiles - 1) / p.m_tiles;
+  const int max_groups = rd > 0 ? wd.nslices : p.n_tiles;
+  if (S > max_groups) S = max_groups;
+  if (S > p.n_tiles) S = p.n_tiles;
+  if (S < 1) S = 1;
   if (rd > 0 && S > 1 && wd.tpart_bytes < (size_t)S * M * rd * 4) return SVDQ_ERR_INVALID_ARG;
   p.S = S;
   p.num_units = p.m_tiles * S;
-  const int npairs = p.num_units < npairs_max ? p.num_units : npairs_max;
-  if (launch_pdl(k_gemm_gelu_quant, dim3(2 * npairs), dim3(THREADS), smem, stream, maps, p) != cudaSuccess)
+  const int grid = p.num_units < sms ? p.num_units : sms;
+  if (launch_pdl(k_gemm_gelu_quant, dim3(grid), dim3(THREADS), smem, stream, maps, p) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }

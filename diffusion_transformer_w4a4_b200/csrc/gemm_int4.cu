@@ -407,17 +407,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_int4(const __grid_constant_
   }
 }
 
-int sm_count_i4(int dev) {
-  static int cache[64] = {0};
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cache[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
-  }
-  return cache[dev];
-}
-
 }  // namespace
 
 int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const Workspace& w, int32_t* acc_dbg,
@@ -467,7 +456,7 @@ int launch_gemm_int4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, const
   p.acc_dbg = acc_dbg;
   p.status = (int*)(ws + w.status);
   p.limit = wait_limit_cycles();
-  const int grid = p.num_tiles < sm_count_i4(L->device) ? p.num_tiles : sm_count_i4(L->device);
+  const int grid = p.num_tiles < device_sm_count(L->device) ? p.num_tiles : device_sm_count(L->device);
   if (acc_dbg) {
     if (cudaFuncSetAttribute(k_gemm_int4<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
         cudaSuccess)

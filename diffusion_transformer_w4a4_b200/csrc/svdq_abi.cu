@@ -19,6 +19,17 @@ unsigned long long wait_limit_cycles() {
   return v ? v : (1ull << 31);
 }
 
+int device_sm_count(int dev) {
+  static std::atomic<int> cache[64];
+  if (dev < 0 || dev >= 64) return 148;
+  int n = cache[dev].load();
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n);
+  }
+  return n;
+}
+
 LowRankChunks lowrank_chunks(int rank) {
   LowRankChunks c{};
   int off = 0;
@@ -73,8 +84,8 @@ Workspace workspace_layout(int64_t N, int64_t K, int rank, int fmt, int64_t M) {
   w.codes_bytes = fmt == SVDQ_NVFP4_G16 ? (size_t)M * K / 2 : (size_t)M * K;
   o = align_up(o + w.codes_bytes, kAlign);
   w.scales = o;
-  if (fmt == SVDQ_NVFP4_G16)  // whole 256-row tiles: the pair GEMM reads both halves' atoms
-    w.scales_bytes = (size_t)((M + kPairBM - 1) / kPairBM) * 2 * (size_t)(K / 64) * kSfAtomBytes;
+  if (fmt == SVDQ_NVFP4_G16)  // whole 128-row atoms
+    w.scales_bytes = (size_t)((M + kSfAtomRows - 1) / kSfAtomRows) * (size_t)(K / 64) * kSfAtomBytes;
   else
     w.scales_bytes = (size_t)(K / 64) * (size_t)int4_scale_ld(M) * 2;
   o = align_up(o + w.scales_bytes, kAlign);
@@ -309,9 +320,6 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   if (fmt == SVDQ_NVFP4_G16) {  // 256 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
                        (uint64_t)K / 2, 128, kNvfp4BN, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (e == SVDQ_OK)
-      e = encode_tmap_2d(&L->map_w_half, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K / 2, (uint64_t)N,
-                         (uint64_t)K / 2, 128, kNvfp4BN / 2, CU_TENSOR_MAP_SWIZZLE_128B);
   } else  // 128 E4M3 codes (128 B) per row per stage, swizzled for the MMA
     e = encode_tmap_2d(&L->map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wcodes, (uint64_t)K, (uint64_t)N, (uint64_t)K,
                        128, kInt4BN, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -326,9 +334,6 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
       if (widths[i] > rank) continue;
       e = encode_tmap_2d(&L->map_l2[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, (uint64_t)rank, (uint64_t)N,
                          (uint64_t)rank * 2, widths[i], bn, swz[i]);
-      if (e == SVDQ_OK && fmt == SVDQ_NVFP4_G16)
-        e = encode_tmap_2d(&L->map_l2_half[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, (uint64_t)rank,
-                           (uint64_t)N, (uint64_t)rank * 2, widths[i], kNvfp4BN / 2, swz[i]);
     }
   }
   if (e != SVDQ_OK) {

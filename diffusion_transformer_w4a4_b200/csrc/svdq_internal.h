@@ -17,7 +17,6 @@ namespace svdq {
 constexpr int kKStage = 256;       // K elements per pipeline stage / per quantizer chunk
 constexpr int kGemmBM = 128;       // GEMM tile rows (tokens), = tcgen05 M
 constexpr int kNvfp4BN = 192;      // NVFP4 GEMM tile columns (output features)
-constexpr int kPairBM = 256;       // NVFP4 CTA-pair GEMM tile rows (128 per CTA)
 constexpr int kInt4BN = 128;       // INT4 GEMM tile columns
 constexpr int kSfAtomRows = 128;   // rows per tensor-core scale-factor atom
 constexpr int kSfAtomBytes = 512;  // 128 rows x 4 blocks of 16
@@ -134,10 +133,6 @@ struct svdq_layer {
   CUtensorMap map_w;         // weight codes
   CUtensorMap map_l1;        // L1^T, box {64, rank}, 128B swizzle (quantizer)
   CUtensorMap map_l2[3];     // L2^T chunks of width 64/32/16
-  // NVFP4, CTA-pair GEMM: each CTA of a pair loads half of a 192-row weight
-  // tile (96 rows) of the codes and of the L2^T chunks
-  CUtensorMap map_w_half;
-  CUtensorMap map_l2_half[3];
 };
 
 namespace svdq {
@@ -157,6 +152,7 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
 
 unsigned long long wait_limit_cycles();
+int device_sm_count(int dev);  // multiprocessor count, cached per device (148 if the query fails)
 
 // Kernel launchers (return svdq_status).
 // dynamic activation scale: grid of the amax pass (its CTA count is the number

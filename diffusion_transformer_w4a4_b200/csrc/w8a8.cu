@@ -283,17 +283,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_w8a8(const __grid_constant_
   }
 }
 
-int w8_sm_count(int dev) {
-  static int cache[64] = {0};
-  if (dev < 0 || dev >= 64) return 148;
-  if (!cache[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
-  }
-  return cache[dev];
-}
-
 int launch_w8_quantize(const svdq_w8a8_layer* L, const void* X, int64_t M, uint8_t* ws, cudaStream_t stream) {
   const W8Ws w = w8_ws_layout(M, L->K);
   int st = launch_act_amax_raw(X, M, L->K, nullptr, (float*)(ws + w.slots), stream);
@@ -302,7 +291,7 @@ int launch_w8_quantize(const svdq_w8a8_layer* L, const void* X, int64_t M, uint8
   act_amax_grid(M, L->K, &gx, &gy);
   const int64_t nvec16 = M * L->K / 16;
   int64_t grid = (nvec16 + kQuantThreads - 1) / kQuantThreads;
-  const int64_t cap = 8 * (int64_t)w8_sm_count(L->device);
+  const int64_t cap = 8 * (int64_t)device_sm_count(L->device);
   if (grid > cap) grid = cap;
   k_w8_quantize<<<(unsigned)grid, kQuantThreads, 0, stream>>>((const uint4*)X, nvec16, (const float*)(ws + w.slots),
                                                               gx * gy, (uint4*)(ws + w.codes),
@@ -344,7 +333,7 @@ int launch_w8_gemm(const svdq_w8a8_layer* L, int64_t M, void* Y, uint8_t* ws, cu
       attr_set[L->device] = true;
     }
   }
-  const int sms = w8_sm_count(L->device);
+  const int sms = device_sm_count(L->device);
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   k_gemm_w8a8<<<grid, THREADS, SMEM_BYTES, stream>>>(maps, p);
   return cudaPeekAtLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;

@@ -212,7 +212,8 @@ svdq_status svdq_int4_group_acc(const svdq_layer* layer, int64_t M, void* ws, si
 /* "Hugging Face встроила Nunchaku в Diffusers ..." (paragraph on Nunchaku
  * Lite): the engine's speed comes from fused, model-specific kernels.  Here the
  * up-projection's GEMM epilogue computes, per output element,
- *     h = bf16(y_up),   x' = bf16(GELU(h)),   GELU(h) = h/2 (1 + erf(h/sqrt 2)) in binary32,
+ *     h = bf16(y_up),   x' = bf16(GELU(h)),   GELU(h) = h/2 (1 + erf(h/sqrt 2)),
+ * evaluated in binary32 as h/2 erfc(-h/sqrt 2) (no cancellation for h < 0),
  * and quantizes x' as the down-projection's input exactly as svdq_quantize_act
  * would (x^' = f32(x') inv_lambda', E4M3 block scales and E2M1 codes under the
  * down layer's static g_x', t' = bf16(bf16(x^') L1')), writing codes, scales and
@@ -224,7 +225,8 @@ svdq_status svdq_mlp_fusable(const svdq_layer* up, const svdq_layer* down);
 
 /* After svdq_quantize_act(up, X, M, ws_up, ...): the fused up-projection GEMM.
  * ws_up / ws_dn are the two layers' workspaces for M tokens (device, 256-byte
- * aligned; ws_dn initialised once with svdq_workspace_init); H, if not NULL, is
+ * aligned; ws_dn initialised once with svdq_workspace_init; M <= 32768, else
+ * SVDQ_ERR_INVALID_ARG); H, if not NULL, is
  * a device bf16 [M, up.N] array (16-byte aligned) that receives x' (a parity
  * export; costs one extra write).  Then svdq_gemm(down, M, Y, ws_dn, ...) gives
  * the block's MLP output.  Asynchronous on `stream`; device-side errors land in

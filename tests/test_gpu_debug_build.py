@@ -1,5 +1,5 @@
 """The bounds-checked debug variant on the GPU: run in a child process with
-SVDQ_LIBRARY=debug, the NVFP4 (single-CTA and CTA-pair GEMM paths), INT4 and
+SVDQ_LIBRARY=debug, the NVFP4 (one and several 128-row tiles), INT4 and
 fused-MLP forwards at ragged shapes report no bounds error (status 0) and give
 outputs bit-identical to the release library's."""
 import os
@@ -21,7 +21,7 @@ import diffusion_transformer_w4a4_b200 as svdq
 from svdq_cases import GpuLayer, oracle_layer
 torch.cuda.set_device(0)
 out = {"debug": svdq.svdq_debug_build()}
-for name, (M, K, N, r, fmt) in {"nvfp4_small": (100, 512, 400, 32, "nvfp4"), "nvfp4_pair": (300, 1024, 576, 48, "nvfp4"),
+for name, (M, K, N, r, fmt) in {"nvfp4_small": (100, 512, 400, 32, "nvfp4"), "nvfp4_multi": (300, 1024, 576, 48, "nvfp4"),
                                 "int4": (300, 512, 400, 32, "int4")}.items():
     X, W, b, prep = oracle_layer(wl.small_layer(M, K, N, r, fmt, layer_id=M + K))
     gl = GpuLayer(prep)
@@ -56,7 +56,7 @@ def test_debug_variant_matches_release(tmp_path):
     rel = _run(tmp_path, "release")
     dbg = _run(tmp_path, "debug")
     assert int(rel["debug"]) == 0 and int(dbg["debug"]) == 1
-    for k in ("nvfp4_small", "nvfp4_pair", "int4", "fused"):
+    for k in ("nvfp4_small", "nvfp4_multi", "int4", "fused"):
         assert int(dbg[k + "_status"]) == 0, (k, int(dbg[k + "_status"]))
         assert int(rel[k + "_status"]) == 0, k
         np.testing.assert_array_equal(dbg[k], rel[k], err_msg=k)

@@ -1,7 +1,7 @@
 """Guard bands around every buffer the kernels write: the output Y and the
 caller workspace are carved out of larger device buffers whose margins hold a
 known byte pattern; after a forward at ragged token / feature counts (partial
-128- and 256-row tiles, partial 192- and 128-column tiles) the margins must be
+128-row tiles, partial 192- and 128-column tiles) the margins must be
 untouched and Y must equal the forward into an ordinary buffer bit for bit."""
 import numpy as np
 import pytest
