@@ -2,7 +2,7 @@
 // quantizer fused into its epilogue (cross-layer fusion of the MLP pair).
 //
 //   h  = bf16( g_x g_w [ sum_blocks (s_x s_w)(qx . qw) + t . L2/(g_x g_w) ] + b )   (the up layer's y)
-//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) = h/2 erfc(-h / sqrt 2) in binary32
+//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) in binary32 (gelu_erf)
 //   x^' = f32(x') * inv_lambda'                                                     (the down layer's input)
 //   codes', E4M3 block scales'  of x^' (blocks of 16, static g_x'),  t' = bf16( bf16(x^') . L1' )
 //
@@ -27,9 +27,13 @@
 //   warps 2-9   epilogue: two warps per tensor-memory lane quarter, 96 columns each
 //   warps 10-13 scale-factor movers             warp 14  scale-factor producer
 //   warp 15     L1'^T slice loader and t' MMA issuer, per tile
-// Tensor memory (512 columns): two 192-column accumulators, two 48-column
-// scale-factor buffers and the 32-column t' accumulator, so the down layer's
-// rank is at most 32.  Every wait is bounded; no load uses cluster multicast.
+// An epilogue thread's codes and scales would be scattered stores (32 rows per
+// warp instruction), so the tile's codes (128 x 96 B) and its three scale atoms
+// are staged in shared memory and written by one thread with a TMA tensor store
+// and one bulk copy.  Tensor memory (512 columns): two 192-column accumulators,
+// two 48-column scale-factor buffers and the 32-column t' accumulator, so the
+// down layer's rank is at most 32.  Every wait is bounded; no load uses cluster
+// multicast.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -48,18 +52,21 @@ constexpr int B_BYTES = BN * 128;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int SFA_BYTES = 4 * kSfAtomBytes;
 constexpr int SFB_BYTES = 4 * 2 * kSfAtomBytes;
-constexpr int SF_SLOTS = 2;
-constexpr int SF_SLOT_BYTES = 2 * (SFA_BYTES + SFB_BYTES);
+constexpr int SF_SLOTS = 3;
+constexpr int SF_SLOT_BYTES = SFA_BYTES + SFB_BYTES;  // one K stage: [SFA | SFB]
 constexpr int XT_BYTES = 3 * BM * 128;  // bf16 x^' tile: three 64-column blocks, 128B-swizzled
 constexpr int L1_MAX_ROWS = 32;         // rank rows of L1'^T (rank <= 32)
 constexpr int L1_BYTES = 3 * L1_MAX_ROWS * 128;
+constexpr int CST_BYTES = BM * BN / 2;  // the tile's down-layer codes, row-major (96 B per row)
+constexpr int SST_BYTES = 3 * kSfAtomBytes;  // the tile's 12 block scales per row: three atoms
 constexpr int THREADS = 512;
 constexpr int SF_WARP = 14, T_WARP = 15;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 2 * BN;     // 384: two buffers of [SFA 16 | SFB 32] columns
 constexpr uint32_t SF_BUF_COLS = 48;
 constexpr uint32_t TP_COL = SF_COL + 2 * SF_BUF_COLS;  // 480
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + XT_BYTES + L1_BYTES;
+constexpr int SMEM_BYTES =
+    STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + XT_BYTES + L1_BYTES + 2 * (CST_BYTES + SST_BYTES);
 constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
 static_assert(STAGE_BYTES % 1024 == 0 && SF_SLOT_BYTES % 1024 == 0 && XT_BYTES % 1024 == 0, "alignment");
@@ -68,6 +75,7 @@ static_assert(TP_COL + 32 <= TMEM_COLS, "tensor memory budget");
 
 struct FusedMaps {
   CUtensorMap a, b, t[3], l2[3], l1dn;
+  CUtensorMap codes_dn;  // the down layer's activation codes [M, N/2] bytes, box 96 x 128 (stores)
 };
 
 struct FParams {
@@ -83,7 +91,6 @@ struct FParams {
   float g_w;
   const float* inv_lambda_dn;
   float den_dn, inv_g_dn;   // 6 g_x' and 1/g_x' of the down layer (powers of two: exact)
-  uint8_t* codes_dn;        // [M, N/2]
   uint8_t* scales_dn;       // atom layout, 128-row tiles, katoms_dn
   uint16_t* t_dn;           // [M, rank_dn]
   float* tpart;             // [S, M, rank_dn]
@@ -92,7 +99,7 @@ struct FParams {
   int* status;
   unsigned long long limit;
   // extents in bytes (debug bounds checks)
-  size_t sfa_bytes, sfb_bytes, codes_dn_bytes, scales_dn_bytes, t_dn_bytes, tpart_bytes, cnt_bytes, H_bytes;
+  size_t sfa_bytes, sfb_bytes, scales_dn_bytes, t_dn_bytes, tpart_bytes, cnt_bytes, H_bytes;
 };
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
@@ -127,8 +134,88 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-// bf16 round-to-nearest-even of a binary32 value, returned as the binary32 it denotes
-__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// GELU(h) = h Phi(h) = h/2 (1 + erf(h / sqrt 2)) in binary32, branch-free.  With
+// x = |h| / sqrt 2:  h >= 0: h - (h/2) erfc(x);  h < 0: (h/2) erfc(x)  (no
+// cancellation on either side).  erfc(x) = t exp(-x^2 + P(t)), t = 1/(1 + x/2):
+// the Chebyshev-fit form of Press et al., "Numerical Recipes" (2nd ed., sec.
+// 6.2), with P a degree-9 polynomial fitted by least squares to
+// log(erfc(x) e^(x^2) / t) at Chebyshev nodes in t in (0, 1], coefficients rounded
+// to binary32 (relative error of erfc below 1.2e-7 before rounding).  exp(y) for
+// y < -80 is taken as exp(y + 64 ln 2) 2^-64 so that tails below the binary32
+// normal range round once, as bf16 keeps them.  A table of the correctly rounded
+// bf16 results (the input is a bf16 value) measured slower: its random reads
+// cost more than the arithmetic.
+__device__ __forceinline__ float gelu_erf(float h) {
+  const float x = fabsf(h) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.5f, x, 1.0f));
+  float p = 1.708930433e-01f;
+  p = fmaf(p, t, -8.222485185e-01f);
+  p = fmaf(p, t, 1.488708496e+00f);
+  p = fmaf(p, t, -1.135414600e+00f);
+  p = fmaf(p, t, 2.790049911e-01f);
+  p = fmaf(p, t, -1.863418519e-01f);
+  p = fmaf(p, t, 9.679660201e-02f);
+  p = fmaf(p, t, 3.740904033e-01f);
+  p = fmaf(p, t, 1.000023723e+00f);
+  p = fmaf(p, t, -1.265512228e+00f);
+  const float y = fmaf(-x, x, p);  // -x^2 + P(t), rounded once
+  const bool low = y < -80.0f;
+  float te = t * __expf(low ? y + 44.3614195558365f : y);
+  te = low ? te * 0x1p-64f : te;   // t exp(y): one rounding into the subnormal range
+  const float q = (0.5f * h) * te;  // (h/2) erfc(x)
+  return __float_as_int(h) < 0 ? q : (te == 0.0f ? h : h - q);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// gelu_erf for two elements with packed f32x2 arithmetic, for inputs h >= -12.5
+// (and +inf, NaN): there exp(-x^2 + P) >= 2^-122 stays normal, so the subnormal
+// scaling is not needed, and with 1/t and the exponent taken in base 2
+// (-h^2 log2(e)/2 + P(t) log2(e)) it costs about half the instructions.  h is
+// clamped to 16 inside the erfc part (h Phi(h) rounds to h from 8 up), and the
+// h >= 0 side is h (1 - erfc/2), so +inf, -0 and NaN come out right without tests
+// of their own.
+__device__ __forceinline__ float2 gelu_erf2(float2 h) {
+  constexpr float L2E = 1.4426950408889634f;
+  const float2 hc = make_float2(fminf(h.x, 16.0f), fminf(h.y, 16.0f));
+  const float2 d = __ffma2_rn(make_float2(fabsf(hc.x), fabsf(hc.y)), make_float2(0.35355339059327376f, 0.35355339059327376f),
+                              make_float2(1.0f, 1.0f));  // 1 + |h| / (2 sqrt 2)
+  const float2 t = make_float2(rcp_approx(d.x), rcp_approx(d.y));
+  float2 p = make_float2(1.708930433e-01f * L2E, 1.708930433e-01f * L2E);
+#define SVDQ_H(c) p = __ffma2_rn(p, t, make_float2((c) * L2E, (c) * L2E))
+  SVDQ_H(-8.222485185e-01f);
+  SVDQ_H(1.488708496e+00f);
+  SVDQ_H(-1.135414600e+00f);
+  SVDQ_H(2.790049911e-01f);
+  SVDQ_H(-1.863418519e-01f);
+  SVDQ_H(9.679660201e-02f);
+  SVDQ_H(3.740904033e-01f);
+  SVDQ_H(1.000023723e+00f);
+  SVDQ_H(-1.265512228e+00f);
+#undef SVDQ_H
+  const float2 y = __ffma2_rn(__fmul2_rn(hc, make_float2(-0.5f * L2E, -0.5f * L2E)), hc, p);  // log2 of erfc / t
+  const float2 te = __fmul2_rn(t, make_float2(ex2_approx(y.x), ex2_approx(y.y)));  // erfc(|h| / sqrt 2)
+  const float2 ht = __fmul2_rn(te, make_float2(0.5f, 0.5f));
+  const float2 q = __fmul2_rn(h, ht);                                        // h < 0: h erfc / 2
+  const float2 r = __fmul2_rn(h, __fadd2_rn(make_float2(1.0f, 1.0f), make_float2(-ht.x, -ht.y)));  // h (1 - erfc / 2)
+  return make_float2(h.x < 0.0f ? q.x : r.x, h.y < 0.0f ? q.y : r.y);  // -0, +inf, NaN: r
+}
+
+// every lane's bounded wait, agreed across the warp (the warp-collective
+// tensor-memory loads that follow need all 32 lanes)
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_gelu_quant(const __grid_constant__ FusedMaps maps, const __grid_constant__ FParams p) {
@@ -137,7 +224,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sfring = smem + STAGES * STAGE_BYTES;
   uint8_t* xt = sfring + SF_SLOTS * SF_SLOT_BYTES;  // 1024-aligned
   uint8_t* l1s = xt + XT_BYTES;                     // 1024-aligned
-  uint64_t* full = (uint64_t*)(l1s + L1_BYTES);
+  uint8_t* cst = l1s + L1_BYTES;                     // codes staging [2][128][96]
+  uint8_t* sst = cst + 2 * CST_BYTES;                // scale staging [2][three atoms]
+  uint64_t* full = (uint64_t*)(sst + 2 * SST_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;    // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]: 8 epilogue warps
@@ -147,12 +236,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* sfs_full = sf_free + 2;       // [SF_SLOTS]
   uint64_t* sfs_empty = sfs_full + SF_SLOTS;
   uint64_t* l1_full = sfs_empty + SF_SLOTS;
-  uint64_t* xt_full = l1_full + 1;        // 8 epilogue warps
-  uint64_t* xt_free = xt_full + 1;        // t' MMAs of the tile done (x^' tile and L1' slot free)
+  uint64_t* xt_full = l1_full + 1;        // [2] per staging buffer, 8 epilogue warps: x^' tile and codes/scales staged
+  uint64_t* xt_free = xt_full + 2;        // t' MMAs of the tile done (x^' tile and L1' slot free)
   uint64_t* tp_full = xt_free + 1;        // the unit's t' sum is complete
   uint64_t* tp_empty = tp_full + 1;       // 4 reader warps
   uint64_t* tdone = tp_empty + 1;
-  uint32_t* tmem_slot = (uint32_t*)(tdone + 1);
+  uint64_t* st_free = tdone + 1;          // [2] a staging buffer's stores have read it
+  uint32_t* tmem_slot = (uint32_t*)(st_free + 2);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   volatile int* ticket = abort_flag + 1;  // [4] one per lane-quarter reader warp
 
@@ -178,11 +268,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sfs_empty[b], 4);
     }
     mbar_init(l1_full, 1);
-    mbar_init(xt_full, 8);
+    mbar_init(&xt_full[0], 8);
+    mbar_init(&xt_full[1], 8);
     mbar_init(xt_free, 1);
     mbar_init(tp_full, 1);
     mbar_init(tp_empty, 4);
     mbar_init(tdone, 1);
+    mbar_init(&st_free[0], 1);
+    mbar_init(&st_free[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -298,30 +391,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == SF_WARP) {
     // ------------------------------------------------------------ scale-factor producer
+    // One slot per K stage: [SFA 4 atoms | SFB 8 atoms], two bulk copies.
     if (lane == 0) {
       pdl_wait();  // the activation scales come from the previous kernel
       int pit = 0;
       bool ok = true;
-      const int pairs_k = (p.k_stages + 1) / 2;
       for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
         const int mt = u % p.m_tiles, sg = u / p.m_tiles;
         const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
         for (int nt = nt0; nt < nt1 && ok; ++nt) {
-          for (int j = 0; j < pairs_k; ++j, ++pit) {
+          for (int ks = 0; ks < p.k_stages; ++ks, ++pit) {
             const int slot = pit % SF_SLOTS;
             if (!mbar_wait(&sfs_empty[slot], ((pit / SF_SLOTS) & 1) ^ 1, wc)) {
               ok = false;
               break;
             }
-            const int ns = (2 * j + 1 < p.k_stages) ? 2 : 1;
             uint8_t* dst = sfring + slot * SF_SLOT_BYTES;
-            mbar_arrive_expect_tx(&sfs_full[slot], (uint32_t)ns * (SFA_BYTES + SFB_BYTES));
-            const size_t oa = ((size_t)mt * p.katoms + 8 * j) * kSfAtomBytes;
-            const size_t ob = ((size_t)nt * p.katoms + 8 * j) * 2 * kSfAtomBytes;
-            if (SVDQ_INB(p.status, oa, ns * SFA_BYTES, p.sfa_bytes))
-              bulk_load(dst, p.sfa + oa, ns * SFA_BYTES, &sfs_full[slot]);
-            if (SVDQ_INB(p.status, ob, ns * SFB_BYTES, p.sfb_bytes))
-              bulk_load(dst + 2 * SFA_BYTES, p.sfb + ob, ns * SFB_BYTES, &sfs_full[slot]);
+            mbar_arrive_expect_tx(&sfs_full[slot], SFA_BYTES + SFB_BYTES);
+            const size_t oa = ((size_t)mt * p.katoms + 4 * ks) * kSfAtomBytes;
+            const size_t ob = ((size_t)nt * p.katoms + 4 * ks) * 2 * kSfAtomBytes;
+            if (SVDQ_INB(p.status, oa, SFA_BYTES, p.sfa_bytes)) bulk_load(dst, p.sfa + oa, SFA_BYTES, &sfs_full[slot]);
+            if (SVDQ_INB(p.status, ob, SFB_BYTES, p.sfb_bytes))
+              bulk_load(dst + SFA_BYTES, p.sfb + ob, SFB_BYTES, &sfs_full[slot]);
           }
         }
       }
@@ -336,20 +427,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     // 128-row atom of the stage, the atom's 16-byte row l into 4 consecutive
     // columns (the replicated layout the block-scaled MMA reads).
     const int q = warp & 3;
-    int kst = 0, pit = 0;
+    int kst = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
       const int sg = u / p.m_tiles;
       const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
       for (int nt = nt0; nt < nt1 && ok; ++nt) {
         for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
-          const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
-          const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
-          if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
-          ok = ok && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+          const int slot = kst % SF_SLOTS, sb = kst & 1;
+          ok = mbar_wait(&sfs_full[slot], (kst / SF_SLOTS) & 1, wc) && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
           if (!ok) break;
-          const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
-          const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
+          const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES;
+          const uint8_t* sfb_s = sfa_s + SFA_BYTES;
           uint32_t ra[16], rb[32];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -369,62 +458,86 @@ __global__ void __launch_bounds__(THREADS, 1)
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(&sf_ready[sb]);
-            if (last_of_pair) mbar_arrive(&sfs_empty[slot]);
+            mbar_arrive(&sfs_empty[slot]);  // the slot's atoms are in registers
           }
-          if (last_of_pair) ++pit;
         }
       }
     }
   } else if (warp == T_WARP) {
-    // ------------------------------------------------------------ L1'^T slices and t' MMAs
-    // Per tile: the rank rows of L1'^T for the tile's 192 columns (three
-    // 64-column boxes, 128-byte swizzle) into the slot; once the epilogue has
-    // written the tile's x^', t' += bf16(x^'_tile) . L1'[tile] (M = 128,
-    // N = rank, K = 192); the x^' tile and the slot are free when those MMAs
-    // complete.
-    if (lane == 0 && p.rank_dn > 0) {
-      prefetch_tmap(&maps.l1dn);
+    // ------------------------------------------------------------ t' MMAs and the staged stores
+    // Per tile: the rank rows of L1'^T for the tile's 192 columns (three 64-column
+    // boxes, 128-byte swizzle) into the slot; once the epilogue has staged the
+    // tile (x^', codes, scales), t' += bf16(x^'_tile) . L1'[tile] (M = 128,
+    // N = rank, K = 192) -- the x^' tile and the slot are free when those MMAs
+    // complete -- then the codes (TMA tensor store, rows past M clipped) and the
+    // three scale atoms (one bulk copy: contiguous in the atom layout) leave from
+    // the tile's staging buffer.  The staging is double-buffered: a buffer is
+    // released when the next tile's stores are issued and its own have been read.
+    if (lane == 0) {
+      const bool lr = p.rank_dn > 0;
+      if (lr) prefetch_tmap(&maps.l1dn);
+      prefetch_tmap(&maps.codes_dn);
       bool ok = true;
       int tt = 0, ut = 0;
-      const uint32_t idesc_t = idesc_bf16_f32(BM, p.rank_dn);
+      const uint32_t idesc_t = lr ? idesc_bf16_f32(BM, p.rank_dn) : 0u;
       for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++ut) {
-        const int sg = u / p.m_tiles;
+        const int mt = u % p.m_tiles, sg = u / p.m_tiles;
         const int nt0 = sg * p.n_tiles / p.S, nt1 = (sg + 1) * p.n_tiles / p.S;
         for (int nt = nt0; nt < nt1 && ok; ++nt, ++tt) {
-          if (!mbar_wait(xt_free, (tt & 1) ^ 1, wc)) {  // the previous tile's t' MMAs completed
+          const int sb = tt & 1;
+          if (lr) {
+            if (!mbar_wait(xt_free, (tt & 1) ^ 1, wc)) {  // the previous tile's t' MMAs completed
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(l1_full, 3u * (uint32_t)p.rank_dn * 128u);
+            for (int hb = 0; hb < 3; ++hb)
+              tma_load_2d(&maps.l1dn, l1_full, l1s + hb * L1_MAX_ROWS * 128, nt * BN + 64 * hb, 0);
+          }
+          // the epilogue staged the tile (one barrier per buffer: the epilogue cannot
+          // complete one twice before this wait, since it reuses the buffer only after
+          // the release below)
+          if (!mbar_wait(&xt_full[sb], (tt >> 1) & 1, wc)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(l1_full, 3u * (uint32_t)p.rank_dn * 128u);
-          for (int hb = 0; hb < 3; ++hb)
-            tma_load_2d(&maps.l1dn, l1_full, l1s + hb * L1_MAX_ROWS * 128, nt * BN + 64 * hb, 0);
-          if (!mbar_wait(l1_full, tt & 1, wc) || !mbar_wait(xt_full, tt & 1, wc)) {
-            ok = false;
-            break;
+          if (lr) {
+            if (!mbar_wait(l1_full, tt & 1, wc) || (nt == nt0 && !mbar_wait(tp_empty, (ut & 1) ^ 1, wc))) {
+              ok = false;  // (the unit's previous t' was read out before its first MMA)
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(xt), b0 = smem_u32(l1s);
+            for (int kk = 0; kk < 12; ++kk) {
+              const uint32_t hb = kk >> 2, koff = (kk & 3) * 32;
+              mma_bf16(tmem + TP_COL, make_sdesc(a0 + hb * (BM * 128) + koff, 16, 1024, LAYOUT_SW128),
+                       make_sdesc(b0 + hb * (L1_MAX_ROWS * 128) + koff, 16, 1024, LAYOUT_SW128), idesc_t,
+                       (nt > nt0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(xt_free);
+            if (nt + 1 == nt1) umma_commit(tp_full);
           }
-          if (nt == nt0 && !mbar_wait(tp_empty, (ut & 1) ^ 1, wc)) {  // the unit's t' was read out
-            ok = false;
-            break;
+          tma_store_2d(&maps.codes_dn, cst + sb * CST_BYTES, nt * (BN / 2), mt * BM);
+          const size_t so = ((size_t)mt * p.katoms_dn + 3 * nt) * kSfAtomBytes;
+          if (SVDQ_INB(p.status, so, SST_BYTES, p.scales_dn_bytes))
+            bulk_store(p.scales_dn + so, sst + sb * SST_BYTES, SST_BYTES);
+          bulk_commit();
+          if (tt > 0) {  // the previous tile's stores have read their buffer
+            bulk_wait_read<1>();
+            mbar_arrive(&st_free[sb ^ 1]);
           }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(xt), b0 = smem_u32(l1s);
-          for (int kk = 0; kk < 12; ++kk) {
-            const uint32_t hb = kk >> 2, koff = (kk & 3) * 32;
-            mma_bf16(tmem + TP_COL, make_sdesc(a0 + hb * (BM * 128) + koff, 16, 1024, LAYOUT_SW128),
-                     make_sdesc(b0 + hb * (L1_MAX_ROWS * 128) + koff, 16, 1024, LAYOUT_SW128), idesc_t,
-                     (nt > nt0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(xt_free);
-          if (nt + 1 == nt1) umma_commit(tp_full);
         }
       }
-      umma_commit(tdone);
-      mbar_wait_drain(tdone, 0, drain_limit);
+      bulk_wait<0>();  // the stores are complete
+      if (lr) {
+        umma_commit(tdone);
+        mbar_wait_drain(tdone, 0, drain_limit);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9)
-    pdl_wait();  // g_x and the down layer's workspace belong to the stream's order
     const int e = warp - 2;         // 0..7
+    pdl_wait();  // g_x and the down layer's workspace belong to the stream's order
     const int q = warp & 3;         // tensor-memory lane quarter
     const int half = e >> 2;        // columns 96*half .. 96*half + 95 of the tile
     const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;
@@ -437,17 +550,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int64_t m = (int64_t)mt * BM + row;
       const bool live = m < p.M;
       for (int nt = nt0; nt < nt1 && ok; ++nt, ++local, ++tt) {
-        const int b = local & 1;
-        if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        // the x^' tile may be overwritten once the previous tile's t' MMAs completed
-        if (p.rank_dn > 0 && !mbar_wait(xt_free, (tt & 1) ^ 1, wc)) {
+        const int b = local & 1, sb = tt & 1;
+        if (!warp_wait(&acc_full[b], (local >> 1) & 1, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        uint8_t* cs = cst + sb * CST_BYTES;
+        uint8_t* ss = sst + sb * SST_BYTES;
         const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN) + 96 * half;
         uint64_t swords = 0;  // the six block scales' of this warp's columns, one byte each
 #pragma unroll 1
@@ -469,20 +579,34 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
           }
-          float2 v[8];
+          float2 v[8], h2[8];
           uint32_t hbits[8];
+          float hmin = 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            // the up layer's bf16 output, GELU in binary32, rounded to bf16 (the down layer's input)
-            const float h0 = bf16_round(fmaf(__uint_as_float(r[2 * j]), out_scale, bb[2 * j]));
-            const float h1 = bf16_round(fmaf(__uint_as_float(r[2 * j + 1]), out_scale, bb[2 * j + 1]));
-            // 1 + erf(h / sqrt 2) = erfc(-h / sqrt 2): no cancellation for negative h
-            const float g0 = 0.5f * h0 * erfcf(-h0 * 0.70710678118654752f);
-            const float g1 = 0.5f * h1 * erfcf(-h1 * 0.70710678118654752f);
-            const __nv_bfloat162 gh = __floats2bfloat162_rn(g0, g1);
-            hbits[j] = *(const uint32_t*)&gh;
-            v[j] = __fmul2_rn(__bfloat1622float2(gh), make_float2(il[2 * j], il[2 * j + 1]));
+            // the up layer's bf16 output h, then x' = bf16(GELU(h)) (the down layer's input)
+            const float2 y2 = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
+                                         make_float2(out_scale, out_scale), make_float2(bb[2 * j], bb[2 * j + 1]));
+            h2[j] = __bfloat1622float2(__float22bfloat162_rn(y2));
+            hmin = fminf(hmin, fminf(h2[j].x, h2[j].y));
           }
+          if (__any_sync(0xffffffffu, hmin < -12.5f)) {  // a far negative tail in the warp: the scalar form
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const __nv_bfloat162 gh = __floats2bfloat162_rn(gelu_erf(h2[j].x), gelu_erf(h2[j].y));
+              hbits[j] = *(const uint32_t*)&gh;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const __nv_bfloat162 gh = __float22bfloat162_rn(gelu_erf2(h2[j]));
+              hbits[j] = *(const uint32_t*)&gh;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            v[j] = __fmul2_rn(make_float2(__uint_as_float(hbits[j] << 16), __uint_as_float(hbits[j] & 0xFFFF0000u)),
+                              make_float2(il[2 * j], il[2 * j + 1]));
           if (p.H != nullptr && live && SVDQ_INB(p.status, ((size_t)m * p.N + n) * 2, 32, p.H_bytes)) {
             // parity export of the down layer's input
             *(uint4*)(p.H + (size_t)m * p.N + n) = make_uint4(hbits[0], hbits[1], hbits[2], hbits[3]);
@@ -494,18 +618,26 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) mx[j] = fmaxf(mx[j], mx[j + 4]);
           const float amax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-          const uint32_t sb = cvt_e4m3(__fdiv_rn(amax, p.den_dn));
-          // 1 / (e4m3(sb) g') = (1 / e4m3(sb)) (1 / g'), exact: g' is a power of two
-          const float inv = sb != 0 ? __frcp_rn(e4m3_value(sb)) * p.inv_g_dn : 0.f;
+          const uint32_t sc = cvt_e4m3(__fdiv_rn(amax, p.den_dn));
+          // 1 / (e4m3(sc) g') = (1 / e4m3(sc)) (1 / g'), exact: g' is a power of two
+          const float inv = sc != 0 ? __frcp_rn(e4m3_value(sc)) * p.inv_g_dn : 0.f;
           const float2 inv2 = make_float2(inv, inv);
           float2 qv[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) qv[j] = __fmul2_rn(v[j], inv2);
           uint32_t c0 = cvt_e2m1x8(qv[0], qv[1], qv[2], qv[3]), c1 = cvt_e2m1x8(qv[4], qv[5], qv[6], qv[7]);
-          if (sb == 0) c0 = c1 = 0u;  // a zero block scale: all codes +0
-          if (live && SVDQ_INB(p.status, (size_t)m * (p.N / 2) + n / 2, 8, p.codes_dn_bytes))
-            *(uint2*)(p.codes_dn + (size_t)m * (p.N / 2) + n / 2) = make_uint2(c0, c1);
-          swords |= (uint64_t)sb << (8 * blk);
+          if (sc == 0) c0 = c1 = 0u;  // a zero block scale: all codes +0
+          if (blk == 0) {
+            // the staging buffer is free once the stores of two tiles back have read it,
+            // the x^' tile once the previous tile's t' MMAs completed
+            if (!warp_wait(&st_free[sb], ((tt >> 1) & 1) ^ 1, wc) ||
+                (p.rank_dn > 0 && !warp_wait(xt_free, (tt & 1) ^ 1, wc))) {
+              ok = false;
+              break;
+            }
+          }
+          *(uint2*)(cs + row * (BN / 2) + 48 * half + 8 * blk) = make_uint2(c0, c1);
+          swords |= (uint64_t)sc << (8 * blk);
           if (p.rank_dn > 0) {  // bf16(x^') into the swizzled x^' tile
             uint32_t xb[8];
 #pragma unroll
@@ -520,28 +652,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             *(uint4*)(rowp + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(xb[4], xb[5], xb[6], xb[7]);
           }
         }
-        if (p.rank_dn > 0) {
-          fence_proxy_async_smem();  // x^' tile -> tensor core
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xt_full);
-        }
-        if (live) {
-          // scale bytes of blocks blk0 .. blk0 + 5 (four consecutive blocks share an atom word)
-          const int blk0 = (nt * BN + 96 * half) / 16;
-          const size_t s0 = sf_offset(m, blk0, p.katoms_dn, kSfAtomRows);
-          const size_t s1 = sf_offset(m, blk0 + (half == 0 ? 4 : 2), p.katoms_dn, kSfAtomRows);
-          if (half == 0) {  // blocks 12t .. 12t+5: a whole word, then the first half of the next
-            if (SVDQ_INB(p.status, s0, 4, p.scales_dn_bytes)) *(uint32_t*)(p.scales_dn + s0) = (uint32_t)swords;
-            if (SVDQ_INB(p.status, s1, 2, p.scales_dn_bytes)) *(uint16_t*)(p.scales_dn + s1) = (uint16_t)(swords >> 32);
-          } else {  // blocks 12t+6 .. 12t+11: the second half of a word, then a whole word
-            if (SVDQ_INB(p.status, s0, 2, p.scales_dn_bytes)) *(uint16_t*)(p.scales_dn + s0) = (uint16_t)swords;
-            if (SVDQ_INB(p.status, s1, 4, p.scales_dn_bytes)) *(uint32_t*)(p.scales_dn + s1) = (uint32_t)(swords >> 16);
+        if (!ok) break;
+        {  // the six block scales' into the staged atoms (tile-local blocks 6*half .. 6*half + 5)
+          const int lb0 = 6 * half;
+          const size_t o0 = sf_offset(row, lb0, 3, kSfAtomRows);
+          const size_t o1 = sf_offset(row, lb0 + (half == 0 ? 4 : 2), 3, kSfAtomRows);
+          if (half == 0) {  // a whole atom word, then the first half of the next
+            *(uint32_t*)(ss + o0) = (uint32_t)swords;
+            *(uint16_t*)(ss + o1) = (uint16_t)(swords >> 32);
+          } else {  // the second half of a word, then a whole word
+            *(uint16_t*)(ss + o0) = (uint16_t)swords;
+            *(uint32_t*)(ss + o1) = (uint32_t)(swords >> 16);
           }
         }
+        fence_proxy_async_smem();  // x^' tile -> tensor core, staging -> bulk copies
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xt_full[sb]);
       }
       // ------------------------------------------------------------ the unit's t' partial
       if (ok && p.rank_dn > 0 && half == 0) {
-        if (!mbar_wait(tp_full, ut & 1, wc)) {
+        if (!warp_wait(tp_full, ut & 1, wc)) {
           ok = false;
           break;
         }
@@ -664,6 +794,9 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
       maps.l2[i] = L->map_l2[i];
     }
   }
+  st = encode_tmap_2d(&maps.codes_dn, CU_TENSOR_MAP_DATA_TYPE_UINT8, wsd + wd.codes, (uint64_t)N / 2, (uint64_t)M,
+                      (uint64_t)N / 2, BN / 2, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != SVDQ_OK) return st;
   const int rd = D->rank;
   if (rd > 0) {  // L1'^T [rd, N] bf16, 64 columns per box
     st = encode_tmap_2d(&maps.l1dn, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D->L1t, (uint64_t)D->K, (uint64_t)rd,
@@ -688,7 +821,6 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.inv_lambda_dn = D->inv_lambda;
   p.den_dn = 6.0f * D->g_x;
   p.inv_g_dn = 1.0f / D->g_x;  // exact: a power of two
-  p.codes_dn = wsd + wd.codes;
   p.scales_dn = wsd + wd.scales;
   p.t_dn = (uint16_t*)(wsd + wd.t);
   p.tpart = (float*)(wsd + wd.tpart);
@@ -701,7 +833,6 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.limit = wait_limit_cycles();
   p.sfa_bytes = w.scales_bytes;
   p.sfb_bytes = L->off.total - L->off.wscales;
-  p.codes_dn_bytes = wd.codes_bytes;
   p.scales_dn_bytes = wd.scales_bytes;
   p.t_dn_bytes = wd.t_bytes;
   p.tpart_bytes = wd.tpart_bytes;
@@ -715,7 +846,7 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   // work units: (128-row M tile) x (one of S contiguous groups of N tiles); the
   // t' partial sums of the groups land in the down layer's split-K area
   // (wd.nslices of them)
-  int S = (sms + p.m_tiles - 1) / p.m_tiles;
+  int S = sms / p.m_tiles;  // one wave of units
   const int max_groups = rd > 0 ? wd.nslices : p.n_tiles;
   if (S > max_groups) S = max_groups;
   if (S > p.n_tiles) S = p.n_tiles;

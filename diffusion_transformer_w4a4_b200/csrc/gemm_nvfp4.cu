@@ -86,6 +86,13 @@ struct GParams {
 
 __device__ __forceinline__ int lr_map_index(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
 
+// Output tile of a persistent CTA's work index: M tiles vary fastest, so the
+// CTAs running at one time share few weight tiles.
+__device__ __forceinline__ void tile_coords(int tile, const GParams& p, int& mt, int& nt) {
+  mt = tile % p.m_tiles;
+  nt = tile / p.m_tiles;
+}
+
 __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant__ GemmMaps maps, const __grid_constant__ GParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -147,7 +154,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        int mt, nt;
+        tile_coords(tile, p, mt, nt);
         for (int u = 0; u < units; ++u, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
@@ -238,7 +246,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       bool ok = true;
       const int pairs = (p.k_stages + 1) / 2;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+        int mt, nt;
+        tile_coords(tile, p, mt, nt);
         for (int j = 0; j < pairs; ++j, ++pit) {
           const int slot = pit % SF_SLOTS;
           if (!mbar_wait(&sfs_empty[slot], ((pit / SF_SLOTS) & 1) ^ 1, wc)) {
@@ -316,7 +325,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       const int b = local & 1;
       if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) break;
       tc_fence_after();
-      const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+      int mt, nt;
+      tile_coords(tile, p, mt, nt);
       const int m0 = mt * BM + 32 * q;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * BN);
 #pragma unroll 1
