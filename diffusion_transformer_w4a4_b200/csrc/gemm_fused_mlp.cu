@@ -211,12 +211,6 @@ __device__ __forceinline__ float2 gelu_erf2(float2 h) {
   return make_float2(h.x < 0.0f ? q.x : r.x, h.y < 0.0f ? q.y : r.y);  // -0, +inf, NaN: r
 }
 
-// every lane's bounded wait, agreed across the warp (the warp-collective
-// tensor-memory loads that follow need all 32 lanes)
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
-}
-
 __global__ void __launch_bounds__(THREADS, 1)
     k_gemm_gelu_quant(const __grid_constant__ FusedMaps maps, const __grid_constant__ FParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -435,7 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int nt = nt0; nt < nt1 && ok; ++nt) {
         for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
           const int slot = kst % SF_SLOTS, sb = kst & 1;
-          ok = mbar_wait(&sfs_full[slot], (kst / SF_SLOTS) & 1, wc) && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+          ok = warp_wait(&sfs_full[slot], (kst / SF_SLOTS) & 1, wc);
           if (!ok) break;
           const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES;
           const uint8_t* sfb_s = sfa_s + SFA_BYTES;
@@ -450,6 +444,13 @@ __global__ void __launch_bounds__(THREADS, 1)
               rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
             }
           }
+          // the atoms are in registers before the wait for the tensor-memory buffer, so
+          // the shared-memory reads stay off the MMA -> mover -> MMA chain
+          if (!warp_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();  // the MMAs that read this buffer completed: order the stores after them
           const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
           tmem_st_32x32b_x16(tq, ra);
           tmem_st_32x32b_x32(tq + 16, rb);
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(&sf_ready[sb]);
-            mbar_arrive(&sfs_empty[slot]);  // the slot's atoms are in registers
+            mbar_arrive(&sfs_empty[slot]);  // after the stores that consumed the loaded registers
           }
         }
       }

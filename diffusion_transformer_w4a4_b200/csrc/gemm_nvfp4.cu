@@ -285,8 +285,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       for (int ks = 0; ks < p.k_stages; ++ks, ++kst) {
         const int h = ks & 1, slot = pit % SF_SLOTS, sb = kst & 1;
         const bool last_of_pair = h == 1 || ks + 1 == p.k_stages;
-        if (h == 0) ok = mbar_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
-        ok = ok && mbar_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc);
+        if (h == 0) ok = warp_wait(&sfs_full[slot], (pit / SF_SLOTS) & 1, wc);
         if (!ok) break;
         const uint8_t* sfa_s = sfring + slot * SF_SLOT_BYTES + h * SFA_BYTES;
         const uint8_t* sfb_s = sfring + slot * SF_SLOT_BYTES + 2 * SFA_BYTES + h * SFB_BYTES;
@@ -301,6 +300,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
             rb[8 * j + 4 * hh] = b4.x; rb[8 * j + 4 * hh + 1] = b4.y; rb[8 * j + 4 * hh + 2] = b4.z; rb[8 * j + 4 * hh + 3] = b4.w;
           }
         }
+        // the atoms are in registers before the wait for the tensor-memory buffer, so
+        // the shared-memory reads stay off the MMA -> mover -> MMA chain
+        if (!warp_wait(&sf_free[sb], ((kst >> 1) & 1) ^ 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();  // the MMAs that read this buffer completed: order the stores after them
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + SF_COL + (uint32_t)sb * SF_BUF_COLS;
         tmem_st_32x32b_x16(tq, ra);
         tmem_st_32x32b_x32(tq + 16, rb);
@@ -309,7 +315,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&sf_ready[sb]);
-          if (last_of_pair) mbar_arrive(&sfs_empty[slot]);  // the slot's atoms are in tensor memory
+          // the slot is released only after the stores that consumed the loaded
+          // registers: releasing it right after the shared-memory loads let the next
+          // bulk copy into the slot overtake them (wrong scales at large K)
+          if (last_of_pair) mbar_arrive(&sfs_empty[slot]);
         }
         if (last_of_pair) ++pit;
       }

@@ -68,6 +68,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// mbar_wait by every lane, agreed across the warp (warp-collective tensor-memory
+// instructions after it need all 32 lanes on the same path).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, c));
+}
+
 // A wait used only on the teardown path after an abort: bounded, raises nothing.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, unsigned long long limit) {
   const unsigned long long t0 = clock64();
