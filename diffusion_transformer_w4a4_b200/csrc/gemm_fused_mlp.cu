@@ -2,7 +2,7 @@
 // quantizer fused into its epilogue (cross-layer fusion of the MLP pair).
 //
 //   h  = bf16( g_x g_w [ sum_blocks (s_x s_w)(qx . qw) + t . L2/(g_x g_w) ] + b )   (the up layer's y)
-//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) in binary32 (gelu_erf)
+//   x' = bf16( GELU(h) ),  GELU(h) = h/2 (1 + erf(h / sqrt 2)) in binary32 (gelu_erf2)
 //   x^' = f32(x') * inv_lambda'                                                     (the down layer's input)
 //   codes', E4M3 block scales'  of x^' (blocks of 16, static g_x'),  t' = bf16( bf16(x^') . L1' )
 //
@@ -135,38 +135,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-// GELU(h) = h Phi(h) = h/2 (1 + erf(h / sqrt 2)) in binary32, branch-free.  With
-// x = |h| / sqrt 2:  h >= 0: h - (h/2) erfc(x);  h < 0: (h/2) erfc(x)  (no
-// cancellation on either side).  erfc(x) = t exp(-x^2 + P(t)), t = 1/(1 + x/2):
-// the Chebyshev-fit form of Press et al., "Numerical Recipes" (2nd ed., sec.
-// 6.2), with P a degree-9 polynomial fitted by least squares to
-// log(erfc(x) e^(x^2) / t) at Chebyshev nodes in t in (0, 1], coefficients rounded
-// to binary32 (relative error of erfc below 1.2e-7 before rounding).  exp(y) for
-// y < -80 is taken as exp(y + 64 ln 2) 2^-64 so that tails below the binary32
-// normal range round once, as bf16 keeps them.  A table of the correctly rounded
-// bf16 results (the input is a bf16 value) measured slower: its random reads
-// cost more than the arithmetic.
-__device__ __forceinline__ float gelu_erf(float h) {
-  const float x = fabsf(h) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.5f, x, 1.0f));
-  float p = 1.708930433e-01f;
-  p = fmaf(p, t, -8.222485185e-01f);
-  p = fmaf(p, t, 1.488708496e+00f);
-  p = fmaf(p, t, -1.135414600e+00f);
-  p = fmaf(p, t, 2.790049911e-01f);
-  p = fmaf(p, t, -1.863418519e-01f);
-  p = fmaf(p, t, 9.679660201e-02f);
-  p = fmaf(p, t, 3.740904033e-01f);
-  p = fmaf(p, t, 1.000023723e+00f);
-  p = fmaf(p, t, -1.265512228e+00f);
-  const float y = fmaf(-x, x, p);  // -x^2 + P(t), rounded once
-  const bool low = y < -80.0f;
-  float te = t * __expf(low ? y + 44.3614195558365f : y);
-  te = low ? te * 0x1p-64f : te;   // t exp(y): one rounding into the subnormal range
-  const float q = (0.5f * h) * te;  // (h/2) erfc(x)
-  return __float_as_int(h) < 0 ? q : (te == 0.0f ? h : h - q);
-}
-
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -178,21 +146,30 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return r;
 }
 
-// gelu_erf for two elements with packed f32x2 arithmetic, for inputs h >= -12.5
-// (and +inf, NaN): there exp(-x^2 + P) >= 2^-122 stays normal, so the subnormal
-// scaling is not needed, and with 1/t and the exponent taken in base 2
-// (-h^2 log2(e)/2 + P(t) log2(e)) it costs about half the instructions.  h is
-// clamped to 16 inside the erfc part (h Phi(h) rounds to h from 8 up), and the
-// h >= 0 side is h (1 - erfc/2), so +inf, -0 and NaN come out right without tests
-// of their own.
+// GELU(h) = h Phi(h) = h/2 (1 + erf(h / sqrt 2)) in binary32 for two elements,
+// packed f32x2 arithmetic, no branches.  With x = |h| / sqrt 2:
+//   h < 0:  (h/2) erfc(x)          h >= 0:  h (1 - erfc(x)/2)
+// (no cancellation on either side).  erfc(x) = t exp(-x^2 + P(t)), t = 1/(1 + x/2):
+// the Chebyshev-fit form of Press et al., "Numerical Recipes" (2nd ed., sec.
+// 6.2), with P a degree-9 polynomial fitted by least squares to
+// log(erfc(x) e^(x^2) / t) at Chebyshev nodes in t in (0, 1], coefficients rounded
+// to binary32 (relative error of erfc below 1.2e-7 before rounding).  The
+// exponential is taken in base 2 and as the square of 2^(y/2), y = log2(erfc/t):
+// 2^(y/2) stays normal down to y = -252, so erfc far below the binary32 normal
+// range still comes out of one rounding of t 2^(y/2) 2^(y/2), as bf16 keeps it.
+// h is clamped to 16 inside erfc (h Phi(h) rounds to h from 8 up), so +inf gives
+// +inf, -0 gives -0 and NaN gives NaN.  Simulated in binary32 over all 65536 bf16
+// inputs, bf16(result) equals the binary64 definition rounded to bf16.  (A table
+// of the correctly rounded results measured slower: its random reads cost more
+// than this arithmetic.)
 __device__ __forceinline__ float2 gelu_erf2(float2 h) {
-  constexpr float L2E = 1.4426950408889634f;
+  constexpr float HL2E = 0.72134752044448170f;  // log2(e) / 2
   const float2 hc = make_float2(fminf(h.x, 16.0f), fminf(h.y, 16.0f));
   const float2 d = __ffma2_rn(make_float2(fabsf(hc.x), fabsf(hc.y)), make_float2(0.35355339059327376f, 0.35355339059327376f),
                               make_float2(1.0f, 1.0f));  // 1 + |h| / (2 sqrt 2)
   const float2 t = make_float2(rcp_approx(d.x), rcp_approx(d.y));
-  float2 p = make_float2(1.708930433e-01f * L2E, 1.708930433e-01f * L2E);
-#define SVDQ_H(c) p = __ffma2_rn(p, t, make_float2((c) * L2E, (c) * L2E))
+  float2 p = make_float2(1.708930433e-01f * HL2E, 1.708930433e-01f * HL2E);
+#define SVDQ_H(c) p = __ffma2_rn(p, t, make_float2((c) * HL2E, (c) * HL2E))
   SVDQ_H(-8.222485185e-01f);
   SVDQ_H(1.488708496e+00f);
   SVDQ_H(-1.135414600e+00f);
@@ -203,8 +180,10 @@ __device__ __forceinline__ float2 gelu_erf2(float2 h) {
   SVDQ_H(1.000023723e+00f);
   SVDQ_H(-1.265512228e+00f);
 #undef SVDQ_H
-  const float2 y = __ffma2_rn(__fmul2_rn(hc, make_float2(-0.5f * L2E, -0.5f * L2E)), hc, p);  // log2 of erfc / t
-  const float2 te = __fmul2_rn(t, make_float2(ex2_approx(y.x), ex2_approx(y.y)));  // erfc(|h| / sqrt 2)
+  // y/2 = (-x^2 + P(t)) log2(e) / 2 = -h^2 log2(e) / 4 + P(t) log2(e) / 2
+  const float2 y2 = __ffma2_rn(__fmul2_rn(hc, make_float2(-0.5f * HL2E, -0.5f * HL2E)), hc, p);
+  const float2 e = make_float2(ex2_approx(y2.x), ex2_approx(y2.y));
+  const float2 te = __fmul2_rn(__fmul2_rn(t, e), e);  // erfc(|h| / sqrt 2)
   const float2 ht = __fmul2_rn(te, make_float2(0.5f, 0.5f));
   const float2 q = __fmul2_rn(h, ht);                                        // h < 0: h erfc / 2
   const float2 r = __fmul2_rn(h, __fadd2_rn(make_float2(1.0f, 1.0f), make_float2(-ht.x, -ht.y)));  // h (1 - erfc / 2)
@@ -580,29 +559,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[b]);
           }
-          float2 v[8], h2[8];
+          float2 v[8];
           uint32_t hbits[8];
-          float hmin = 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             // the up layer's bf16 output h, then x' = bf16(GELU(h)) (the down layer's input)
             const float2 y2 = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])),
                                          make_float2(out_scale, out_scale), make_float2(bb[2 * j], bb[2 * j + 1]));
-            h2[j] = __bfloat1622float2(__float22bfloat162_rn(y2));
-            hmin = fminf(hmin, fminf(h2[j].x, h2[j].y));
-          }
-          if (__any_sync(0xffffffffu, hmin < -12.5f)) {  // a far negative tail in the warp: the scalar form
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const __nv_bfloat162 gh = __floats2bfloat162_rn(gelu_erf(h2[j].x), gelu_erf(h2[j].y));
-              hbits[j] = *(const uint32_t*)&gh;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const __nv_bfloat162 gh = __float22bfloat162_rn(gelu_erf2(h2[j]));
-              hbits[j] = *(const uint32_t*)&gh;
-            }
+            const __nv_bfloat162 gh = __float22bfloat162_rn(gelu_erf2(__bfloat1622float2(__float22bfloat162_rn(y2))));
+            hbits[j] = *(const uint32_t*)&gh;
           }
 #pragma unroll
           for (int j = 0; j < 8; ++j)
