@@ -13,8 +13,11 @@
 //
 // Persistent, warp-specialized CTA (one per SM), tile 128 x 192:
 //   warp 0      TMA producer: per stage a 128x256 activation-code tile and a
-//               192x256 weight-code tile (128-byte swizzle); the t / L2^T chunks
-//               of the low-rank branch ride the same ring first.
+//               192x256 weight-code tile (128-byte swizzle).  The low-rank
+//               branch's t / L2^T tiles: for ranks up to 32 into a buffer of
+//               their own, once per tile (a slot of the operand ring costs a
+//               whole stage of the pipeline, ~7 % of a 3072-deep tile); larger
+//               ranks ride the ring in chunks ahead of the K stages.
 //   warp 10     scale-factor producer: the E4M3 scale-factor atoms of two K
 //               stages per bulk copy (activation and weight side) into a ring of
 //               their own, so they arrive ahead of the codes they scale.
@@ -29,7 +32,8 @@
 //               ring they finish before the stage's codes land.
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator rows, scale, bias,
 //               bf16 round-to-nearest-even into a 128B-swizzled shared-memory
-//               staging tile, written to Y by TMA bulk-tensor stores.
+//               staging tile (one per warp), written to Y by TMA bulk-tensor
+//               stores.
 // Every wait is bounded (see sm100.cuh); no load uses cluster multicast.
 #include <cuda_bf16.h>
 
@@ -57,10 +61,16 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 2 * BN;  // 384: two buffers of [SFA 16 | SFB 32] columns
 constexpr uint32_t SF_BUF_COLS = 48;
 constexpr int EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 rows x 64 bf16, 128B-swizzled
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + 4 * 2 * EPI_STAGE_BYTES;
+// Ranks up to 32 (one low-rank chunk) have a buffer of their own, loaded once per
+// tile ahead of the tile's first MMA, instead of a slot of the operand ring: t
+// [128 x r] and the L2^T chunk [192 x r], bf16.
+constexpr int LR_MAX = 32;
+constexpr int LR_T_BYTES = BM * LR_MAX * 2;
+constexpr int LR_BYTES = LR_T_BYTES + BN * LR_MAX * 2;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_SLOTS * SF_SLOT_BYTES + 4 * EPI_STAGE_BYTES + LR_BYTES;
 constexpr uint32_t IDESC_NVF4 = idesc_nvf4_ue4m3(BM, BN);
 constexpr uint32_t IDESC_BF16 = idesc_bf16_f32(BM, BN);
-static_assert(STAGE_BYTES % 1024 == 0 && SF_SLOT_BYTES % 1024 == 0, "stage alignment");
+static_assert(STAGE_BYTES % 1024 == 0 && SF_SLOT_BYTES % 1024 == 0 && LR_T_BYTES % 1024 == 0, "stage alignment");
 static_assert(SMEM_BYTES + 1024 + 256 <= 227 * 1024, "shared memory budget");
 static_assert(SF_COL + 2 * SF_BUF_COLS <= TMEM_COLS, "tensor memory budget");
 
@@ -72,6 +82,7 @@ struct GParams {
   int M, N, K, m_tiles, n_tiles, num_tiles, k_stages, katoms;
   int n_lr;
   int lr_off[4], lr_w[4];
+  int lr_buf_w;  // width of the single low-rank chunk held in its own buffer (0: none / on the ring)
   const uint8_t* sfa;
   const uint8_t* sfb;
   const float* bias;
@@ -97,7 +108,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sfring = smem + STAGES * STAGE_BYTES;                // [SF_SLOTS][SF_SLOT_BYTES]
-  uint8_t* epi_stage = sfring + SF_SLOTS * SF_SLOT_BYTES;       // [4 warps][2][EPI_STAGE_BYTES]
+  uint8_t* epi_stage = sfring + SF_SLOTS * SF_SLOT_BYTES;       // [4 warps][EPI_STAGE_BYTES]
+  uint8_t* lrbuf = epi_stage + 4 * EPI_STAGE_BYTES;             // [t | L2^T chunk], 1024-aligned
   uint64_t* full = (uint64_t*)(smem + SMEM_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;  // [2]
@@ -107,7 +119,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
   uint64_t* sf_free = sf_ready + 2;     // [2]
   uint64_t* sfs_full = sf_free + 2;     // [SF_SLOTS]
   uint64_t* sfs_empty = sfs_full + SF_SLOTS;
-  uint32_t* tmem_slot = (uint32_t*)(sfs_empty + SF_SLOTS);
+  uint64_t* lr_full = sfs_empty + SF_SLOTS;
+  uint64_t* lr_free = lr_full + 1;
+  uint32_t* tmem_slot = (uint32_t*)(lr_free + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -123,6 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       mbar_init(&acc_empty[b], 128);
     }
     mbar_init(mma_done, 1);
+    mbar_init(lr_full, 1);
+    mbar_init(lr_free, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sf_ready[b], 4);
       mbar_init(&sf_free[b], 1);
@@ -151,11 +167,22 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       prefetch_tmap(&maps.a);
       prefetch_tmap(&maps.b);
       pdl_wait();  // the quantized activations come from the previous kernel
-      int it = 0;
+      int it = 0, lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
         int mt, nt;
         tile_coords(tile, p, mt, nt);
+        if (p.lr_buf_w > 0) {  // the tile's t and L2^T chunk, once the previous tile's MMAs read theirs
+          const int w = p.lr_buf_w, mi = lr_map_index(w);
+          if (!mbar_wait(lr_free, (lt & 1) ^ 1, wc)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(lr_full, (uint32_t)(BM + BN) * 2 * w);
+          tma_load_2d(&maps.t[mi], lr_full, lrbuf, 0, mt * BM);
+          tma_load_2d(&maps.l2[mi], lr_full, lrbuf + LR_T_BYTES, 0, nt * BN);
+          ++lt;
+        }
         for (int u = 0; u < units; ++u, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, wc)) {
@@ -179,6 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
       if (!ok) {  // drain the copies still in flight
         for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
           mbar_wait_drain(&full[j % STAGES], (j / STAGES) & 1, p.limit);
+        if (lt > 0) mbar_wait_drain(lr_full, (lt - 1) & 1, p.limit);
       }
     }
   } else if (warp == 1) {
@@ -192,6 +220,23 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(b * BN);
         uint32_t accum = 0;
+        if (p.lr_buf_w > 0) {  // the low-rank product first, from its own buffer
+          if (!mbar_wait(lr_full, local & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int w = p.lr_buf_w;
+          const uint32_t layout = w == 32 ? LAYOUT_SW64 : LAYOUT_SW32;
+          const uint32_t sbo = 8u * 2u * (uint32_t)w;
+          const uint32_t a_addr = smem_u32(lrbuf), b_addr = a_addr + LR_T_BYTES;
+          for (int kk = 0; kk < w / 16; ++kk) {
+            mma_bf16(d, make_sdesc(a_addr + 32 * kk, 16, sbo, layout), make_sdesc(b_addr + 32 * kk, 16, sbo, layout),
+                     IDESC_BF16, accum);
+            accum = 1;
+          }
+          umma_commit(lr_free);
+        }
         for (int u = 0; u < units; ++u, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&full[s], (it / STAGES) & 1, wc)) {
@@ -328,8 +373,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
     pdl_wait();  // g_x and Y belong to the stream's order
     const float out_scale = p.gx_dev != nullptr ? *p.gx_dev * p.g_w : p.out_scale;  // exact: powers of two
     const int q = warp & 3;  // tensor-memory lane quarter this warp may access
-    uint8_t* stg = epi_stage + (warp - 2) * 2 * EPI_STAGE_BYTES;
-    int local = 0, sbuf = 0;
+    uint8_t* stg = epi_stage + (warp - 2) * EPI_STAGE_BYTES;
+    int local = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
       const int b = local & 1;
       if (!mbar_wait(&acc_full[b], (local >> 1) & 1, wc)) break;
@@ -341,7 +386,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
 #pragma unroll 1
       for (int c = 0; c < BN / 64; ++c) {
         const int n0 = nt * BN + 64 * c;
-        uint8_t* dst = stg + sbuf * EPI_STAGE_BYTES + lane * 128;
+        uint8_t* dst = stg + lane * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float bb[32];
@@ -379,12 +424,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gemm_nvfp4(const __grid_constant
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&maps.y, stg + sbuf * EPI_STAGE_BYTES, n0, m0);
+          tma_store_2d(&maps.y, stg, n0, m0);
           bulk_commit();
-          bulk_wait_read<1>();  // the other staging buffer is free again
+          bulk_wait_read<0>();  // the staging buffer is free again
         }
         __syncwarp();
-        sbuf ^= 1;
       }
     }
     if (lane == 0) bulk_wait<0>();
@@ -404,10 +448,16 @@ int launch_gemm_nvfp4(const svdq_layer* L, int64_t M, void* Y, uint8_t* ws, cons
   const int K = (int)L->K, N = (int)L->N, r = L->rank;
   GParams p{};
   const LowRankChunks ch = lowrank_chunks(r);
-  p.n_lr = ch.n;
-  for (int i = 0; i < ch.n; ++i) {
-    p.lr_off[i] = ch.off[i];
-    p.lr_w[i] = ch.width[i];
+  if (ch.n == 1 && ch.width[0] <= LR_MAX) {  // one chunk of at most 32: its own buffer
+    p.n_lr = 0;
+    p.lr_buf_w = ch.width[0];
+  } else {
+    p.n_lr = ch.n;
+    p.lr_buf_w = 0;
+    for (int i = 0; i < ch.n; ++i) {
+      p.lr_off[i] = ch.off[i];
+      p.lr_w[i] = ch.width[i];
+    }
   }
   p.M = (int)M;
   p.N = N;
