@@ -42,23 +42,27 @@ def _dense(x_bits, w_bits, b_bits):
     return oracle.f32_to_bf16(np.ascontiguousarray(y, np.float32))
 
 
-def _pair(M, K, N, N2, r_up, r_dn, lid):
+def _pair(M, K, N, N2, r_up, r_dn, lid, dyn_up=False):
     up = wl.Layer(f"mlp_up_{M}x{K}x{N}", M, K, N, r_up, wl.NVFP4, 0.005, 50.0, False, lid)
     dn = wl.Layer(f"mlp_dn_{M}x{N}x{N2}", M, N, N2, r_dn, wl.NVFP4, 0.0, 1.0, True, lid + 1)
     X, W1, b1 = wl.make_layer_inputs(up)
     W2, b2 = wl.make_w(dn), wl.make_bias(dn)
     p_up = oracle.prepare(W1, b1, oracle.calib_absmax(X), 0.5, r_up, "nvfp4")
+    if dyn_up:  # the up layer's activation scale taken per call (g_x = 0), on an input away from calibration
+        p_up = dict(p_up)
+        p_up["g_x"] = 0.0
+        X = wl.f32_to_bf16_bits(oracle.bf16_to_f32(X) * np.float32(3.7))
     h_cal = oracle.gelu_bf16(_dense(X, W1, b1))
     p_dn = oracle.prepare(W2, b2, oracle.calib_absmax(h_cal), 0.5, r_dn, "nvfp4")
     return X, p_up, p_dn
 
 
-def _run(M, K, N, N2, r_up, r_dn, lid, rows=None):
+def _run(M, K, N, N2, r_up, r_dn, lid, rows=None, dyn_up=False):
     import torch
 
     import diffusion_transformer_w4a4_b200 as svdq
 
-    X, p_up, p_dn = _pair(M, K, N, N2, r_up, r_dn, lid)
+    X, p_up, p_dn = _pair(M, K, N, N2, r_up, r_dn, lid, dyn_up)
     g_up, g_dn = GpuLayer(p_up), GpuLayer(p_dn)
     assert svdq.svdq_mlp_fusable(g_up.lin.handle, g_dn.lin.handle) == svdq.SVDQ_OK
     x = g_up.x_dev(X)
@@ -115,6 +119,13 @@ def _run(M, K, N, N2, r_up, r_dn, lid, rows=None):
                                                (600, 1024, 1536, 512, 32, 32)])
 def test_fused_mlp_small(M, K, N, N2, r_up, r_dn):
     print(M, K, N, N2, r_up, r_dn, _run(M, K, N, N2, r_up, r_dn, lid=M + N))
+
+
+def test_fused_mlp_dynamic_up_scale():
+    """The up layer with a per-call activation scale (its first pass over X, the
+    scale read by the fused kernel from the workspace); X scaled by 3.7 away from
+    the calibration so the per-call scale differs from a static one."""
+    print("dynamic up", _run(300, 512, 768, 256, 32, 32, lid=77, dyn_up=True))
 
 
 def test_fused_mlp_flux_shape_sampled_rows():
