@@ -406,6 +406,50 @@ def w8a8_measure(dev, xs, steps=20):
             "gpu_launches": 6 * steps}
 
 
+def library_fp4_ceiling(dev, ours_us):
+    """Context for the GEMM roofline: a black-box library NVFP4 GEMM (cuBLASLt
+    through torch._scaled_mm: E2M1 operands with E4M3 block-16 scales, bf16
+    output) at the two MLP shapes, seeded random codes, L2 flushed, CUDA events.
+    It is not on the product path; `ours_over_library` compares its time with the
+    k_gemm_nvfp4 medians of the main line."""
+    import torch
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    out = {"library": "cuBLASLt NVFP4 via torch._scaled_mm", "codes": "seeded random"}
+    try:
+        for key, l in zip(("up", "down"), LAYERS):
+            ru = lambda x, m: (x + m - 1) // m * m
+            a = torch.randint(0, 256, (l.M, l.K // 2), dtype=torch.uint8, device=dev, generator=g)
+            b = torch.randint(0, 256, (l.N, l.K // 2), dtype=torch.uint8, device=dev, generator=g)
+            sa = torch.randint(0x30, 0x40, (ru(l.M, 128) * ru(l.K // 16, 4),), dtype=torch.uint8, device=dev,
+                               generator=g).view(torch.float8_e4m3fn)
+            sb = torch.randint(0x30, 0x40, (ru(l.N, 128) * ru(l.K // 16, 4),), dtype=torch.uint8, device=dev,
+                               generator=g).view(torch.float8_e4m3fn)
+            af, bf = a.view(torch.float4_e2m1fn_x2), b.view(torch.float4_e2m1fn_x2)
+            fn = lambda: torch._scaled_mm(af, bf.t(), sa, sb, out_dtype=torch.bfloat16)
+            fn()
+            torch.cuda.synchronize()
+            ts = []
+            for i in range(23):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                if i >= 3:
+                    ts.append(e0.elapsed_time(e1) * 1e3)
+            us = statistics.median(ts)
+            out[key] = {"us": us, "tflops": _layer_flops(l) / (us * 1e-6) / 1e12, "ours_us": ours_us[key],
+                        "ours_over_library": us / ours_us[key]}
+    except Exception as e:  # the library or its fp4 types missing: context only
+        out["unavailable"] = repr(e)[:200]
+    del flush
+    return out
+
+
 def fused_mlp_measure(dev, lins, xs, steps=20):
     """The same MLP pair with cross-layer fusion: per step the up layer's
     quantizer, the up GEMM whose epilogue applies GELU and writes the down layer's
@@ -765,6 +809,8 @@ def run_ours(args, world, rank, local):
     out["dynamic_act_scale"] = dynamic_measure(dev, canons, xs)
     out["w8a8"] = w8a8_measure(dev, xs)
     out["fused_mlp"] = fused_mlp_measure(dev, lins, xs)
+    out["library_fp4_ceiling"] = library_fp4_ceiling(
+        dev, {"up": statistics.median(g_up) * 1e3, "down": statistics.median(g_dn) * 1e3})
     if not args.no_configs:
         out["configs"] = configs_measure(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
