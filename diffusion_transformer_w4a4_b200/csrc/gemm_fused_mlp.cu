@@ -678,17 +678,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ticket[q] == p.S - 1) {
           __threadfence();
           if (live) {
+            // the groups' partials in group order; a batch of groups' loads is issued together
+            constexpr int SB = 4;
+#pragma unroll 1
             for (int j = 0; j < R; j += 4) {
               float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (SVDQ_INB(p.status, ((size_t)m * R + j) * 4, 16, p.tpart_bytes))
-                sum = __ldcg((const float4*)(p.tpart + (size_t)m * R + j));
-              for (int g = 1; g < p.S; ++g) {
-                if (!SVDQ_INB(p.status, (((size_t)g * p.M + m) * R + j) * 4, 16, p.tpart_bytes)) continue;
-                const float4 v4 = __ldcg((const float4*)(p.tpart + ((size_t)g * p.M + m) * R + j));
-                sum.x += v4.x;
-                sum.y += v4.y;
-                sum.z += v4.z;
-                sum.w += v4.w;
+#pragma unroll 1
+              for (int g0 = 0; g0 < p.S; g0 += SB) {
+                float4 v[SB];
+#pragma unroll
+                for (int i = 0; i < SB; ++i) {
+                  const size_t e = ((size_t)(g0 + i) * p.M + m) * R + j;
+                  v[i] = (g0 + i < p.S && SVDQ_INB(p.status, e * 4, 16, p.tpart_bytes)) ? __ldcg((const float4*)(p.tpart + e))
+                                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int i = 0; i < SB; ++i) {
+                  if (g0 + i >= p.S) break;
+                  if (g0 + i == 0) {
+                    sum = v[0];
+                  } else {
+                    sum.x += v[i].x;
+                    sum.y += v[i].y;
+                    sum.z += v[i].z;
+                    sum.w += v[i].w;
+                  }
+                }
               }
               const __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
               const __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);

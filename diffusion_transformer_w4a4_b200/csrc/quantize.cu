@@ -459,23 +459,48 @@ __global__ void __launch_bounds__(Roles<RANK>::kThreads, 1)
             if (*ticket == p.nslices - 1) {  // last slice of this row block: fixed-order sum
               __threadfence();
               if (m < p.M) {
+                // the slices' partials in slice order; the loads of a batch of slices (and of
+                // two column quads) are issued together, the sums keep their order
+                constexpr int SB = RANK > 80 ? 2 : 4;
+#pragma unroll 1
+                for (int j = 0; j < RANK; j += 8) {
+                  float4 sum[2];
+#pragma unroll 1
+                  for (int s0 = 0; s0 < p.nslices; s0 += SB) {
+                    float4 v[2][SB];
 #pragma unroll
-                for (int j = 0; j < RANK; j += 4) {
-                  float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                  if (SVDQ_INB(p.status, ((size_t)m * RANK + j) * 4, 16, p.tpart_bytes))
-                    sum = __ldcg((const float4*)(p.tpart + (size_t)m * RANK + j));
-                  for (int sl = 1; sl < p.nslices; ++sl) {
-                    if (!SVDQ_INB(p.status, (((size_t)sl * p.M + m) * RANK + j) * 4, 16, p.tpart_bytes)) continue;
-                    const float4 v = __ldcg((const float4*)(p.tpart + ((size_t)sl * p.M + m) * RANK + j));
-                    sum.x += v.x;
-                    sum.y += v.y;
-                    sum.z += v.z;
-                    sum.w += v.w;
+                    for (int i = 0; i < SB; ++i)
+#pragma unroll
+                      for (int h = 0; h < 2; ++h) {
+                        const size_t e = ((size_t)(s0 + i) * p.M + m) * RANK + j + 4 * h;
+                        v[h][i] = (s0 + i < p.nslices && j + 4 * h < RANK && SVDQ_INB(p.status, e * 4, 16, p.tpart_bytes))
+                                      ? __ldcg((const float4*)(p.tpart + e))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                      }
+#pragma unroll
+                    for (int i = 0; i < SB; ++i)
+#pragma unroll
+                      for (int h = 0; h < 2; ++h) {
+                        if (s0 + i >= p.nslices) continue;
+                        if (s0 + i == 0) {
+                          sum[h] = v[h][0];
+                        } else {
+                          sum[h].x += v[h][i].x;
+                          sum[h].y += v[h][i].y;
+                          sum[h].z += v[h][i].z;
+                          sum[h].w += v[h][i].w;
+                        }
+                      }
                   }
-                  __nv_bfloat162 h0 = scale_t(__floats2bfloat162_rn(sum.x, sum.y), tsc);
-                  __nv_bfloat162 h1 = scale_t(__floats2bfloat162_rn(sum.z, sum.w), tsc);
-                  if (SVDQ_INB(p.status, ((size_t)m * RANK + j) * 2, 8, p.t_bytes))
-                    *(uint2*)(p.t + (size_t)m * RANK + j) = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const int jj = j + 4 * h;
+                    if (jj >= RANK) break;
+                    __nv_bfloat162 h0 = scale_t(__floats2bfloat162_rn(sum[h].x, sum[h].y), tsc);
+                    __nv_bfloat162 h1 = scale_t(__floats2bfloat162_rn(sum[h].z, sum[h].w), tsc);
+                    if (SVDQ_INB(p.status, ((size_t)m * RANK + jj) * 2, 8, p.t_bytes))
+                      *(uint2*)(p.t + (size_t)m * RANK + jj) = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+                  }
                 }
               }
               if (threadIdx.x == 0 && SVDQ_INB(p.status, (size_t)rowblock * 4, 4, p.cnt_bytes))
