@@ -798,7 +798,7 @@ int launch_gemm_gelu_quant(const svdq_layer* L, const svdq_layer* D, int64_t M, 
   p.tpart = (float*)(wsd + wd.tpart);
   // one counter per 32-row group in the down workspace's first-pass slots (idle:
   // the down layer has a static activation scale); zero between calls
-  if (4 * (int64_t)p.m_tiles > kAmaxSlots) return SVDQ_ERR_INVALID_ARG;
+  if (M > kFusedMlpMaxM || 4 * (int64_t)p.m_tiles > kAmaxSlots) return SVDQ_ERR_INVALID_ARG;
   p.counters = (int*)(wsd + wd.amax);
   p.H = (uint16_t*)H;
   p.status = (int*)(ws + w.status);

@@ -428,6 +428,7 @@ svdq_status svdq_gemm_gelu_quantize(const svdq_layer* up, const svdq_layer* down
   if (st != SVDQ_OK) return st;
   st = (svdq_status)fused_mlp_supported(up, down);
   if (st != SVDQ_OK) return st;
+  if (M > kFusedMlpMaxM) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (H && ((uintptr_t)H & 15)) return SVDQ_ERR_INVALID_ARG;
   NvtxRange range("svdq/gemm_gelu_quantize");
@@ -439,6 +440,7 @@ svdq_status svdq_mlp_forward(const svdq_layer* up, const svdq_layer* down, const
                              void* ws_up, size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* stream) {
   svdq_status st = (svdq_status)fused_mlp_supported(up, down);
   if (st != SVDQ_OK) return st;
+  if (M > kFusedMlpMaxM) return SVDQ_ERR_INVALID_ARG;  // before anything is enqueued
   st = svdq_quantize_act(up, X, M, ws_up, ws_up_bytes, stream);
   if (st != SVDQ_OK) return st;
   st = svdq_gemm_gelu_quantize(up, down, M, ws_up, ws_up_bytes, ws_dn, ws_dn_bytes, nullptr, stream);

@@ -26,6 +26,9 @@ constexpr int kQChunk = 256;  // activation quantizer: K columns per chunk
 constexpr int kQSmCount = 148;  // SM count the quantizer's K-split is sized for (fixed, so sizes are device-free)
 constexpr size_t kAlign = 1024;
 constexpr int kAmaxSlots = 1024;  // per-CTA maxima of the dynamic activation-scale pass
+// The fused MLP kernel keeps one counter per 32-row group in the down layer's
+// first-pass slots (4 per 128-row tile), which bounds its token count.
+constexpr int64_t kFusedMlpMaxM = 32 * (int64_t)kAmaxSlots;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

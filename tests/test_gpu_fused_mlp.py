@@ -142,3 +142,10 @@ def test_fused_mlp_rejects_unfusable_pairs():
     dyn = dict(p_dn)
     dyn["g_x"] = 0.0
     assert svdq.svdq_mlp_fusable(g_up.lin.handle, GpuLayer(dyn).lin.handle) == svdq.SVDQ_ERR_INVALID_ARG
+    # more tokens than the per-group counters cover: refused before anything is enqueued
+    import torch
+
+    dummy = torch.zeros(1024, dtype=torch.uint8, device="cuda:0")
+    with pytest.raises(svdq.SvdqError) as e:
+        svdq.svdq_mlp_forward(g_up.lin.handle, g_dn.lin.handle, dummy, 32 * 1024 + 1, dummy, dummy, dummy)
+    assert e.value.status == svdq.SVDQ_ERR_INVALID_ARG
