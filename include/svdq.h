@@ -235,7 +235,8 @@ svdq_status svdq_gemm_gelu_quantize(const svdq_layer* up, const svdq_layer* down
                                     size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* H, void* stream);
 
 /* Y[M, down.N] = down(GELU(up(X))): svdq_quantize_act(up), svdq_gemm_gelu_quantize,
- * svdq_gemm(down), all on `stream`. */
+ * svdq_gemm(down), all on `stream`.  The pair and M <= 32768 are checked before
+ * anything is enqueued (SVDQ_ERR_INVALID_ARG). */
 svdq_status svdq_mlp_forward(const svdq_layer* up, const svdq_layer* down, const void* X, int64_t M, void* Y,
                              void* ws_up, size_t ws_up_bytes, void* ws_dn, size_t ws_dn_bytes, void* stream);
 
