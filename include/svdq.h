@@ -165,6 +165,7 @@ typedef struct svdq_layer svdq_layer; /* opaque host-side handle */
  * t, and leaves g_x in word 1 of the control block for svdq_gemm. */
 svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K, int rank, int fmt,
                               float g_x, float g_w, svdq_layer** out);
+/* Frees the host handle only (never the blob); NULL is a no-op. */
 void svdq_layer_destroy(svdq_layer* layer);
 
 /* Workspace for M tokens: quantized activations, low-rank t and a status word.
@@ -176,7 +177,14 @@ void svdq_layer_destroy(svdq_layer* layer);
  * int32, the first word of a control block that also holds the per-call g_x of a
  * dynamic-scale layer (word 1, float), the quantizer's split-K counters and the
  * first pass's per-CTA maxima.  The total size also covers the quantizer's fp32
- * partial sums of t. */
+ * partial sums of t.  Both calls are host-only; INVALID_ARG for a NULL argument
+ * or M < 0.
+ * Every call below that takes (ws, ws_bytes) checks first that ws (device
+ * memory) is non-NULL, 256-byte aligned, ws_bytes >= svdq_workspace_size(M) and
+ * 0 <= M <= 2^30, and returns SVDQ_ERR_INVALID_ARG with nothing enqueued
+ * otherwise.  The workspace is caller-owned.  Region offsets depend on M, so a
+ * buffer sized for M serves a call with M' < M only after svdq_workspace_init
+ * for M' (the control block then sits at M''s offset). */
 svdq_status svdq_workspace_size(const svdq_layer* layer, int64_t M, size_t* bytes);
 svdq_status svdq_workspace_layout(const svdq_layer* layer, int64_t M, size_t offsets[4], size_t sizes[4]);
 
@@ -329,6 +337,7 @@ typedef struct svdq_awq_layer svdq_awq_layer; /* opaque host-side handle */
  * device memory; UNSUPPORTED_DEVICE on a device other than CC 10.0. */
 svdq_status svdq_awq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K,
                                   svdq_awq_layer** out);
+/* Frees the host handle only (never the blob); NULL is a no-op. */
 void svdq_awq_layer_destroy(svdq_awq_layer* layer);
 
 /* Synchronous read of the blob's status word: 0, or SVDQ_ERR_TIMEOUT after a
@@ -369,6 +378,7 @@ svdq_status svdq_w8a8_pack(int64_t N, int64_t K, const int8_t* wcodes, const uin
  * UNSUPPORTED_DEVICE on a device other than CC 10.0. */
 svdq_status svdq_w8a8_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K, float s_w,
                                    svdq_w8a8_layer** out);
+/* Frees the host handle only (never the blob); NULL is a no-op. */
 void svdq_w8a8_layer_destroy(svdq_w8a8_layer* layer);
 
 /* Workspace for M tokens (caller device memory, 256-byte aligned): activation
