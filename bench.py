@@ -284,14 +284,14 @@ def awq_measure(dev, hbm_peak):
     x = x.view(torch.bfloat16).to(dev)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     for lin in lins:
-        lin.forward(x, out=y)
+        svdq.svdq_awq_forward(lin.handle, x, M, y)
     torch.cuda.synchronize()
     reps = 10
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    with torch.cuda.graph(graph):  # the C-ABI call itself is captured (the current stream is the capture stream)
         for _ in range(reps):
             for lin in lins:
-                lin.forward(x, out=y)
+                svdq.svdq_awq_forward(lin.handle, x, M, y)
     for _ in range(3):
         graph.replay()
     torch.cuda.synchronize()

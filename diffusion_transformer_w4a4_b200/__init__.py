@@ -334,11 +334,13 @@ def svdq_set_wait_limit(cycles: int) -> None:
 
 # ----------------------------------------------------------------------------- convenience
 class SvdqLinear:
-    """One svdq_w4a4 layer resident on the current CUDA device.
+    """One svdq_w4a4 layer resident on `device` (default: the current CUDA device).
 
     Built from canonical prepared weights (svdq_prepare output, or any dict with
-    the same arrays); `forward(x)` takes a bf16 CUDA tensor [M, K] and returns
-    bf16 [M, N].  Workspaces are cached per token count."""
+    the same arrays); `forward(x)` takes a bf16 CUDA tensor [M, K] on that device
+    and returns bf16 [M, N].  Workspaces are cached per token count.  The handle
+    is created, and every call that enqueues work is made, with the layer's
+    device current (the library refuses a call from another device)."""
 
     def __init__(self, canonical: dict, device=None):
         import torch
@@ -349,8 +351,9 @@ class SvdqLinear:
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         blob = svdq_pack(canonical)
         self.blob = torch.from_numpy(blob).to(self.device)
-        self.handle = svdq_layer_create(self.blob, self.blob.numel(), self.N, self.K, self.rank, self.fmt,
-                                        self.g_x, self.g_w)
+        with torch.cuda.device(self.device):
+            self.handle = svdq_layer_create(self.blob, self.blob.numel(), self.N, self.K, self.rank, self.fmt,
+                                            self.g_x, self.g_w)
         self._ws = {}
 
     def workspace(self, M: int):
@@ -359,7 +362,8 @@ class SvdqLinear:
         ws = self._ws.get(M)
         if ws is None:
             ws = torch.empty(max(svdq_workspace_size(self.handle, M), 1024), dtype=torch.uint8, device=self.device)
-            svdq_workspace_init(self.handle, M, ws)
+            with torch.cuda.device(self.device):
+                svdq_workspace_init(self.handle, M, ws)
             self._ws[M] = ws
         return ws
 
@@ -369,7 +373,9 @@ class SvdqLinear:
         assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
         M = x.numel() // self.K
         y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
-        svdq_forward(self.handle, x, M, y, self.workspace(M), stream)
+        ws = self.workspace(M)
+        with torch.cuda.device(self.device):
+            svdq_forward(self.handle, x, M, y, ws, stream)
         return y
 
     __call__ = forward
@@ -460,9 +466,10 @@ def svdq_awq_forward(h, X, M: int, Y, stream=None) -> None:
 
 
 class AwqLinear:
-    """One awq_w4a16 layer (4-bit weights, bf16 activations) on the current CUDA
-    device, built from canonical prepared weights (svdq_awq_prepare output or a
-    dict with the same arrays); `forward(x)` maps bf16 [M, K] to bf16 [M, N]."""
+    """One awq_w4a16 layer (4-bit weights, bf16 activations) on `device` (default:
+    the current CUDA device), built from canonical prepared weights
+    (svdq_awq_prepare output or a dict with the same arrays); `forward(x)` maps
+    bf16 [M, K] to bf16 [M, N], enqueued with the layer's device current."""
 
     def __init__(self, canonical: dict, device=None):
         import torch
@@ -470,7 +477,8 @@ class AwqLinear:
         self.N, self.K = int(canonical["N"]), int(canonical["K"])
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.blob = torch.from_numpy(svdq_awq_pack(canonical)).to(self.device)
-        self.handle = svdq_awq_layer_create(self.blob, self.blob.numel(), self.N, self.K)
+        with torch.cuda.device(self.device):
+            self.handle = svdq_awq_layer_create(self.blob, self.blob.numel(), self.N, self.K)
 
     def forward(self, x, out=None, stream=None):
         import torch
@@ -478,7 +486,8 @@ class AwqLinear:
         assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
         M = x.numel() // self.K
         y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
-        svdq_awq_forward(self.handle, x, M, y, stream)
+        with torch.cuda.device(self.device):
+            svdq_awq_forward(self.handle, x, M, y, stream)
         return y
 
     __call__ = forward
@@ -559,9 +568,10 @@ def svdq_w8a8_read_status(h, M: int, ws) -> int:
 
 
 class W8A8Linear:
-    """One INT8 tensorwise W8A8 layer on the current CUDA device, from prepared
-    int8 weight codes [N,K], the weight scale s_w and an optional bf16 bias;
-    `forward(x)` maps bf16 [M, K] to bf16 [M, N]."""
+    """One INT8 tensorwise W8A8 layer on `device` (default: the current CUDA
+    device), from prepared int8 weight codes [N,K], the weight scale s_w and an
+    optional bf16 bias; `forward(x)` maps bf16 [M, K] to bf16 [M, N], enqueued
+    with the layer's device current."""
 
     def __init__(self, wcodes, s_w: float, bias=None, device=None):
         import torch
@@ -570,7 +580,8 @@ class W8A8Linear:
         self.s_w = float(s_w)
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.blob = torch.from_numpy(svdq_w8a8_pack(wcodes, bias)).to(self.device)
-        self.handle = svdq_w8a8_layer_create(self.blob, self.blob.numel(), self.N, self.K, self.s_w)
+        with torch.cuda.device(self.device):
+            self.handle = svdq_w8a8_layer_create(self.blob, self.blob.numel(), self.N, self.K, self.s_w)
         self._ws = {}
 
     def workspace_size(self, M: int) -> int:
@@ -584,10 +595,18 @@ class W8A8Linear:
         return self._ws[M]
 
     def quantize_act(self, x, M: int, stream=None):
-        svdq_w8a8_quantize_act(self.handle, x, M, self.workspace(M), stream)
+        import torch
+
+        ws = self.workspace(M)
+        with torch.cuda.device(self.device):
+            svdq_w8a8_quantize_act(self.handle, x, M, ws, stream)
 
     def gemm(self, M: int, y, stream=None):
-        svdq_w8a8_gemm(self.handle, M, y, self.workspace(M), stream)
+        import torch
+
+        ws = self.workspace(M)
+        with torch.cuda.device(self.device):
+            svdq_w8a8_gemm(self.handle, M, y, ws, stream)
 
     def forward(self, x, out=None, stream=None):
         import torch
@@ -595,7 +614,9 @@ class W8A8Linear:
         assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
         M = x.numel() // self.K
         y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
-        svdq_w8a8_forward(self.handle, x, M, y, self.workspace(M), stream)
+        ws = self.workspace(M)
+        with torch.cuda.device(self.device):
+            svdq_w8a8_forward(self.handle, x, M, y, ws, stream)
         return y
 
     __call__ = forward

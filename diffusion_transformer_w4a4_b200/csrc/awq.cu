@@ -469,7 +469,9 @@ svdq_status svdq_awq_layer_create(const void* dev_blob, size_t blob_bytes, int64
     cudaGetLastError();
     return SVDQ_ERR_UNSUPPORTED_DEVICE;
   }
-  const svdq_status st = svdq_device_check(dev);
+  svdq_status st = svdq_device_check(dev);
+  if (st != SVDQ_OK) return st;
+  st = (svdq_status)check_blob_pointer(dev_blob, dev);
   if (st != SVDQ_OK) return st;
   svdq_awq_layer* L = new (std::nothrow) svdq_awq_layer();
   if (!L) return SVDQ_ERR_OOM;
@@ -500,6 +502,7 @@ svdq_status svdq_awq_forward(const svdq_awq_layer* L, const void* X, int64_t M, 
   if (!L || M < 0) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!X || !Y || ((uintptr_t)X & 15) || ((uintptr_t)Y & 15) || M > (1 << 30)) return SVDQ_ERR_INVALID_ARG;
+  if (const int e = require_current_device(L->device); e != SVDQ_OK) return (svdq_status)e;
   AwqParams p{};
   p.M = (int)M;
   p.N = (int)L->N;

@@ -30,6 +30,26 @@ int device_sm_count(int dev) {
   return n;
 }
 
+int require_current_device(int dev) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return cur == dev ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
+}
+
+int check_blob_pointer(const void* p, int dev) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_OK;
+  }
+  if (a.type == cudaMemoryTypeHost || a.type == cudaMemoryTypeUnregistered) return SVDQ_ERR_INVALID_ARG;
+  if (a.type == cudaMemoryTypeDevice && a.device != dev) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
 LowRankChunks lowrank_chunks(int rank) {
   LowRankChunks c{};
   int off = 0;
@@ -298,6 +318,8 @@ svdq_status svdq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N
   }
   svdq_status st = svdq_device_check(dev);
   if (st != SVDQ_OK) return st;
+  st = (svdq_status)check_blob_pointer(dev_blob, dev);
+  if (st != SVDQ_OK) return st;
   svdq_layer* L = new (std::nothrow) svdq_layer();
   if (!L) return SVDQ_ERR_OOM;
   L->N = N;
@@ -377,6 +399,8 @@ svdq_status svdq_workspace_init(const svdq_layer* L, int64_t M, void* ws, size_t
   Workspace w;
   svdq_status st = check_ws(L, M, ws, ws_bytes, &w);
   if (st != SVDQ_OK) return st;
+  st = (svdq_status)require_current_device(L->device);
+  if (st != SVDQ_OK) return st;
   if (cudaMemsetAsync((uint8_t*)ws + w.status, 0, w.ctrl_bytes, (cudaStream_t)stream) != cudaSuccess)
     return SVDQ_ERR_CUDA;
   return SVDQ_OK;
@@ -389,6 +413,8 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!X || ((uintptr_t)X & 15)) return SVDQ_ERR_INVALID_ARG;
+  st = (svdq_status)require_current_device(L->device);
+  if (st != SVDQ_OK) return st;
   NvtxRange range("svdq/quantize");
   if (L->dyn_gx) {  // first pass: the tensor's largest |x^|
     const int e = launch_act_amax(L, X, M, (uint8_t*)ws, w, (cudaStream_t)stream);
@@ -403,6 +429,8 @@ svdq_status svdq_gemm(const svdq_layer* L, int64_t M, void* Y, void* ws, size_t 
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!Y || ((uintptr_t)Y & 15)) return SVDQ_ERR_INVALID_ARG;
+  st = (svdq_status)require_current_device(L->device);
+  if (st != SVDQ_OK) return st;
   NvtxRange range("svdq/gemm");
   if (L->fmt == SVDQ_NVFP4_G16) return (svdq_status)launch_gemm_nvfp4(L, M, Y, (uint8_t*)ws, w, (cudaStream_t)stream);
   return (svdq_status)launch_gemm_int4(L, M, Y, (uint8_t*)ws, w, nullptr, (cudaStream_t)stream);
@@ -431,6 +459,8 @@ svdq_status svdq_gemm_gelu_quantize(const svdq_layer* up, const svdq_layer* down
   if (M > kFusedMlpMaxM) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (H && ((uintptr_t)H & 15)) return SVDQ_ERR_INVALID_ARG;
+  st = (svdq_status)require_current_device(up->device);  // the pair shares one device
+  if (st != SVDQ_OK) return st;
   NvtxRange range("svdq/gemm_gelu_quantize");
   return (svdq_status)launch_gemm_gelu_quant(up, down, M, (uint8_t*)ws_up, wu, (uint8_t*)ws_dn, wd, H,
                                              (cudaStream_t)stream);
@@ -455,6 +485,8 @@ svdq_status svdq_int4_group_acc(const svdq_layer* L, int64_t M, void* ws, size_t
   if (st != SVDQ_OK) return st;
   if (L->fmt != SVDQ_INT4_G64 || !acc || ((uintptr_t)acc & 15)) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
+  st = (svdq_status)require_current_device(L->device);
+  if (st != SVDQ_OK) return st;
   return (svdq_status)launch_gemm_int4(L, M, nullptr, (uint8_t*)ws, w, acc, (cudaStream_t)stream);
 }
 

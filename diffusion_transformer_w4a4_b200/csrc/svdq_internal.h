@@ -156,6 +156,14 @@ int encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
 
 unsigned long long wait_limit_cycles();
 int device_sm_count(int dev);  // multiprocessor count, cached per device (148 if the query fails)
+// SVDQ_OK iff `dev` (a layer's device) is the calling thread's current device,
+// INVALID_ARG otherwise (kernels launched there would read another GPU's memory),
+// SVDQ_ERR_CUDA if the query fails.
+int require_current_device(int dev);
+// INVALID_ARG when the runtime reports `p` as host memory or as memory of a
+// device other than `dev`; SVDQ_OK otherwise (managed memory, or a pointer the
+// runtime cannot classify, is left to the caller).
+int check_blob_pointer(const void* p, int dev);
 
 // Kernel launchers (return svdq_status).
 // dynamic activation scale: grid of the amax pass (its CTA count is the number

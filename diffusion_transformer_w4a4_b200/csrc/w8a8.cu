@@ -397,7 +397,9 @@ svdq_status svdq_w8a8_layer_create(const void* dev_blob, size_t blob_bytes, int6
     cudaGetLastError();
     return SVDQ_ERR_UNSUPPORTED_DEVICE;
   }
-  const svdq_status st = svdq_device_check(dev);
+  svdq_status st = svdq_device_check(dev);
+  if (st != SVDQ_OK) return st;
+  st = (svdq_status)check_blob_pointer(dev_blob, dev);
   if (st != SVDQ_OK) return st;
   svdq_w8a8_layer* L = new (std::nothrow) svdq_w8a8_layer();
   if (!L) return SVDQ_ERR_OOM;
@@ -437,6 +439,8 @@ svdq_status svdq_w8a8_quantize_act(const svdq_w8a8_layer* L, const void* X, int6
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!X || ((uintptr_t)X & 15)) return SVDQ_ERR_INVALID_ARG;
+  st = (svdq_status)require_current_device(L->device);
+  if (st != SVDQ_OK) return st;
   NvtxRange range("svdq/w8a8_quantize");
   return (svdq_status)launch_w8_quantize(L, X, M, (uint8_t*)ws, (cudaStream_t)stream);
 }
@@ -446,6 +450,8 @@ svdq_status svdq_w8a8_gemm(const svdq_w8a8_layer* L, int64_t M, void* Y, void* w
   if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!Y || ((uintptr_t)Y & 15)) return SVDQ_ERR_INVALID_ARG;
+  st = (svdq_status)require_current_device(L->device);
+  if (st != SVDQ_OK) return st;
   NvtxRange range("svdq/w8a8_gemm");
   return (svdq_status)launch_w8_gemm(L, M, Y, (uint8_t*)ws, (cudaStream_t)stream);
 }

@@ -38,6 +38,11 @@
  *     Device-side failures (an in-kernel wait that ran past its limit) are
  *     recorded in a status word inside the caller's workspace and read with
  *     svdq_read_status.  A failed call leaves its outputs unspecified.
+ *   - Devices: a layer belongs to the device that was current when it was
+ *     created, and its blob must be memory of that device.  Every call that
+ *     enqueues work must be made with that device current (it is a per-thread
+ *     setting); otherwise the call returns SVDQ_ERR_INVALID_ARG and enqueues
+ *     nothing, instead of launching kernels that would read another GPU's memory.
  *   - Thread safety: functions are re-entrant; a layer handle may be used from
  *     several threads at once; calls that share a workspace must not overlap.
  */
@@ -155,7 +160,9 @@ typedef struct svdq_layer svdq_layer; /* opaque host-side handle */
 
 /* Bind a device-resident packed blob (from svdq_pack) to a host handle.  No
  * device memory is allocated; the blob must outlive the handle.  Fails with
- * UNSUPPORTED_DEVICE on a device other than CC 10.0 (current device).
+ * UNSUPPORTED_DEVICE on a device other than CC 10.0 (current device), and with
+ * INVALID_ARG when the CUDA runtime reports the blob as host memory or as memory
+ * of another device.
  * NVFP4: g_w and g_x must be powers of two, or g_x = 0 for the dynamic
  * activation scale (the blob must then have been packed with g_x = 0 too: its
  * L2 carries 1/g_w only).  A dynamic layer's svdq_quantize_act runs a first pass
@@ -334,7 +341,8 @@ svdq_status svdq_awq_pack(const svdq_awq_canonical* c, void* blob, size_t blob_b
 typedef struct svdq_awq_layer svdq_awq_layer; /* opaque host-side handle */
 
 /* Bind a device-resident awq blob (256-byte aligned) to a handle; allocates no
- * device memory; UNSUPPORTED_DEVICE on a device other than CC 10.0. */
+ * device memory; UNSUPPORTED_DEVICE on a device other than CC 10.0, INVALID_ARG
+ * for a blob in host memory or on another device. */
 svdq_status svdq_awq_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K,
                                   svdq_awq_layer** out);
 /* Frees the host handle only (never the blob); NULL is a no-op. */
@@ -375,7 +383,8 @@ svdq_status svdq_w8a8_pack(int64_t N, int64_t K, const int8_t* wcodes, const uin
 
 /* Bind a device-resident w8a8 blob (256-byte aligned) to a handle with the
  * weight scale s_w (finite, >= 0); allocates no device memory.
- * UNSUPPORTED_DEVICE on a device other than CC 10.0. */
+ * UNSUPPORTED_DEVICE on a device other than CC 10.0, INVALID_ARG for a blob in
+ * host memory or on another device. */
 svdq_status svdq_w8a8_layer_create(const void* dev_blob, size_t blob_bytes, int64_t N, int64_t K, float s_w,
                                    svdq_w8a8_layer** out);
 /* Frees the host handle only (never the blob); NULL is a no-op. */
