@@ -40,12 +40,18 @@ E4M3_MAX = 448.0
 E2M1_MAX = 6.0
 
 
+def compile_source(src: str, out: str) -> None:
+    """gcc with the flags the oracle's arithmetic relies on (no fused
+    multiply-add, no fast-math)."""
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+                           "-shared", "-fPIC", "-o", out, src, "-lm"])
+
+
 def build(force: bool = False) -> str:
-    """Compile svdq_oracle.c with gcc (no fused multiply-add, no fast-math)."""
+    """Compile svdq_oracle.c into liboracle.so when it is missing or stale."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
-                               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        compile_source(_SRC, tmp)
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -56,34 +62,38 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
-        L = _lib
-        i64, f32, f64, vp, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
-        L.orc_f64_to_bf16.restype = ctypes.c_uint16
-        L.orc_f64_to_bf16.argtypes = [f64]
-        L.orc_f32_to_bf16.restype = ctypes.c_uint16
-        L.orc_f32_to_bf16.argtypes = [f32]
-        L.orc_f32_to_f16.restype = ctypes.c_uint16
-        L.orc_f32_to_f16.argtypes = [f32]
-        L.orc_f32_to_e4m3_satfinite.restype = ctypes.c_uint8
-        L.orc_f32_to_e4m3_satfinite.argtypes = [f32]
-        L.orc_f32_to_e2m1_satfinite.restype = ctypes.c_uint8
-        L.orc_f32_to_e2m1_satfinite.argtypes = [f32]
-        for name in ("orc_vec_f64_to_bf16", "orc_vec_f32_to_bf16", "orc_vec_f32_to_f16", "orc_vec_f16_to_f32",
-                     "orc_vec_f32_to_e4m3", "orc_vec_e4m3_to_f32", "orc_vec_f32_to_e2m1", "orc_vec_e2m1_to_f32"):
-            getattr(L, name).argtypes = [i64, vp, vp]
-            getattr(L, name).restype = None
-        L.orc_smooth_factors.argtypes = [i64, vp, vp, f64, vp, vp, vp]
-        L.orc_smooth_act.argtypes = [i64, i64, vp, vp, vp]
-        L.orc_quant_int4_rows.argtypes = [i64, i64, vp, vp, vp]
-        L.orc_quant_nvfp4_rows.argtypes = [i64, i64, vp, f32, vp, vp]
-        L.orc_dequant_int4_rows.argtypes = [i64, i64, vp, vp, vp]
-        L.orc_dequant_nvfp4_rows.argtypes = [i64, i64, vp, vp, f32, vp]
-        L.orc_lowrank_down.argtypes = [i64, i64, i64, vp, vp, vp]
-        L.orc_int4_group_acc.argtypes = [i64, i64, i64, vp, vp, vp]
-        L.orc_forward_out.argtypes = [i64, i64, i64, i64, i32, vp, vp, vp, vp, f32, f32, vp, vp, vp, vp, vp]
-        L.orc_num_threads.restype = i32
+        _lib = bind(ctypes.CDLL(build()))
     return _lib
+
+
+def bind(L):
+    """Declare the C signatures on a loaded copy of the oracle library."""
+    i64, f32, f64, vp, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
+    L.orc_f64_to_bf16.restype = ctypes.c_uint16
+    L.orc_f64_to_bf16.argtypes = [f64]
+    L.orc_f32_to_bf16.restype = ctypes.c_uint16
+    L.orc_f32_to_bf16.argtypes = [f32]
+    L.orc_f32_to_f16.restype = ctypes.c_uint16
+    L.orc_f32_to_f16.argtypes = [f32]
+    L.orc_f32_to_e4m3_satfinite.restype = ctypes.c_uint8
+    L.orc_f32_to_e4m3_satfinite.argtypes = [f32]
+    L.orc_f32_to_e2m1_satfinite.restype = ctypes.c_uint8
+    L.orc_f32_to_e2m1_satfinite.argtypes = [f32]
+    for name in ("orc_vec_f64_to_bf16", "orc_vec_f32_to_bf16", "orc_vec_f32_to_f16", "orc_vec_f16_to_f32",
+                 "orc_vec_f32_to_e4m3", "orc_vec_e4m3_to_f32", "orc_vec_f32_to_e2m1", "orc_vec_e2m1_to_f32"):
+        getattr(L, name).argtypes = [i64, vp, vp]
+        getattr(L, name).restype = None
+    L.orc_smooth_factors.argtypes = [i64, vp, vp, f64, vp, vp, vp]
+    L.orc_smooth_act.argtypes = [i64, i64, vp, vp, vp]
+    L.orc_quant_int4_rows.argtypes = [i64, i64, vp, vp, vp]
+    L.orc_quant_nvfp4_rows.argtypes = [i64, i64, vp, f32, vp, vp]
+    L.orc_dequant_int4_rows.argtypes = [i64, i64, vp, vp, vp]
+    L.orc_dequant_nvfp4_rows.argtypes = [i64, i64, vp, vp, f32, vp]
+    L.orc_lowrank_down.argtypes = [i64, i64, i64, vp, vp, vp]
+    L.orc_int4_group_acc.argtypes = [i64, i64, i64, vp, vp, vp]
+    L.orc_forward_out.argtypes = [i64, i64, i64, i64, i32, vp, vp, vp, vp, f32, f32, vp, vp, vp, vp, vp]
+    L.orc_num_threads.restype = i32
+    return L
 
 
 def _p(a: np.ndarray):

@@ -185,6 +185,37 @@ def test_int4_group_acc_equals_matmul():
         assert np.array_equal(acc[g], qx[:, g * 64:(g + 1) * 64] @ qw[:, g * 64:(g + 1) * 64].T)
 
 
+def test_int4_subnormal_scales_saturate_codes():
+    """Groups whose amax / 7 lies among the fp16 subnormals: the scale rounds down
+    to 2^-24, so |v| / S reaches 7.35-10.15 and the codes must saturate.  Every
+    code is the member of [-8, 7] nearest to fl32(v * fl32(1/S)) (brute force
+    over all 16 codes, ties to the even code)."""
+    rng = np.random.default_rng(8)
+    rows, K = 6, 256
+    v = np.empty((rows, K), np.float32)
+    for r in range(rows):
+        for g in range(K // 64):
+            amax = 7.0 * rng.uniform(1.05, 1.45) * 2.0**-24  # amax / 7 rounds down to 2^-24 in fp16
+            x = rng.uniform(-1.0, 1.0, 64) * amax
+            x[0], x[1] = amax, -amax
+            v[r, g * 64:(g + 1) * 64] = x
+    codes, scales = oracle.quant_int4(v)
+    S = oracle.f16_to_f32(scales).astype(np.float64)
+    assert np.all(S == 2.0**-24)
+    q = _unpack_int4(codes)
+    inv = np.float32(1.0) / np.float32(2.0**-24)
+    p = (v * inv).astype(np.float64)
+    assert (p > 7.5).any() and (p < -8.5).any()  # both ends of the code range are exercised
+    cand = np.arange(-8, 8)
+    for pv, qv in zip(p.ravel(), q.ravel()):
+        d = np.abs(pv - cand)
+        best = cand[d == d.min()]
+        if best.size > 1:
+            best = best[best % 2 == 0]
+        assert qv == best[0], (pv, qv)
+    assert (q == 7).any() and (q == -8).any()
+
+
 @pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
 def test_forward_equals_dequantized_matmul(fmt):
     layer = wl.small_layer(40, 256, 96, 16, fmt)
