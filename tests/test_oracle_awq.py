@@ -52,6 +52,19 @@ def test_awq_exact_layer_equals_dense_product():
     np.testing.assert_array_equal(oracle.awq_forward(X, prep), y_ref)
 
 
+def test_awq_statistic_is_the_channel_mean():
+    """Worked example: the activation-aware statistic is mean |x| per input channel
+    (not the maximum), and s = mean^alpha with s = 1 for an all-zero channel."""
+    X = _bf16([[1.0, -2.0, 0.0, 0.5], [3.0, 6.0, 0.0, -0.5], [-2.0, 4.0, 0.0, 1.5]])
+    np.testing.assert_allclose(oracle.awq_mean_abs(X), [2.0, 4.0, 0.0, 2.5 / 3], rtol=1e-15)
+    s, s_f, inv = oracle.awq_channel_scales(oracle.awq_mean_abs(X), 0.5)
+    np.testing.assert_allclose(s, [np.sqrt(2.0), 2.0, 1.0, np.sqrt(2.5 / 3)], rtol=1e-15)
+    W = _bf16(np.random.default_rng(9).standard_normal((3, 64 * 1))[:, :4].repeat(16, axis=1) * 0.05)
+    Xw = np.tile(X, (1, 16))
+    prep = oracle.awq_prepare(W, None, Xw, alphas=(1.0,))
+    np.testing.assert_array_equal(prep["s"], np.tile(np.float32([2.0, 4.0, 1.0, 2.5 / 3]), 16))
+
+
 def test_awq_forward_brute_force_tiny():
     """Loop-level evaluation from the stored codes and scales (no matrix routines)."""
     rng = np.random.default_rng(6)

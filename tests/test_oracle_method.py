@@ -94,6 +94,9 @@ def test_prepare_residual_uses_rounded_factors():
     # full rank: the residual is only the bf16 rounding noise of the factors
     pf = oracle.prepare(W, b, oracle.calib_absmax(X), 0.5, 128, "nvfp4")
     assert np.linalg.norm(pf["R"]) < 0.02 * np.linalg.norm(What)
+    # the layer's bias passes through unchanged; no bias means zeros
+    assert np.array_equal(p["bias"], b) and b.any()
+    assert not oracle.prepare(W, None, oracle.calib_absmax(X), 0.5, 32, "nvfp4")["bias"].any()
 
 
 # ----------------------------------------------------------------------------- quantizers
@@ -157,6 +160,38 @@ def test_nvfp4_error_bound():
     a = np.abs(v) / d
     half = np.where(a < 2, 0.25, np.where(a < 4, 0.5, 1.0)) * d
     assert np.all(np.abs(dq - v) <= half * (1 + 1e-6))
+
+
+def test_nvfp4_zero_scale_blocks_have_zero_codes():
+    """A block whose amax / (6 g) rounds to the E4M3 zero (below half the smallest
+    subnormal, 2^-10) has scale 0, and every code of it is +0 (0x0) -- for an all-zero
+    block and for tiny nonzero values of either sign alike."""
+    g = 1.0
+    v = np.zeros((3, 64), np.float32)
+    v[1, 16:32] = np.linspace(-0.005, 0.004, 16)  # amax / 6 < 2^-10
+    v[2, 48:64] = -0.0051
+    v[0, 0:16] = np.linspace(-3, 3, 16)  # a normal block beside them
+    codes, scales = oracle.quant_nvfp4(v, g)
+    assert scales[0, 0] != 0
+    zero_blocks = [(0, 1), (0, 2), (0, 3), (1, 0), (1, 1), (1, 2), (1, 3), (2, 0), (2, 1), (2, 2), (2, 3)]
+    for r, blk in zero_blocks:
+        assert scales[r, blk] == 0
+        assert not codes[r, 8 * blk:8 * blk + 8].any(), (r, blk)
+
+
+def test_tensor_scales_are_tight():
+    """g is the smallest power of two with 6 * 448 * g >= amax of the tensor it scales,
+    so the block holding that amax gets an E4M3 scale in [224, 448]: for the weight
+    residual (g_w from |R|) and, on the calibration input itself, for the activations
+    (static g_x from the smoothed calibration maxima)."""
+    layer = wl.small_layer(64, 512, 128, 32, "nvfp4")
+    X, W, b = wl.make_layer_inputs(layer)
+    p = oracle.prepare(W, b, oracle.calib_absmax(X), 0.5, 32, "nvfp4")
+    sw = oracle.e4m3_to_f32(p["wscales"]).astype(np.float64)
+    assert 224.0 <= sw.max() <= 448.0, sw.max()
+    act = oracle.quantize_act(X, p)
+    sx = oracle.e4m3_to_f32(act["scales"]).astype(np.float64)
+    assert 224.0 <= sx.max() <= 448.0, sx.max()
 
 
 def test_pow2_scale():
@@ -239,6 +274,31 @@ def test_lowrank_down_matches_matmul():
     t = oracle.lowrank_down(xhat, p["L1"])
     ref = oracle.f64_to_bf16(_bf(oracle.f32_to_bf16(xhat)) @ _bf(p["L1"]))
     assert np.array_equal(t, ref)
+
+
+def test_lowrank_down_rounds_once():
+    """t is the binary64 sum rounded once to bf16: 1 + 2^-8 + 2^-30 lies above the bf16
+    tie at 1 + 2^-8 and rounds up, where a detour through binary32 would land on the tie
+    and round to 1.  The tie itself rounds to the even neighbour, 1."""
+    xhat = np.array([[1.0, 2.0**-8, 2.0**-30], [1.0, 2.0**-8, 0.0]], np.float32)
+    L1 = oracle.f64_to_bf16(np.ones((3, 1)))
+    t = oracle.lowrank_down(xhat, L1)
+    assert t[0, 0] == 0x3F81 and t[1, 0] == 0x3F80
+
+
+def test_output_rounds_once_from_binary64():
+    """y is formed in binary64 and rounded once to bf16: with zero codes (main term 0),
+    t = (1, 2^-8, 2^-30), L2 = 1 and no bias, y = 1 + 2^-8 + 2^-30 exactly, which rounds
+    up to 0x3F81 (a binary32 detour would give the tie and 0x3F80)."""
+    K, N, r = 64, 1, 3
+    prep = dict(N=N, K=K, rank=r, fmt=oracle.INT4, g_x=1.0, g_w=1.0,
+                wcodes=np.zeros((N, K // 2), np.uint8), wscales=np.zeros((N, 1), np.uint16),
+                L2=oracle.f64_to_bf16(np.ones((r, N))), bias=np.zeros(N, np.uint16))
+    act = dict(codes=np.zeros((1, K // 2), np.uint8), scales=np.zeros((1, 1), np.uint16),
+               t=oracle.f64_to_bf16(np.array([[1.0, 2.0**-8, 2.0**-30]])), g_x=1.0)
+    y, yd = oracle.forward_from_act(act, prep, want_f64=True)
+    assert yd[0, 0] == 1.0 + 2.0**-8 + 2.0**-30
+    assert y[0, 0] == 0x3F81
 
 
 # ----------------------------------------------------------------------------- method invariants

@@ -92,6 +92,32 @@ C_MUTANTS = [
      "double blk = (fmt == 1) ? (double)s : (double)s * 0.5;", FWD_NVFP4),
     ("output_weight_scales_of_the_wrong_group", "main_ += sxd[m * G + g] * swd[n * G + g] * blk;",
      "main_ += sxd[m * G + g] * swd[n * G + (G - 1 - g)] * blk;", FWD),
+    ("rounding_without_the_subnormal_floor", "if (E < emin) E = emin;", "", CODEC_PINS),
+    ("e2m1_drops_the_subnormal_half", "if (y < 1.0) return sign | 0x1;", "if (y < 1.0) return sign;",
+     [t_codecs.test_e2m1_bruteforce_dense, _all_golden_points]),
+    ("fp16_exponent_bias", "return sign | (uint16_t)((E + 15) << 10) | mant;",
+     "return sign | (uint16_t)((E + 14) << 10) | mant;", [t_codecs.test_fp16_against_numpy]),
+    ("fp16_max_is_overflow", "if (y > 65504.0 || isinf(y)) return sign | 0x7C00;",
+     "if (y >= 65504.0 || isinf(y)) return sign | 0x7C00;", [t_codecs.test_fp16_against_numpy, _all_golden_points]),
+    ("inverse_lambda_of_the_rounded_lambda", "inv_lambda_f[j] = (float)(1.0 / lam);",
+     "inv_lambda_f[j] = 1.0f / (float)lam;", [t_method.test_smoothing_closed_forms]),
+    ("int4_group_max_of_signed_values", "for (int i = 0; i < 64; ++i) { float a = fabsf(x[i]);",
+     "for (int i = 0; i < 64; ++i) { float a = x[i];", [t_method.test_int4_error_bound_and_zero_group]),
+    ("int4_rounds_toward_zero", "double r = nearbyint((double)p);", "double r = trunc((double)p);",
+     [t_method.test_int4_error_bound_and_zero_group]),
+    ("int4_scale_not_rounded_to_fp16", "float S = orc_f16_to_f32(s);", "float S = q7;",
+     [t_method.test_int4_error_bound_and_zero_group, t_method.test_int4_subnormal_scales_saturate_codes]),
+    ("nvfp4_block_max_of_signed_values", "for (int i = 0; i < 16; ++i) { float a = fabsf(x[i]);",
+     "for (int i = 0; i < 16; ++i) { float a = x[i];", [t_method.test_nvfp4_error_bound]),
+    ("nvfp4_zero_scale_block_quantized", "if (sb != 0) {\n          volatile float inv = 1.0f / d;",
+     "{\n          volatile float inv = 1.0f / d;", [t_method.test_nvfp4_zero_scale_blocks_have_zero_codes]),
+    ("nvfp4_dequant_without_tensor_scale",
+     "double d = (double)orc_e4m3_to_f32(scales[m * B + k / 16]) * (double)g;",
+     "double d = (double)orc_e4m3_to_f32(scales[m * B + k / 16]);", [t_method.test_nvfp4_roundtrip_on_grid]),
+    ("t_rounded_through_binary32", "t[m * r + j] = orc_f64_to_bf16(acc[j]);",
+     "t[m * r + j] = orc_f32_to_bf16((float)acc[j]);", [t_method.test_lowrank_down_rounds_once]),
+    ("output_rounded_through_binary32", "y_bf16[m * N + n] = orc_f64_to_bf16(y);",
+     "y_bf16[m * N + n] = orc_f32_to_bf16((float)y);", [t_method.test_output_rounds_once_from_binary64]),
 ]
 
 
@@ -171,8 +197,42 @@ def _awq_scales_exponent_swapped(mean_abs, alpha):
     return _REAL["awq_channel_scales"](mean_abs, 1.0 - alpha)
 
 
+def _awq_statistic_max(X_bf16):
+    return np.abs(oracle.bf16_to_f32(X_bf16).astype(np.float64)).max(axis=0)
+
+
+def _quantize_act_t_from_unsmoothed_x(X_bf16, prep):
+    act = _REAL["quantize_act"](X_bf16, prep)
+    act["t"] = oracle.lowrank_down(oracle.bf16_to_f32(X_bf16), prep["L1"])
+    return act
+
+
+def _prepare_g_w_from_smoothed_weight(W_bf16, bias_bf16, amax_x, alpha, rank, fmt, svd=None):
+    out = _REAL["prepare"](W_bf16, bias_bf16, amax_x, alpha, rank, fmt, svd)
+    if oracle._FMT[fmt] == oracle.NVFP4:
+        What, _ = oracle.smoothed_weight(W_bf16, amax_x, alpha)
+        out["g_w"] = oracle.pow2_scale(float(np.abs(What).max()))
+        out["wcodes"], out["wscales"] = oracle.quant_nvfp4(out["R"], out["g_w"])
+    return out
+
+
+def _prepare_static_g_x_unsmoothed(W_bf16, bias_bf16, amax_x, alpha, rank, fmt, svd=None):
+    out = _REAL["prepare"](W_bf16, bias_bf16, amax_x, alpha, rank, fmt, svd)
+    if oracle._FMT[fmt] == oracle.NVFP4:
+        out["g_x"] = oracle.pow2_scale(float(np.asarray(amax_x, np.float32).max()))
+    return out
+
+
+def _prepare_drops_bias(W_bf16, bias_bf16, amax_x, alpha, rank, fmt, svd=None):
+    return _REAL["prepare"](W_bf16, None, amax_x, alpha, rank, fmt, svd)
+
+
+def _calibration_mean(X_bf16):
+    return np.abs(oracle.bf16_to_f32(X_bf16)).mean(axis=0).astype(np.float32)
+
+
 _REAL = {n: getattr(oracle, n) for n in ("svd_lowrank_factors", "smoothed_weight", "prepare", "act_tensor_scale",
-                                         "awq_channel_scales")}
+                                         "awq_channel_scales", "quantize_act")}
 
 # (name, oracle attribute, its mistaken value, pins expected to catch it)
 PY_MUTANTS = [
@@ -189,6 +249,16 @@ PY_MUTANTS = [
     ("w8_step_max_over_126", "W8_QMAX", 126, [functools.partial(t_w8.test_w8_quantizer_properties, 0)]),
     ("awq_scale_exponent_swapped", "awq_channel_scales", _awq_scales_exponent_swapped,
      [t_awq.test_awq_unit_scale_is_plain_group_int4, t_awq.test_awq_exact_layer_equals_dense_product]),
+    ("awq_statistic_max_not_mean", "awq_mean_abs", _awq_statistic_max, [t_awq.test_awq_statistic_is_the_channel_mean]),
+    ("t_from_the_unsmoothed_input", "quantize_act", _quantize_act_t_from_unsmoothed_x,
+     [functools.partial(t_method.test_error_decreases_with_rank_and_full_rank_is_near_exact, "int4")]),
+    ("g_w_from_the_smoothed_weight_not_the_residual", "prepare", _prepare_g_w_from_smoothed_weight,
+     [t_method.test_tensor_scales_are_tight]),
+    ("static_g_x_without_the_smoothing", "prepare", _prepare_static_g_x_unsmoothed,
+     [t_method.test_tensor_scales_are_tight, t_dyn.test_dynamic_equals_static_calibrated_on_the_same_input]),
+    ("prepare_drops_the_bias", "prepare", _prepare_drops_bias, [t_method.test_prepare_residual_uses_rounded_factors]),
+    ("calibration_mean_not_max", "calib_absmax", _calibration_mean,
+     [t_dyn.test_dynamic_equals_static_calibrated_on_the_same_input]),
 ]
 
 
