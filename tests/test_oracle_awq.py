@@ -3,11 +3,15 @@ the definition and the mathematics fix, independently of the oracle's own code:
 exactly representable layers, a loop-level brute force from the nibble format,
 the unit-scale reduction to plain group-INT4, and the method's claim that the
 activation-aware scale protects the weights of outlier channels."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
 import oracle
 import workloads as wl
+from fp_exact import bf16 as bf16_exact
+from fp_exact import f32_of_bits, fl32
 
 bf = oracle.bf16_to_f32
 
@@ -63,6 +67,27 @@ def test_awq_statistic_is_the_channel_mean():
     Xw = np.tile(X, (1, 16))
     prep = oracle.awq_prepare(W, None, Xw, alphas=(1.0,))
     np.testing.assert_array_equal(prep["s"], np.tile(np.float32([2.0, 4.0, 1.0, 2.5 / 3]), 16))
+
+
+def test_awq_smoothed_input_is_binary32():
+    """The smoothed activation is one binary32 product fl32(x * inv_s) before the binary64
+    sum: with x = 3 and this inv_s, 3 * inv_s lies just above the bf16 tie 1.03515625 and
+    rounds onto it in binary32, so y = bf16(tie) = 1.03125 (the even neighbour, 0x3F84);
+    the unrounded product would give 1.0390625."""
+    inv = f32_of_bits(0x3EB0AAAB)
+    tie = fl32(3 * inv)
+    assert tie == 1 + Fraction(9, 256) and 3 * inv > tie
+    assert bf16_exact(tie) == Fraction(33, 32) and bf16_exact(3 * inv) == 1 + Fraction(5, 128)
+    K = 64
+    inv_s = np.ones(K, np.float32)
+    inv_s[0] = float(inv)
+    wcodes = np.zeros((1, K // 2), np.uint8)
+    wcodes[0, 0] = 0x01  # q = 1 at k = 0
+    prep = dict(N=1, K=K, inv_s=inv_s, wcodes=wcodes, wscales=np.array([[0x3C00]], np.uint16),
+                bias=np.zeros(1, np.uint16))
+    X = np.zeros((1, K), np.uint16)
+    X[0, 0] = 0x4040  # 3.0
+    assert oracle.awq_forward(X, prep)[0, 0] == 0x3F84
 
 
 def test_awq_forward_brute_force_tiny():

@@ -1,10 +1,13 @@
 """Pins for the oracle's method steps against closed forms, invariants, brute
 force and independent library routines (numpy matmul / eigvalsh)."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
 import oracle
 import workloads as wl
+from fp_exact import fl32
 
 
 def _bf(x):
@@ -177,6 +180,38 @@ def test_nvfp4_zero_scale_blocks_have_zero_codes():
     for r, blk in zero_blocks:
         assert scales[r, blk] == 0
         assert not codes[r, 8 * blk:8 * blk + 8].any(), (r, blk)
+
+
+def test_int4_code_uses_the_binary32_reciprocal():
+    """Worked example of the INT4 reading code = rne(fl32(x * fl32(1/S))): with S = fp16
+    0x3D25 = 1317/1024 and x = 3.5 S exactly, the exact quotient is the tie 3.5 (a
+    division would round it to 4), while the binary32 reciprocal puts the product just
+    below the tie: code 3."""
+    S = Fraction(1317, 1024)
+    x = Fraction(7, 2) * S
+    p = fl32(x * fl32(1 / S))
+    assert p < Fraction(7, 2) and round(p) == 3 and round(x / S) == 4
+    v = np.zeros((1, 64), np.float32)
+    v[0, 0], v[0, 1] = float(7 * S), float(x)  # the group's amax makes fp16(amax / 7) = S exactly
+    codes, scales = oracle.quant_int4(v)
+    assert oracle.f16_to_f32(scales)[0, 0] == float(S)
+    q = _unpack_int4(codes)
+    assert q[0, 0] == 7 and q[0, 1] == 3
+
+
+def test_nvfp4_code_uses_the_binary32_reciprocal():
+    """Worked example of the NVFP4 reading code = e2m1_rne(fl32(x * fl32(1/d))): with the
+    block scale d = 1.875 (E4M3 0x3F, g = 1) and x = 1.25 d, the exact quotient is the
+    tie 1.25 between 1 and 1.5 (a division would round to the even neighbour 1), while
+    the binary32 reciprocal lands just above it: 1.5, code 0x3."""
+    d = Fraction(15, 8)
+    x = Fraction(5, 4) * d
+    assert fl32(x * fl32(1 / d)) > Fraction(5, 4)
+    v = np.zeros((1, 16), np.float32)
+    v[0, 0], v[0, 1] = float(6 * d), float(x)  # amax / 6 = d exactly
+    codes, scales = oracle.quant_nvfp4(v, 1.0)
+    assert scales[0, 0] == 0x3F
+    assert codes[0, 0] & 0xF == 0x7 and codes[0, 0] >> 4 == 0x3  # 6 and 1.5 (E2M1: sign, 2 exponent bits, 1 mantissa bit)
 
 
 def test_tensor_scales_are_tight():

@@ -118,6 +118,10 @@ C_MUTANTS = [
      "t[m * r + j] = orc_f32_to_bf16((float)acc[j]);", [t_method.test_lowrank_down_rounds_once]),
     ("output_rounded_through_binary32", "y_bf16[m * N + n] = orc_f64_to_bf16(y);",
      "y_bf16[m * N + n] = orc_f32_to_bf16((float)y);", [t_method.test_output_rounds_once_from_binary64]),
+    ("int4_divides_instead_of_the_reciprocal", "volatile float p = x[i + h] * inv;\n            double r",
+     "volatile float p = x[i + h] / S;\n            double r", [t_method.test_int4_code_uses_the_binary32_reciprocal]),
+    ("nvfp4_divides_instead_of_the_reciprocal", "volatile float p = x[i + h] * inv;\n            c[h]",
+     "volatile float p = x[i + h] / d;\n            c[h]", [t_method.test_nvfp4_code_uses_the_binary32_reciprocal]),
 ]
 
 
@@ -231,6 +235,37 @@ def _calibration_mean(X_bf16):
     return np.abs(oracle.bf16_to_f32(X_bf16)).mean(axis=0).astype(np.float32)
 
 
+def _w8_ties_away(v, s):
+    v = np.asarray(v, np.float32)
+    if s == 0:
+        return np.zeros(v.shape, np.int8)
+    p = (v * np.float32(np.float32(1.0) / np.float32(s))).astype(np.float64)
+    return np.clip(np.sign(p) * np.floor(np.abs(p) + 0.5), -127, 127).astype(np.int8)
+
+
+def _w8_divides(v, s):
+    v = np.asarray(v, np.float32)
+    if s == 0:
+        return np.zeros(v.shape, np.int8)
+    return np.clip(np.rint((v / np.float32(s)).astype(np.float32)), -127, 127).astype(np.int8)
+
+
+def _w8a8_output_in_binary32(act, prep, want_f64=False):
+    acc = act["codes"].astype(np.int64) @ prep["wcodes"].astype(np.int64).T
+    yd = (np.float32(act["s_x"]) * np.float32(prep["s_w"]) * acc.astype(np.float32) +
+          oracle.bf16_to_f32(prep["bias"])[None, :]).astype(np.float64)
+    y = oracle.f64_to_bf16(np.ascontiguousarray(yd))
+    return (y, yd) if want_f64 else y
+
+
+def _awq_smoothed_input_in_binary64(X_bf16, prep, want_f64=False):
+    xhat = oracle.bf16_to_f32(X_bf16).astype(np.float64) * prep["inv_s"].astype(np.float64)
+    yd = xhat @ oracle.dequant(prep["wcodes"], prep["wscales"], oracle.INT4).T + \
+        oracle.bf16_to_f32(prep["bias"]).astype(np.float64)[None, :]
+    y = oracle.f64_to_bf16(np.ascontiguousarray(yd))
+    return (y, yd) if want_f64 else y
+
+
 _REAL = {n: getattr(oracle, n) for n in ("svd_lowrank_factors", "smoothed_weight", "prepare", "act_tensor_scale",
                                          "awq_channel_scales", "quantize_act")}
 
@@ -259,6 +294,13 @@ PY_MUTANTS = [
     ("prepare_drops_the_bias", "prepare", _prepare_drops_bias, [t_method.test_prepare_residual_uses_rounded_factors]),
     ("calibration_mean_not_max", "calib_absmax", _calibration_mean,
      [t_dyn.test_dynamic_equals_static_calibrated_on_the_same_input]),
+    ("w8_ties_away_from_zero", "quant_w8", _w8_ties_away, [t_w8.test_w8_ties_round_to_even]),
+    ("w8_divides_instead_of_the_reciprocal", "quant_w8", _w8_divides,
+     [t_w8.test_w8_code_uses_the_binary32_reciprocal]),
+    ("w8a8_output_in_binary32", "w8a8_forward_from_act", _w8a8_output_in_binary32,
+     [t_w8.test_w8a8_output_rounds_once]),
+    ("awq_smoothed_input_in_binary64", "awq_forward", _awq_smoothed_input_in_binary64,
+     [t_awq.test_awq_smoothed_input_is_binary32]),
 ]
 
 

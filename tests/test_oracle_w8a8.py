@@ -3,11 +3,14 @@ plain arithmetic: a layer built so that every step is exact equals the dense
 product; a loop-level brute force in Python integers; the quantizer's error is
 at most half a step, it is odd-symmetric and maps +-max|v| to +-127; an all-zero
 input gives codes 0 and y = bias."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
 import oracle
 import workloads as wl
+from fp_exact import f32_of_bits, fl32
 
 bf = oracle.bf16_to_f32
 
@@ -65,6 +68,43 @@ def test_w8_quantizer_properties(seed):
     assert abs(int(q[i])) == 127
     err = np.abs(q.astype(np.float64) * float(s) - v.astype(np.float64))
     assert np.all(err <= 0.5 * float(s) * (1 + 2.0 ** -20))  # half a step (the reciprocal is rounded)
+
+
+def test_w8_code_uses_the_binary32_reciprocal():
+    """Worked example of the reading q = rne(fl32(v * fl32(1/s))), s = fl32(max|v| / 127):
+    for these two binary32 values the exact quotient v / s is -110.500004..., which a
+    division would round to -111; the binary32 reciprocal gives -110."""
+    amax, v = f32_of_bits(0x3FBA4BF1), f32_of_bits(0xBFA217BF)
+    s = fl32(amax / 127)
+    assert round(fl32(v * fl32(1 / s))) == -110 and round(v / s) == -111
+    x = np.array([[float(amax), float(v)]], np.float32)
+    assert Fraction(float(oracle.w8_tensor_scale(x))) == s
+    q = oracle.quant_w8(x, oracle.w8_tensor_scale(x))
+    assert q[0, 0] == 127 and q[0, 1] == -110
+
+
+def test_w8_ties_round_to_even():
+    """With s = 2^-3 every value (k + 1/2) / 8 is an exact tie; the codes take the even
+    neighbour (0.5 -> 0, 1.5 -> 2, -2.5 -> -2, ...)."""
+    k = np.arange(-127, 126)
+    x = np.concatenate([[127 / 8.0], (k + 0.5) / 8.0]).astype(np.float32)[None, :]
+    s = oracle.w8_tensor_scale(x)
+    assert s == np.float32(0.125)
+    q = oracle.quant_w8(x, s)[0, 1:]
+    want = [round(Fraction(int(j)) + Fraction(1, 2)) for j in k]
+    np.testing.assert_array_equal(q, want)
+
+
+def test_w8a8_output_rounds_once():
+    """y is formed in binary64 and rounded once: with unit scales and an integer product
+    of 2^24 + 2^16 + 1 (above the bf16 tie at 2^24 + 2^16), y rounds up to 2^24 + 2^17
+    (0x4B81); a binary32 detour would land on the tie and give 2^24."""
+    qx = np.array([127] * 1044 + [127, 13], np.int8)
+    qw = np.array([127] * 1044 + [32, 1], np.int8)
+    assert int(qx.astype(np.int64) @ qw.astype(np.int64)) == 2**24 + 2**16 + 1
+    act = dict(codes=qx[None, :], s_x=np.float32(1.0))
+    prep = dict(wcodes=qw[None, :], s_w=np.float32(1.0), bias=np.zeros(1, np.uint16))
+    assert oracle.w8a8_forward_from_act(act, prep)[0, 0] == 0x4B81
 
 
 def test_w8a8_zero_input_gives_bias():
