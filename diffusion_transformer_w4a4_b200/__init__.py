@@ -333,6 +333,25 @@ def svdq_set_wait_limit(cycles: int) -> None:
 
 
 # ----------------------------------------------------------------------------- convenience
+def _layer_device(device):
+    """The CUDA device a layer lives on, always with its index."""
+    import torch
+
+    d = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if d.type != "cuda":
+        raise ValueError(f"a layer lives on a CUDA device, not {d}")
+    return d if d.index is not None else torch.device("cuda", torch.cuda.current_device())
+
+
+def _check_input(x, K: int, device):
+    import torch
+
+    if not (x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == K):
+        raise ValueError(f"expected a contiguous bf16 CUDA tensor [..., {K}], got {x.dtype} {tuple(x.shape)}")
+    if x.device != device:
+        raise ValueError(f"input on {x.device}, layer on {device}")
+
+
 class SvdqLinear:
     """One svdq_w4a4 layer resident on `device` (default: the current CUDA device).
 
@@ -348,7 +367,7 @@ class SvdqLinear:
         self.N, self.K, self.rank = int(canonical["N"]), int(canonical["K"]), int(canonical["rank"])
         self.fmt = _fmt(canonical["fmt"])
         self.g_x, self.g_w = float(canonical.get("g_x", 1.0)), float(canonical.get("g_w", 1.0))
-        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = _layer_device(device)
         blob = svdq_pack(canonical)
         self.blob = torch.from_numpy(blob).to(self.device)
         with torch.cuda.device(self.device):
@@ -370,7 +389,7 @@ class SvdqLinear:
     def forward(self, x, out=None, stream=None):
         import torch
 
-        assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
+        _check_input(x, self.K, self.device)
         M = x.numel() // self.K
         y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         ws = self.workspace(M)
@@ -475,7 +494,7 @@ class AwqLinear:
         import torch
 
         self.N, self.K = int(canonical["N"]), int(canonical["K"])
-        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = _layer_device(device)
         self.blob = torch.from_numpy(svdq_awq_pack(canonical)).to(self.device)
         with torch.cuda.device(self.device):
             self.handle = svdq_awq_layer_create(self.blob, self.blob.numel(), self.N, self.K)
@@ -483,7 +502,7 @@ class AwqLinear:
     def forward(self, x, out=None, stream=None):
         import torch
 
-        assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
+        _check_input(x, self.K, self.device)
         M = x.numel() // self.K
         y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         with torch.cuda.device(self.device):
@@ -578,7 +597,7 @@ class W8A8Linear:
 
         self.N, self.K = int(wcodes.shape[0]), int(wcodes.shape[1])
         self.s_w = float(s_w)
-        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.device = _layer_device(device)
         self.blob = torch.from_numpy(svdq_w8a8_pack(wcodes, bias)).to(self.device)
         with torch.cuda.device(self.device):
             self.handle = svdq_w8a8_layer_create(self.blob, self.blob.numel(), self.N, self.K, self.s_w)
@@ -611,7 +630,7 @@ class W8A8Linear:
     def forward(self, x, out=None, stream=None):
         import torch
 
-        assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous() and x.shape[-1] == self.K
+        _check_input(x, self.K, self.device)
         M = x.numel() // self.K
         y = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         ws = self.workspace(M)
