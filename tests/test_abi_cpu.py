@@ -142,6 +142,34 @@ def test_product_prepare_agrees_with_oracle(lib, fmt):
     np.testing.assert_array_equal(ours["bias"], b)
 
 
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+def test_product_prepare_degenerate_inputs(lib, fmt):
+    """A zero weight channel and a zero activation channel get lambda = 1; an all-zero
+    weight gives a zero branch, zero codes and scales and g_w = 1 (nothing non-finite);
+    at full rank the branch reconstructs the smoothed weight as well as the oracle's."""
+    bf = lambda h: oracle.bf16_to_f32(h).astype(np.float64)
+    X, W, b = wl.make_layer_inputs(wl.small_layer(64, 256, 128, 16, fmt))
+    W = W.copy()
+    W[:, 7] = 0
+    amax = oracle.calib_absmax(X).copy()
+    amax[11] = 0.0
+    ours = svdq.svdq_prepare(W, b, amax, 0.5, 16, fmt)
+    assert ours["lambda_"][7] == 1.0 and ours["lambda_"][11] == 1.0
+    assert ours["inv_lambda"][7] == 1.0 and ours["inv_lambda"][11] == 1.0
+    zero = svdq.svdq_prepare(np.zeros_like(W), None, amax, 0.5, 16, fmt)
+    assert np.isfinite(bf(zero["L1"])).all() and np.isfinite(bf(zero["L2"])).all()
+    assert not (bf(zero["L1"]) @ bf(zero["L2"])).any()
+    assert not zero["wcodes"].any() and not np.asarray(zero["wscales"]).any()
+    assert zero["g_w"] == 1.0
+    X, W, b = wl.make_layer_inputs(wl.small_layer(64, 256, 128, 128, fmt))
+    amax = oracle.calib_absmax(X)
+    full = svdq.svdq_prepare(W, b, amax, 0.5, 128, fmt)
+    ref = oracle.prepare(W, b, amax, 0.5, 128, fmt)
+    What = bf(W) * ref["lam"].astype(np.float64)[None, :]
+    err = lambda c: np.linalg.norm(What - (bf(c["L1"]) @ bf(c["L2"])).T) / np.linalg.norm(What)
+    assert err(full) <= 1.01 * err(ref) + 1e-12 and err(ref) < 0.01
+
+
 def test_product_codecs_match_oracle_via_prepare_rank0(lib):
     # rank 0 and alpha 0: the residual is W * lambda exactly, so the weight codes
     # and scales come from identical binary32 inputs on both sides and must be
