@@ -170,6 +170,32 @@ def test_product_prepare_degenerate_inputs(lib, fmt):
     assert err(full) <= 1.01 * err(ref) + 1e-12 and err(ref) < 0.01
 
 
+def test_product_svd_on_adversarial_spectra(lib):
+    """The product's truncated SVD (randomized subspace iteration) on the two spectra
+    that are hardest for it: a weight of exact rank 8 at r = 16 must be reconstructed
+    as well as by the oracle's full SVD (only bf16 rounding of the factors remains),
+    and a flat spectrum (no gap, slowest convergence) must still come within 1 % of
+    the Eckart-Young optimum."""
+    bf = lambda h: oracle.bf16_to_f32(h).astype(np.float64)
+    rng = np.random.default_rng(0)
+    N, K = 192, 256
+    amax = (np.abs(rng.standard_normal(K)) + 0.5).astype(np.float32)
+    W = wl.f32_to_bf16_bits((rng.standard_normal((N, 8)) @ rng.standard_normal((8, K)) * 0.01).astype(np.float32))
+    ours = svdq.svdq_prepare(W, None, amax, 0.5, 16, "int4")
+    ref = oracle.prepare(W, None, amax, 0.5, 16, "int4")
+    What = bf(W) * ref["lam"].astype(np.float64)[None, :]
+    err = lambda c: np.linalg.norm(What - (bf(c["L1"]) @ bf(c["L2"])).T) / np.linalg.norm(What)
+    assert err(ours) <= 1.01 * err(ref) and err(ref) < 0.01
+    Q1, _ = np.linalg.qr(rng.standard_normal((N, N)))
+    Q2, _ = np.linalg.qr(rng.standard_normal((K, K)))
+    W = wl.f32_to_bf16_bits((Q1 @ np.diag(np.linspace(1.0, 0.98, N)) @ Q2[:, :N].T * 0.05).astype(np.float32))
+    ours = svdq.svdq_prepare(W, None, amax, 0.5, 32, "int4")
+    ref = oracle.prepare(W, None, amax, 0.5, 32, "int4")
+    What = bf(W) * ref["lam"].astype(np.float64)[None, :]
+    trunc = np.linalg.norm(What - (bf(ours["L1"]) @ bf(ours["L2"])).T) ** 2
+    assert trunc <= 1.01 * np.sum(ref["sing"][32:] ** 2)
+
+
 def test_product_codecs_match_oracle_via_prepare_rank0(lib):
     # rank 0 and alpha 0: the residual is W * lambda exactly, so the weight codes
     # and scales come from identical binary32 inputs on both sides and must be
