@@ -20,6 +20,10 @@ per-tensor NVFP4 activation scale (act_tensor_scale, selected by g_x = 0), and
 the INT8 tensorwise W8A8 layer the ainews.so section compares (w8a8_*), each
 pinned in its own tests/test_oracle_*.py, and the GELU between a block's MLP
 linears (gelu_bf16, for the fused MLP pair; pinned in test_oracle_gelu.py).
+
+The pins themselves are tested: tests/test_oracle_mutants.py plants plausible
+mistakes in copies of this oracle (compile_source / bind load a mutated copy of
+svdq_oracle.c; single Python steps are replaced) and requires a pin to catch each.
 """
 from __future__ import annotations
 
